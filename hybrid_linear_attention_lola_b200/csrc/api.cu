@@ -1,0 +1,407 @@
+// Host side of the C ABI declared in include/lola.h: argument checks, the
+// workspace layout, and the order in which one prefill call or decode step
+// enqueues its kernels on the caller's stream.
+#include <cstdio>
+#include <cstring>
+#include <new>
+
+#include "../../include/lola.h"
+#include "lola_internal.cuh"
+
+namespace lola {
+size_t chain_smem_bytes(const Dims &dm);
+size_t attn_smem_bytes(const Dims &dm);
+}
+
+struct lola_state {
+    lola_config cfg;
+    lola::Dims dm;
+    lola::DevState S;
+    lola::PrefillScratch P;
+    void *ws;
+    size_t ws_bytes;
+    long long pos;           // tokens processed per sequence
+    long long interval_end;  // end of the open decode interval (== pos when none is open)
+    long long t0_open;       // start of the open (or last) decode interval
+    int nS;                  // cache occupancy (identical for every stream)
+    long long pend_lo;       // leaving pairs of the last interval: [pend_lo, pend_lo + pend_n)
+    int pend_n;
+    long long n_int;         // update intervals run since init/reset
+    int32_t *sel_log;
+    long long sel_cap;
+    const int32_t *ovr;
+    long long ovr_n;
+};
+
+namespace {
+
+using lola::Dims;
+
+constexpr size_t kAlign = 256;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+lola_status derive_dims(const lola_config *c, Dims *dm)
+{
+    if (!c) return LOLA_ERR_INVALID_ARG;
+    if (c->dtype != LOLA_F32 && c->dtype != LOLA_BF16) return LOLA_ERR_DTYPE;
+    if (c->batch < 1 || c->n_kv_heads < 1 || c->n_q_heads < 1 || c->n_q_heads % c->n_kv_heads)
+        return LOLA_ERR_INVALID_ARG;
+    const int g = c->n_q_heads / c->n_kv_heads;
+    if (g > 8) return LOLA_ERR_INVALID_ARG;
+    if (c->head_dim != 32 && c->head_dim != 64 && c->head_dim != 128) return LOLA_ERR_INVALID_ARG;
+    if (c->feat_dim % 32 != 0 || c->feat_dim < 32 || c->feat_dim > 256) return LOLA_ERR_INVALID_ARG;
+    if (c->window < 0 || c->window > 65536) return LOLA_ERR_INVALID_ARG;
+    if (c->lambda_ < 0 || c->lambda_ > 4096) return LOLA_ERR_INVALID_ARG;
+    if (c->chunk < 1 || c->chunk > 256) return LOLA_ERR_INVALID_ARG;
+    if (c->decode_interval < 1 || c->decode_interval > 256 || c->decode_interval > c->window + 1)
+        return LOLA_ERR_INVALID_ARG;
+    if (!(c->eps >= 0.f)) return LOLA_ERR_INVALID_ARG;
+    const int nmax = c->max_prefill_tokens > 0 ? c->max_prefill_tokens : c->chunk;
+    if (nmax % c->chunk != 0) return LOLA_ERR_INVALID_ARG;
+    dm->B = c->batch;
+    dm->Hq = c->n_q_heads;
+    dm->Hkv = c->n_kv_heads;
+    dm->g = g;
+    dm->d = c->head_dim;
+    dm->D = c->feat_dim;
+    dm->Dh = c->feat_dim / 2;
+    dm->eta = c->window;
+    dm->lam = c->lambda_;
+    dm->C = c->chunk;
+    dm->Cdec = c->decode_interval;
+    dm->Lmax = c->chunk > c->decode_interval ? c->chunk : c->decode_interval;
+    dm->R = c->window + dm->Lmax + 1;
+    dm->ns = c->batch * c->n_kv_heads;
+    dm->dtype = c->dtype;
+    dm->Nmax = nmax;
+    dm->mmax = nmax / c->chunk;
+    dm->eps = c->eps;
+    const long long nkeys = (long long)dm->lam + dm->eta + dm->Cdec;
+    const long long tiles = (nkeys + 31) / 32;
+    long long ns = (296 + dm->ns - 1) / dm->ns;
+    if (ns > tiles) ns = tiles;
+    if (ns < 1) ns = 1;
+    dm->nsplit = (int)ns;
+    if (lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
+    if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
+    return LOLA_OK;
+}
+
+size_t elem_bytes(const Dims &dm) { return dm.dtype == LOLA_F32 ? 4 : 2; }
+
+// Carves the workspace; with base == nullptr only the size is computed.
+size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratch *P)
+{
+    size_t off = 0;
+    auto take = [&](size_t bytes) -> void * {
+        void *p = base ? base + off : nullptr;
+        off = align_up(off + bytes);
+        return p;
+    };
+    const size_t e = elem_bytes(dm);
+    const size_t ns = dm.ns;
+    lola::DevState s{};
+    s.err = (int *)take(16);
+    s.H = (float *)take(ns * dm.D * dm.d * 4);
+    s.s = (float *)take(ns * dm.D * 4);
+    s.KS = take(ns * dm.lam * dm.d * e);
+    s.VS = take(ns * dm.lam * dm.d * e);
+    s.idxS = (int *)take(ns * dm.lam * 4);
+    s.KR = take(ns * dm.R * dm.d * e);
+    s.VR = take(ns * dm.R * dm.d * e);
+    s.pend = (uint8_t *)take(ns * dm.Lmax);
+    s.W = (float *)take((size_t)dm.d * dm.Dh * 4);
+    s.phiV = (float *)take(ns * (dm.lam + dm.R) * dm.D * 4);
+    s.phiQd = (float *)take((size_t)dm.B * dm.Hq * dm.D * 4);
+    s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
+    lola::PrefillScratch p{};
+    const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
+    p.phiK = (float *)take(ns * nv * dm.D * 4);
+    p.phiQ = (float *)take((size_t)dm.B * dm.Nmax * dm.Hq * dm.D * 4);
+    p.snapH = (float *)take(ns * dm.mmax * dm.D * dm.d * 4);
+    p.snapS = (float *)take(ns * dm.mmax * dm.D * 4);
+    p.logTok = (int *)take(ns * dm.mmax * dm.lam * 4);
+    p.logVrow = (int *)take(ns * dm.mmax * dm.lam * 4);
+    p.logCount = (int *)take(ns * dm.mmax * 4);
+    p.logLf = (uint8_t *)take(ns * dm.mmax * dm.Lmax);
+    p.slotTok = (int *)take(ns * dm.lam * 4);
+    p.slotVrow = (int *)take(ns * dm.lam * 4);
+    if (S) *S = s;
+    if (P) *P = p;
+    return off;
+}
+
+lola_status check_launch()
+{
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) {
+        fprintf(stderr, "lola: CUDA error: %s\n", cudaGetErrorString(e));
+        return LOLA_ERR_CUDA;
+    }
+    return LOLA_OK;
+}
+
+bool aligned16(const void *p) { return ((uintptr_t)p & 15u) == 0; }
+
+void reset_host(lola_state *st)
+{
+    st->pos = 0;
+    st->interval_end = 0;
+    st->t0_open = 0;
+    st->nS = 0;
+    st->pend_lo = 0;
+    st->pend_n = 0;
+    st->n_int = 0;
+}
+
+// Host mirror of one interval's bookkeeping (identical for every stream).
+void advance_interval(lola_state *st, long long t0, int len)
+{
+    const long long t1 = t0 + len;
+    long long lo = t0 - st->dm.eta;
+    if (lo < 0) lo = 0;
+    long long hi = t1 - st->dm.eta;
+    if (hi < lo) hi = lo;
+    const int nL = (int)(hi - lo);
+    const int nQ = st->nS + nL;
+    st->nS = nQ < st->dm.lam ? nQ : st->dm.lam;
+    st->pend_lo = lo;
+    st->pend_n = nL;
+    st->n_int += 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *lola_status_string(lola_status s)
+{
+    switch (s) {
+    case LOLA_OK: return "ok";
+    case LOLA_ERR_INVALID_ARG: return "invalid argument";
+    case LOLA_ERR_SHAPE: return "bad shape (n_tokens must be a positive multiple of chunk)";
+    case LOLA_ERR_DTYPE: return "unsupported dtype";
+    case LOLA_ERR_STATE: return "call not allowed at the state's position";
+    case LOLA_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case LOLA_ERR_CUDA: return "CUDA error";
+    case LOLA_ERR_TIMEOUT: return "device wait timed out";
+    case LOLA_ERR_DEVICE: return "device-side check failed";
+    }
+    return "unknown status";
+}
+
+lola_status lola_state_bytes(const lola_config *cfg, size_t *device_bytes)
+{
+    if (!device_bytes) return LOLA_ERR_INVALID_ARG;
+    Dims dm;
+    const lola_status r = derive_dims(cfg, &dm);
+    if (r != LOLA_OK) return r;
+    *device_bytes = layout(dm, nullptr, nullptr, nullptr);
+    return LOLA_OK;
+}
+
+lola_status lola_state_stream_bytes(const lola_config *cfg, size_t *bytes)
+{
+    if (!bytes) return LOLA_ERR_INVALID_ARG;
+    Dims dm;
+    const lola_status r = derive_dims(cfg, &dm);
+    if (r != LOLA_OK) return r;
+    const size_t e = elem_bytes(dm);
+    *bytes = (size_t)dm.D * dm.d * 4 + (size_t)dm.D * 4 + 2 * (size_t)dm.lam * dm.d * e +
+             (size_t)dm.lam * 4 + 2 * (size_t)dm.R * dm.d * e + dm.Lmax;
+    return LOLA_OK;
+}
+
+lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspace,
+                            size_t workspace_bytes, void *cuda_stream, lola_state **out)
+{
+    if (!cfg || !W || !workspace || !out) return LOLA_ERR_INVALID_ARG;
+    Dims dm;
+    lola_status r = derive_dims(cfg, &dm);
+    if (r != LOLA_OK) return r;
+    if (((uintptr_t)workspace & (kAlign - 1)) != 0) return LOLA_ERR_WORKSPACE;
+    const size_t need = layout(dm, nullptr, nullptr, nullptr);
+    if (workspace_bytes < need) return LOLA_ERR_WORKSPACE;
+    lola_state *st = new (std::nothrow) lola_state();
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    st->cfg = *cfg;
+    st->dm = dm;
+    st->ws = workspace;
+    st->ws_bytes = workspace_bytes;
+    layout(dm, (char *)workspace, &st->S, &st->P);
+    reset_host(st);
+    lola::launch_init_state(dm, st->S, W, (cudaStream_t)cuda_stream);
+    r = check_launch();
+    if (r != LOLA_OK) {
+        delete st;
+        return r;
+    }
+    *out = st;
+    return LOLA_OK;
+}
+
+lola_status lola_reset_state(lola_state *st, void *cuda_stream)
+{
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    reset_host(st);
+    lola::launch_init_state(st->dm, st->S, nullptr, (cudaStream_t)cuda_stream);
+    return check_launch();
+}
+
+int64_t lola_position(const lola_state *st) { return st ? st->pos : -1; }
+
+lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, const void *v,
+                               int64_t n_tokens, void *out, void *cuda_stream)
+{
+    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return LOLA_ERR_INVALID_ARG;
+    const Dims &dm = st->dm;
+    if (n_tokens <= 0 || n_tokens % dm.C != 0) return LOLA_ERR_SHAPE;
+    if (n_tokens > dm.Nmax) return LOLA_ERR_WORKSPACE;
+    if (st->pos != st->interval_end) return LOLA_ERR_STATE;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    const int n = (int)n_tokens;
+    const int m = n / dm.C;
+    const long long pos0 = st->pos;
+
+    lola::launch_phi_kv(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, 0, st->P.phiK, st->nS,
+                        stream);
+    lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
+
+    lola::ChainArgs ca{};
+    ca.mode = 0;
+    ca.pos0 = pos0;
+    ca.n_int = m;
+    ca.ilen = dm.C;
+    ca.call_start = pos0;
+    ca.n_call = n;
+    ca.kin = k;
+    ca.vin = v;
+    ca.nS0 = st->nS;
+    ca.pend_lo = st->pend_lo;
+    ca.pend_n = st->pend_n;
+    ca.iglob0 = st->n_int;
+    ca.phi = st->P.phiK;
+    ca.nvrows = dm.lam + dm.R + dm.Nmax;
+    ca.sel_log = st->sel_log;
+    ca.sel_cap = st->sel_cap;
+    ca.ovr = st->ovr;
+    ca.ovr_n = st->ovr_n;
+    lola::launch_chain(dm, st->S, &st->P, ca, stream);
+
+    lola::AttnArgs aa{};
+    aa.pos0 = pos0;
+    aa.m = m;
+    aa.n_call = n;
+    aa.q = q;
+    aa.kin = k;
+    aa.vin = v;
+    aa.out = out;
+    lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+
+    for (int ci = 0; ci < m; ++ci) advance_interval(st, pos0 + (long long)ci * dm.C, dm.C);
+    lola::launch_finalize_prefill(dm, st->S, st->P, k, v, pos0, n, st->nS, stream);
+    st->pos = pos0 + n;
+    st->interval_end = st->pos;
+    return check_launch();
+}
+
+lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const void *v,
+                             void *out, void *cuda_stream)
+{
+    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return LOLA_ERR_INVALID_ARG;
+    const Dims &dm = st->dm;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    const long long pos = st->pos;
+    lola::launch_decode_append(dm, st->S, k, v, pos, stream);
+    if (pos == st->interval_end) {
+        lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
+        lola::ChainArgs ca{};
+        ca.mode = 1;
+        ca.pos0 = pos;
+        ca.n_int = 1;
+        ca.ilen = dm.Cdec;
+        ca.call_start = 0;
+        ca.n_call = 0;
+        ca.kin = nullptr;
+        ca.vin = nullptr;
+        ca.nS0 = st->nS;
+        ca.pend_lo = st->pend_lo;
+        ca.pend_n = st->pend_n;
+        ca.iglob0 = st->n_int;
+        ca.phi = st->S.phiV;
+        ca.nvrows = dm.lam + dm.R;
+        ca.sel_log = st->sel_log;
+        ca.sel_cap = st->sel_cap;
+        ca.ovr = st->ovr;
+        ca.ovr_n = st->ovr_n;
+        lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        advance_interval(st, pos, dm.Cdec);
+        st->t0_open = pos;
+        st->interval_end = pos + dm.Cdec;
+    }
+    lola::DecodeArgs da{};
+    da.pos = pos;
+    da.t0 = st->t0_open;
+    da.nS = st->nS;
+    da.L_lo = st->pend_lo;
+    da.L_hi = st->pend_lo + st->pend_n;
+    da.q = q;
+    da.k = k;
+    da.v = v;
+    da.out = out;
+    lola::launch_decode_attn(dm, st->S, da, stream);
+    st->pos = pos + 1;
+    return check_launch();
+}
+
+lola_status lola_get_cache_indices(const lola_state *st, int32_t *dev_idx, int32_t *dev_count,
+                                   void *cuda_stream)
+{
+    if (!st || !dev_idx) return LOLA_ERR_INVALID_ARG;
+    lola::launch_get_indices(st->dm, st->S, st->nS, dev_idx, dev_count, (cudaStream_t)cuda_stream);
+    return check_launch();
+}
+
+lola_status lola_set_selection_log(lola_state *st, int32_t *dev_buf, int64_t capacity)
+{
+    if (!st || capacity < 0) return LOLA_ERR_INVALID_ARG;
+    st->sel_log = dev_buf;
+    st->sel_cap = dev_buf ? capacity : 0;
+    return LOLA_OK;
+}
+
+lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept, int64_t n_intervals)
+{
+    if (!st || n_intervals < 0) return LOLA_ERR_INVALID_ARG;
+    st->ovr = dev_kept;
+    st->ovr_n = dev_kept ? n_intervals : 0;
+    return LOLA_OK;
+}
+
+lola_status lola_sync(lola_state *st, void *cuda_stream)
+{
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return check_launch();
+    int err[4] = {0, 0, 0, 0};
+    if (cudaMemcpy(err, st->S.err, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return check_launch();
+    if (err[0] != 0) {
+        cudaMemset(st->S.err, 0, sizeof(err));
+        return (err[0] & lola::ERR_TIMEOUT) ? LOLA_ERR_TIMEOUT : LOLA_ERR_DEVICE;
+    }
+    return LOLA_OK;
+}
+
+lola_status lola_free_state(lola_state *st)
+{
+    delete st;
+    return LOLA_OK;
+}
+
+}  // extern "C"

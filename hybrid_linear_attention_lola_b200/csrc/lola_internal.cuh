@@ -1,0 +1,181 @@
+// Internal definitions shared by the LoLA CUDA kernels (sm_100a).
+//
+// One "stream" is one (batch, kv-head) pair; every piece of state is per
+// stream and read by the n_q_heads / n_kv_heads query heads of its group.
+//
+// Virtual rows. Keys and values that a prefill call touches live in three
+// places: the state's sparse-cache slots, the state's window ring, and the
+// caller's k/v buffers. The kernels address them through one row index per
+// stream:  [0, lam)            cache slot i
+//          [lam, lam + R)      ring slot (token mod R)
+//          [lam + R, lam+R+n)  token call_start + (row - lam - R) of the call
+// phi(k) scratch is laid out over the same rows.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace lola {
+
+enum : int { ERR_BOUNDS = 1, ERR_TIMEOUT = 2 };
+
+struct Dims {
+    int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
+    int Nmax, mmax;   // prefill scratch capacity: tokens per call, intervals per call
+    int nsplit;       // decode key splits per stream
+    float eps;
+};
+
+// Persistent state (device pointers into the caller's workspace).
+struct DevState {
+    float *H;          // [ns][D][d]   fp32 linear-attention state
+    float *s;          // [ns][D]      fp32 normaliser
+    void *KS, *VS;     // [ns][lam][d] sparse-cache keys / values (dtype)
+    int *idxS;         // [ns][lam]    token index per cache slot, -1 = empty
+    void *KR, *VR;     // [ns][R][d]   window ring (slot = token mod R)
+    uint8_t *pend;     // [ns][Lmax]   1 = leaving pair of the last interval that is folded
+    float *W;          // [d][Dh]      feature-map matrix, fp32 copy
+    int *err;          // [4]          device error words
+    // decode scratch
+    float *phiV;       // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
+    float *phiQd;      // [B][Hq][D]
+    float *part;       // [ns][nsplit][g][2d + 4] split partials
+};
+
+// Per-prefill-call scratch.
+struct PrefillScratch {
+    float *phiK;       // [ns][lam + R + Nmax][D]
+    float *phiQ;       // [B][Nmax][Hq][D]
+    float *snapH;      // [ns][mmax][D][d]  H' of each interval (after the cache eviction fold)
+    float *snapS;      // [ns][mmax][D]
+    int *logTok;       // [ns][mmax][lam]   kept set of each interval (token)
+    int *logVrow;      // [ns][mmax][lam]   kept set of each interval (virtual row)
+    int *logCount;     // [ns][mmax]
+    uint8_t *logLf;    // [ns][mmax][Cmax]  leaving-pair fate per interval, 1 = folded
+    int *slotTok;      // [ns][lam]         slot contents at the end of the call
+    int *slotVrow;     // [ns][lam]
+};
+
+template <typename T> __device__ __forceinline__ float to_f(T x);
+template <> __device__ __forceinline__ float to_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 x)
+{
+    return __bfloat162float(x);
+}
+template <typename T> __device__ __forceinline__ T from_f(float x);
+template <> __device__ __forceinline__ float from_f<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float x)
+{
+    return __float2bfloat16_rn(x);
+}
+
+// Key/value row addressing over virtual rows (see the file comment).
+template <typename T> struct KVSrc {
+    const T *KS, *VS;    // [ns][lam][d]
+    const T *KR, *VR;    // [ns][R][d]
+    const T *kin, *vin;  // [B][n][Hkv][d] (prefill call), may be null
+    int lam, R, n, Hkv, d;
+    long long call_start; // token index of call row 0
+
+    __device__ __forceinline__ const T *row(const T *cache, const T *ring, const T *in, int st,
+                                            int vrow) const
+    {
+        if (vrow < lam) return cache + ((size_t)st * lam + vrow) * d;
+        if (vrow < lam + R) return ring + ((size_t)st * R + (vrow - lam)) * d;
+        const int b = st / Hkv, hk = st % Hkv;
+        return in + (((size_t)b * n + (vrow - lam - R)) * Hkv + hk) * d;
+    }
+    __device__ __forceinline__ const T *krow(int st, int vrow) const { return row(KS, KR, kin, st, vrow); }
+    __device__ __forceinline__ const T *vrow(int st, int vrow) const { return row(VS, VR, vin, st, vrow); }
+    // virtual row of a window/call token (never a cache slot)
+    __device__ __forceinline__ int tok2vrow(long long tok) const
+    {
+        if (kin != nullptr && tok >= call_start) return lam + R + (int)(tok - call_start);
+        return lam + (int)(tok % R);
+    }
+};
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+__device__ __forceinline__ float warp_max(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+__device__ __forceinline__ float warp_min(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    return x;
+}
+
+__device__ __forceinline__ void raise_error(int *err, int code)
+{
+    if (err) atomicOr(err, code);
+}
+
+// ---- host launch wrappers (defined in the .cu files) ----
+void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream);
+void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long call_start,
+                   int n, int nvrows, int row_begin_call, float *phi_out, int nS,
+                   cudaStream_t stream);
+void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, float *phi_out,
+                  cudaStream_t stream);
+
+struct ChainArgs {
+    int mode;               // 0 = prefill call, 1 = decode interval
+    long long pos0;         // first token of the first interval
+    int n_int, ilen;        // intervals and their length
+    long long call_start;   // prefill: token of call row 0
+    int n_call;             // prefill: tokens in the call
+    const void *kin, *vin;  // prefill: call k/v
+    int nS0;                // cache occupancy before the first interval
+    long long pend_lo;      // pending leaving range of the previous interval
+    int pend_n;
+    long long iglob0;       // interval counter of the first interval
+    const float *phi;       // [ns][nvrows][D]
+    int nvrows;
+    int32_t *sel_log;       // test hook, may be null
+    long long sel_cap;
+    const int32_t *ovr;     // test hook, may be null
+    long long ovr_n;
+};
+void launch_chain(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
+                  cudaStream_t stream);
+
+struct AttnArgs {
+    long long pos0;         // first token of the call
+    int m;                  // chunks in the call
+    int n_call;
+    const void *q, *kin, *vin;
+    void *out;
+};
+void launch_attn_prefill(const Dims &dm, const DevState &S, const PrefillScratch &P,
+                         const AttnArgs &a, cudaStream_t stream);
+void launch_finalize_prefill(const Dims &dm, const DevState &S, const PrefillScratch &P,
+                             const void *kin, const void *vin, long long call_start, int n,
+                             int nK, cudaStream_t stream);
+
+struct DecodeArgs {
+    long long pos;          // token index of this step
+    long long t0;           // start of the open interval
+    int nS;                 // cache occupancy during the interval
+    long long L_lo;         // leaving range of the open interval [L_lo, L_hi)
+    long long L_hi;
+    const void *q, *k, *v;
+    void *out;
+};
+void launch_decode_append(const Dims &dm, const DevState &S, const void *k, const void *v,
+                          long long pos, cudaStream_t stream);
+void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a,
+                        cudaStream_t stream);
+void launch_get_indices(const Dims &dm, const DevState &S, int nS, int32_t *idx, int32_t *cnt,
+                        cudaStream_t stream);
+
+}  // namespace lola

@@ -1,0 +1,177 @@
+// Feature map phi(x) = [softmax(x W), softmax(-x W)] (the low-rank positive
+// feature map of LoLA's linear attention, gist.science technical summary,
+// "Probleemstelling"; the two-sided softmax form is this engine's fixed choice),
+// and state initialisation.
+#include "lola_internal.cuh"
+
+namespace lola {
+
+// One warp maps one row. W (fp32, [d][Dh]) sits in shared memory; lane l owns
+// features l, l + 32, ... The row max / min shift is exact in real arithmetic.
+template <typename T>
+__device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const float *__restrict__ Ws,
+                                             float *__restrict__ xs, int d, int Dh,
+                                             float *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    for (int a = lane; a < d; a += 32) xs[a] = to_f<T>(x[a]);
+    __syncwarp();
+    float z[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) z[u] = 0.f;
+    for (int a = 0; a < d; ++a) {
+        const float xa = xs[a];
+        const float *wr = Ws + (size_t)a * Dh;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = lane + 32 * u;
+            if (i < Dh) z[u] = fmaf(xa, wr[i], z[u]);
+        }
+    }
+    float zmax = -INFINITY, zmin = INFINITY;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (lane + 32 * u < Dh) {
+            zmax = fmaxf(zmax, z[u]);
+            zmin = fminf(zmin, z[u]);
+        }
+    }
+    zmax = warp_max(zmax);
+    zmin = warp_min(zmin);
+    float ep[4], en[4], sp = 0.f, sn = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const bool ok = lane + 32 * u < Dh;
+        ep[u] = ok ? __expf(z[u] - zmax) : 0.f;
+        en[u] = ok ? __expf(zmin - z[u]) : 0.f;
+        sp += ep[u];
+        sn += en[u];
+    }
+    sp = warp_sum(sp);
+    sn = warp_sum(sn);
+    const float rp = 1.f / sp, rn = 1.f / sn;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = lane + 32 * u;
+        if (i < Dh) {
+            out[i] = ep[u] * rp;
+            out[Dh + i] = en[u] * rn;
+        }
+    }
+    __syncwarp();
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, const float *__restrict__ W,
+                                                     int nS, int n, int nvrows,
+                                                     float *__restrict__ phi_out)
+{
+    extern __shared__ float sm[];
+    float *Ws = sm;                                   // [d][Dh]
+    float *xs = sm + dm.d * dm.Dh + (threadIdx.x >> 5) * dm.d;
+    for (int e = threadIdx.x; e < dm.d * dm.Dh; e += blockDim.x) Ws[e] = W[e];
+    __syncthreads();
+    const int per_stream = nS + dm.R + n;
+    const long long total = (long long)dm.ns * per_stream;
+    const int warps = blockDim.x >> 5;
+    for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < total;
+         r += (long long)gridDim.x * warps) {
+        const int st = (int)(r / per_stream);
+        const int i = (int)(r % per_stream);
+        const int vrow = i < nS ? i : dm.lam + (i - nS);
+        phi_row_warp<T>(src.krow(st, vrow), Ws, xs, dm.d, dm.Dh,
+                        phi_out + ((size_t)st * nvrows + vrow) * dm.D);
+    }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(256) phi_q_kernel(int d, int Dh, const float *__restrict__ W,
+                                                    const T *__restrict__ q, long long rows,
+                                                    float *__restrict__ phi_out)
+{
+    extern __shared__ float sm[];
+    float *Ws = sm;
+    float *xs = sm + d * Dh + (threadIdx.x >> 5) * d;
+    for (int e = threadIdx.x; e < d * Dh; e += blockDim.x) Ws[e] = W[e];
+    __syncthreads();
+    const int warps = blockDim.x >> 5;
+    for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < rows;
+         r += (long long)gridDim.x * warps)
+        phi_row_warp<T>(q + (size_t)r * d, Ws, xs, d, Dh, phi_out + (size_t)r * 2 * Dh);
+}
+
+static int grid_for(long long rows, int warps_per_block)
+{
+    long long g = (rows + warps_per_block - 1) / warps_per_block;
+    if (g > 148 * 16) g = 148 * 16;
+    return (int)(g < 1 ? 1 : g);
+}
+
+void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long call_start,
+                   int n, int nvrows, int /*row_begin_call*/, float *phi_out, int nS,
+                   cudaStream_t stream)
+{
+    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
+    const long long rows = (long long)dm.ns * (nS + dm.R + n);
+    const int grid = grid_for(rows, 8);
+    if (dm.dtype == 0) {
+        KVSrc<float> src{(const float *)S.KS, (const float *)S.VS, (const float *)S.KR,
+                         (const float *)S.VR, (const float *)kin, nullptr,
+                         dm.lam, dm.R, n, dm.Hkv, dm.d, call_start};
+        phi_kv_kernel<float><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows, phi_out);
+    } else {
+        KVSrc<__nv_bfloat16> src{(const __nv_bfloat16 *)S.KS, (const __nv_bfloat16 *)S.VS,
+                                 (const __nv_bfloat16 *)S.KR, (const __nv_bfloat16 *)S.VR,
+                                 (const __nv_bfloat16 *)kin, nullptr,
+                                 dm.lam, dm.R, n, dm.Hkv, dm.d, call_start};
+        phi_kv_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows,
+                                                                  phi_out);
+    }
+}
+
+void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, float *phi_out,
+                  cudaStream_t stream)
+{
+    const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
+    const int grid = grid_for(rows, 8);
+    if (dm.dtype == 0)
+        phi_q_kernel<float><<<grid, 256, smem, stream>>>(dm.d, dm.Dh, W, (const float *)q, rows,
+                                                         phi_out);
+    else
+        phi_q_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(
+            dm.d, dm.Dh, W, (const __nv_bfloat16 *)q, rows, phi_out);
+}
+
+// ---------------------------------------------------------------- init
+
+template <typename T>
+__global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
+{
+    const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    const long long nH = (long long)dm.ns * dm.D * dm.d;
+    for (long long e = tid; e < nH; e += stride) S.H[e] = 0.f;
+    for (long long e = tid; e < (long long)dm.ns * dm.D; e += stride) S.s[e] = 0.f;
+    for (long long e = tid; e < (long long)dm.ns * dm.lam; e += stride) S.idxS[e] = -1;
+    for (long long e = tid; e < (long long)dm.ns * dm.Lmax; e += stride) S.pend[e] = 0;
+    const long long nR = (long long)dm.ns * dm.R * dm.d;
+    T *KR = (T *)S.KR, *VR = (T *)S.VR;
+    for (long long e = tid; e < nR; e += stride) {
+        KR[e] = from_f<T>(0.f);
+        VR[e] = from_f<T>(0.f);
+    }
+    if (W != nullptr)
+        for (long long e = tid; e < (long long)dm.d * dm.Dh; e += stride) S.W[e] = to_f<T>(W[e]);
+    if (tid < 4) S.err[tid] = 0;
+}
+
+void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream)
+{
+    if (dm.dtype == 0)
+        init_state_kernel<float><<<148 * 4, 256, 0, stream>>>(dm, S, (const float *)W);
+    else
+        init_state_kernel<__nv_bfloat16><<<148 * 4, 256, 0, stream>>>(dm, S,
+                                                                      (const __nv_bfloat16 *)W);
+}
+
+}  // namespace lola

@@ -1,0 +1,258 @@
+"""Thin Python binding of the LoLA C ABI (include/lola.h).
+
+Argument marshalling only: every step of the inference path runs in the CUDA
+kernels of liblola.so. PyTorch provides device memory and the current stream.
+There is no CPU fallback: without the built library or a CUDA device the calls
+raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "liblola.so")
+HEADER = os.path.join(os.path.dirname(PKG), "include", "lola.h")
+
+LOLA_F32, LOLA_BF16 = 0, 1
+STATUS = {0: "LOLA_OK", 1: "LOLA_ERR_INVALID_ARG", 2: "LOLA_ERR_SHAPE", 3: "LOLA_ERR_DTYPE",
+          4: "LOLA_ERR_STATE", 5: "LOLA_ERR_WORKSPACE", 6: "LOLA_ERR_CUDA",
+          7: "LOLA_ERR_TIMEOUT", 8: "LOLA_ERR_DEVICE"}
+
+
+class LolaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)} ({_status_string(code)})")
+        self.code = code
+
+
+class lola_config(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("n_q_heads", ctypes.c_int32),
+                ("n_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("feat_dim", ctypes.c_int32), ("window", ctypes.c_int32),
+                ("lambda_", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("decode_interval", ctypes.c_int32), ("max_prefill_tokens", ctypes.c_int32),
+                ("eps", ctypes.c_float), ("dtype", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load_library() -> ctypes.CDLL:
+    """Loads liblola.so from the package directory (raises if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"liblola.so not built at {LIB_PATH}; run __graft_entry__.build()")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I32, I64, SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    C = ctypes.POINTER(lola_config)
+    sigs = {
+        "lola_state_bytes": (I32, [C, ctypes.POINTER(SZ)]),
+        "lola_state_stream_bytes": (I32, [C, ctypes.POINTER(SZ)]),
+        "lola_init_state": (I32, [C, P, P, SZ, P, ctypes.POINTER(P)]),
+        "lola_reset_state": (I32, [P, P]),
+        "lola_prefill_chunk": (I32, [P, P, P, P, I64, P, P]),
+        "lola_decode_step": (I32, [P, P, P, P, P, P]),
+        "lola_position": (I64, [P]),
+        "lola_get_cache_indices": (I32, [P, P, P, P]),
+        "lola_set_selection_log": (I32, [P, P, I64]),
+        "lola_set_selection_override": (I32, [P, P, I64]),
+        "lola_sync": (I32, [P, P]),
+        "lola_free_state": (I32, [P]),
+        "lola_status_string": (ctypes.c_char_p, [I32]),
+    }
+    for name, (res, args) in sigs.items():
+        f = getattr(lib, name)
+        f.restype, f.argtypes = res, args
+    _lib = lib
+    return lib
+
+
+def header_symbols() -> list:
+    """Function names declared in include/lola.h."""
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[\w\s\*]*?\b(lola_\w+)\s*\(", text, re.M)))
+
+
+def _status_string(code: int) -> str:
+    try:
+        return load_library().lola_status_string(code).decode()
+    except Exception:
+        return "?"
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise LolaError(code, what)
+
+
+def make_config(*, batch, n_q_heads, n_kv_heads, head_dim, feat_dim, window, lambda_, chunk,
+                decode_interval, max_prefill_tokens=0, eps=1e-6, dtype="bf16") -> lola_config:
+    return lola_config(batch, n_q_heads, n_kv_heads, head_dim, feat_dim, window, lambda_, chunk,
+                       decode_interval, max_prefill_tokens, eps,
+                       LOLA_F32 if dtype in ("f32", "float32") else LOLA_BF16)
+
+
+def config_from_workload(w, max_prefill_tokens: Optional[int] = None, **over) -> lola_config:
+    kw = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
+              head_dim=w.head_dim, feat_dim=w.feat_dim, window=w.window, lambda_=w.lambda_,
+              chunk=w.chunk, decode_interval=w.decode_interval,
+              max_prefill_tokens=max_prefill_tokens or w.seq_len, eps=w.eps, dtype=w.dtype)
+    kw.update(over)
+    return make_config(**kw)
+
+
+# ---- C-ABI entry points with the same names (pointer arguments are ints) ----
+
+def lola_state_bytes(cfg: lola_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().lola_state_bytes(ctypes.byref(cfg), ctypes.byref(n)), "lola_state_bytes")
+    return n.value
+
+
+def lola_state_stream_bytes(cfg: lola_config) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().lola_state_stream_bytes(ctypes.byref(cfg), ctypes.byref(n)),
+           "lola_state_stream_bytes")
+    return n.value
+
+
+def lola_init_state(cfg: lola_config, W: int, workspace: int, nbytes: int, stream: int) -> int:
+    h = ctypes.c_void_p(0)
+    _check(load_library().lola_init_state(ctypes.byref(cfg), W, workspace, nbytes, stream,
+                                          ctypes.byref(h)), "lola_init_state")
+    return h.value
+
+
+def lola_reset_state(h: int, stream: int):
+    _check(load_library().lola_reset_state(h, stream), "lola_reset_state")
+
+
+def lola_prefill_chunk(h: int, q: int, k: int, v: int, n_tokens: int, out: int, stream: int):
+    _check(load_library().lola_prefill_chunk(h, q, k, v, n_tokens, out, stream),
+           "lola_prefill_chunk")
+
+
+def lola_decode_step(h: int, q: int, k: int, v: int, out: int, stream: int):
+    _check(load_library().lola_decode_step(h, q, k, v, out, stream), "lola_decode_step")
+
+
+def lola_position(h: int) -> int:
+    return load_library().lola_position(h)
+
+
+def lola_get_cache_indices(h: int, idx: int, count: int, stream: int):
+    _check(load_library().lola_get_cache_indices(h, idx, count, stream), "lola_get_cache_indices")
+
+
+def lola_set_selection_log(h: int, buf: int, capacity: int):
+    _check(load_library().lola_set_selection_log(h, buf, capacity), "lola_set_selection_log")
+
+
+def lola_set_selection_override(h: int, buf: int, n_intervals: int):
+    _check(load_library().lola_set_selection_override(h, buf, n_intervals),
+           "lola_set_selection_override")
+
+
+def lola_sync(h: int, stream: int):
+    _check(load_library().lola_sync(h, stream), "lola_sync")
+
+
+def lola_free_state(h: int):
+    _check(load_library().lola_free_state(h), "lola_free_state")
+
+
+# ---- convenience wrapper over torch device memory ----
+
+class LolaState:
+    """Owns a device workspace (torch) and a state handle."""
+
+    def __init__(self, cfg: lola_config, W, device="cuda"):
+        import torch
+        self.torch = torch
+        if not torch.cuda.is_available():
+            raise RuntimeError("LolaState needs a CUDA device")
+        self.cfg = cfg
+        self.device = torch.device(device)
+        self.dtype = torch.float32 if cfg.dtype == LOLA_F32 else torch.bfloat16
+        self.nbytes = lola_state_bytes(cfg)
+        self.workspace = torch.empty(self.nbytes, dtype=torch.uint8, device=self.device)
+        self.W = self._dev(W)
+        self.handle = lola_init_state(cfg, self.W.data_ptr(), self.workspace.data_ptr(),
+                                      self.nbytes, self._stream())
+        self._keep = []
+
+    def _stream(self) -> int:
+        return self.torch.cuda.current_stream(self.device).cuda_stream
+
+    def _dev(self, x):
+        t = self.torch.as_tensor(x)
+        return t.to(device=self.device, dtype=self.dtype).contiguous()
+
+    @property
+    def streams(self) -> int:
+        return self.cfg.batch * self.cfg.n_kv_heads
+
+    def reset(self):
+        lola_reset_state(self.handle, self._stream())
+
+    def prefill(self, q, k, v, out=None):
+        q, k, v = self._dev(q), self._dev(k), self._dev(v)
+        n = q.shape[1]
+        if out is None:
+            out = self.torch.empty_like(q)
+        lola_prefill_chunk(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), n,
+                           out.data_ptr(), self._stream())
+        return out
+
+    def decode(self, q, k, v, out=None):
+        q, k, v = self._dev(q), self._dev(k), self._dev(v)
+        if out is None:
+            out = self.torch.empty_like(q)
+        lola_decode_step(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(),
+                         self._stream())
+        return out
+
+    @property
+    def position(self) -> int:
+        return lola_position(self.handle)
+
+    def cache_indices(self):
+        idx = self.torch.empty((self.cfg.batch, self.cfg.n_kv_heads, max(self.cfg.lambda_, 1)),
+                               dtype=self.torch.int32, device=self.device)
+        cnt = self.torch.empty((self.cfg.batch, self.cfg.n_kv_heads), dtype=self.torch.int32,
+                               device=self.device)
+        lola_get_cache_indices(self.handle, idx.data_ptr(), cnt.data_ptr(), self._stream())
+        return idx[..., : self.cfg.lambda_], cnt
+
+    def enable_selection_log(self, capacity: int):
+        buf = self.torch.full((capacity, self.streams, self.cfg.lambda_ + 1), -2,
+                              dtype=self.torch.int32, device=self.device)
+        lola_set_selection_log(self.handle, buf.data_ptr(), capacity)
+        self._keep.append(buf)
+        return buf
+
+    def set_selection_override(self, kept):
+        """kept: int32 [n_int, streams, lambda+1] (count, ascending ids, -1 pad)."""
+        buf = self.torch.as_tensor(kept, dtype=self.torch.int32).to(self.device).contiguous()
+        lola_set_selection_override(self.handle, buf.data_ptr(), buf.shape[0])
+        self._keep.append(buf)
+        return buf
+
+    def sync(self):
+        lola_sync(self.handle, self._stream())
+
+    def close(self):
+        if getattr(self, "handle", None):
+            lola_free_state(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass

@@ -1,0 +1,152 @@
+/*
+ * lola.h -- C ABI of the B200 (sm_100a) LoLA hybrid-attention inference engine.
+ *
+ * LoLA (Low-Rank Linear Attention with Sparse Caching, arXiv 2505.23666) splits
+ * the past key/value pairs of each (batch, kv-head) stream over three memories
+ * (gist.science technical summary, section "Methodologie"):
+ *   - a sliding window of the `window` most recent pairs, attended by softmax;
+ *   - a sparse global cache of at most `lambda_` pairs, attended by softmax;
+ *   - the linear-attention state H (feat_dim x head_dim) and s (feat_dim),
+ *     holding every other pair folded in as H += phi(k) v^T, s += phi(k).
+ * At each update interval ("Inferentiestrategie" section) the pairs leaving the
+ * window and the pairs already cached are scored by the Self-Recall Error
+ * SRE(k,v|H,s) = || phi(k)^T H / (phi(k)^T s + eps) - v ||^2 (section
+ * "Het Self-Recall Error (SRE) Mechanisme"), the lambda_ highest stay cached
+ * (ties: the lower token index stays), the rest are folded, and each query's
+ * output combines softmax over window and cache with the linear readout of the
+ * state under one shared normaliser. The feature map is
+ * phi(x) = [softmax(x W), softmax(-x W)] with W of shape head_dim x feat_dim/2.
+ *
+ * Conventions for every entry point:
+ *   - Tensors are caller-owned DEVICE pointers, contiguous, 16-byte aligned,
+ *     in the state's dtype (float32 or bfloat16), token-major per batch:
+ *       q, out: [batch][n_tokens][n_q_heads][head_dim]
+ *       k, v:   [batch][n_tokens][n_kv_heads][head_dim]
+ *     Query head h reads kv-head h / (n_q_heads / n_kv_heads) (grouped queries).
+ *   - The library allocates no device memory. The caller allocates
+ *     lola_state_bytes() bytes of device memory (the "workspace") and passes it
+ *     to lola_init_state(); it holds the persistent state and all scratch.
+ *   - Work is enqueued on the caller's CUDA stream (`cuda_stream` is a
+ *     cudaStream_t; NULL = the legacy default stream). Calls return once the
+ *     work is enqueued; results are ready when the stream reaches them.
+ *   - Host-side argument checks return a status synchronously and enqueue
+ *     nothing. Errors raised on the device (bounds checks) are recorded in an
+ *     error word inside the workspace and reported by lola_sync().
+ *   - A state handle is not thread-safe: one host thread at a time per handle.
+ */
+#ifndef LOLA_H
+#define LOLA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    LOLA_OK = 0,
+    LOLA_ERR_INVALID_ARG = 1, /* null pointer, unsupported size, bad config value */
+    LOLA_ERR_SHAPE = 2,       /* n_tokens not a positive multiple of chunk */
+    LOLA_ERR_DTYPE = 3,       /* dtype not LOLA_F32 / LOLA_BF16 */
+    LOLA_ERR_STATE = 4,       /* call not allowed in the state's current position */
+    LOLA_ERR_WORKSPACE = 5,   /* workspace too small, misaligned, or n_tokens > max_prefill_tokens */
+    LOLA_ERR_CUDA = 6,        /* a CUDA launch or query failed */
+    LOLA_ERR_TIMEOUT = 7,     /* a bounded device wait gave up */
+    LOLA_ERR_DEVICE = 8       /* a device-side bounds check fired (see lola_sync) */
+} lola_status;
+
+typedef enum { LOLA_F32 = 0, LOLA_BF16 = 1 } lola_dtype;
+
+typedef struct {
+    int32_t batch;              /* B >= 1 */
+    int32_t n_q_heads;          /* multiple of n_kv_heads */
+    int32_t n_kv_heads;         /* >= 1 */
+    int32_t head_dim;           /* d: 32, 64 or 128 */
+    int32_t feat_dim;           /* D: even, D/2 in [8, 128] */
+    int32_t window;             /* eta >= 0 (0 = no softmax window) */
+    int32_t lambda_;            /* sparse-cache capacity, 0..8192 (0 = no cache) */
+    int32_t chunk;              /* prefill update interval C, 1..256 */
+    int32_t decode_interval;    /* decode update interval, 1..min(256, window + 1) */
+    int32_t max_prefill_tokens; /* largest n_tokens of one prefill call (multiple of chunk) */
+    float eps;                  /* >= 0, added to every denominator (SRE and output) */
+    int32_t dtype;              /* lola_dtype of q, k, v, out and W */
+} lola_config;
+
+typedef struct lola_state lola_state; /* opaque host handle */
+
+/* Bytes of device workspace a state with this config needs (persistent state
+ * plus per-call scratch sized by max_prefill_tokens). Pure host computation. */
+lola_status lola_state_bytes(const lola_config *cfg, size_t *device_bytes);
+
+/* Creates a state in `workspace` (device, >= lola_state_bytes, 256-byte
+ * aligned, owned by the caller and kept alive until lola_free_state) and
+ * resets it to the empty state at position 0: H = 0, s = 0, empty cache and
+ * window. W: device [head_dim][feat_dim/2] in cfg->dtype, copied in (the
+ * caller may free it after the stream has passed this call). On success
+ * *out receives a host handle. */
+lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspace,
+                            size_t workspace_bytes, void *cuda_stream, lola_state **out);
+
+/* Returns the state to position 0 (empty memories); W is kept. */
+lola_status lola_reset_state(lola_state *st, void *cuda_stream);
+
+/* Chunkwise prefill of n_tokens new tokens per sequence (all sequences at the
+ * same position). n_tokens must be a positive multiple of cfg.chunk and at most
+ * max_prefill_tokens (else LOLA_ERR_SHAPE / LOLA_ERR_WORKSPACE). The call runs
+ * n_tokens / chunk update intervals of length chunk starting at the current
+ * position and writes every query's output. Not allowed while a decode
+ * interval is open (position not at an interval boundary): LOLA_ERR_STATE. */
+lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, const void *v,
+                               int64_t n_tokens, void *out, void *cuda_stream);
+
+/* One token per sequence: q [B][n_q_heads][head_dim], k, v [B][n_kv_heads][head_dim],
+ * out [B][n_q_heads][head_dim]. When the position is at an interval boundary,
+ * an update interval of length decode_interval opens here (score, select, fold);
+ * the next decode_interval steps belong to it. */
+lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const void *v,
+                             void *out, void *cuda_stream);
+
+/* Current position (tokens processed per sequence). */
+int64_t lola_position(const lola_state *st);
+
+/* Copies the cached token indices: dev_idx [B][n_kv_heads][lambda_] int32
+ * (slot order, -1 for empty slots) and, if dev_count is not NULL,
+ * dev_count [B][n_kv_heads] int32. Device pointers, enqueued on the stream. */
+lola_status lola_get_cache_indices(const lola_state *st, int32_t *dev_idx, int32_t *dev_count,
+                                   void *cuda_stream);
+
+/* Bytes of persistent state + cache per stream (excludes scratch): constant
+ * in the sequence length. */
+lola_status lola_state_stream_bytes(const lola_config *cfg, size_t *bytes);
+
+/* Test hook: log every update interval's kept set. dev_buf is a device int32
+ * buffer of capacity * B * n_kv_heads * (lambda_ + 1) entries; interval i
+ * (counted from the last init/reset) of stream s writes
+ * [count, token ids in slot order, -1 padding] at ((i * streams) + s) * (lambda_ + 1).
+ * Intervals >= capacity are not logged. NULL disables the log. */
+lola_status lola_set_selection_log(lola_state *st, int32_t *dev_buf, int64_t capacity);
+
+/* Test hook: force the kept set of each interval instead of the one the
+ * selection kernel computes (the kernel still runs and still logs its own
+ * choice). dev_kept has the selection-log layout with ASCENDING token ids;
+ * intervals >= n_intervals are not forced. NULL disables forcing. Used to keep
+ * a GPU run on the reference trajectory where the top-lambda choice is
+ * numerically ambiguous. */
+lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept,
+                                        int64_t n_intervals);
+
+/* Waits for the stream work of this state to finish and reports device-side
+ * errors recorded since the last lola_sync (LOLA_ERR_DEVICE / LOLA_ERR_TIMEOUT),
+ * clearing them. */
+lola_status lola_sync(lola_state *st, void *cuda_stream);
+
+/* Frees the host handle only; the workspace stays the caller's. */
+lola_status lola_free_state(lola_state *st);
+
+const char *lola_status_string(lola_status s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* LOLA_H */

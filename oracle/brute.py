@@ -66,7 +66,7 @@ def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6):
                 K = set(order[:min(lam, len(order))])
                 kept_log[-1].append(sorted(K))
                 sre_log[-1].append(sres)
-                for p in range(t0, t1):
+                for p in range(t0, min(t1, T)):
                     for r in range(g):
                         hq = hk * g + r
                         qp = q[b, p, hq, :]

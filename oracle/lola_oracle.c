@@ -353,8 +353,10 @@ static void *worker(void *arg)
 /*
  * Runs the recurrence for every (batch, kv-head) stream from an empty state.
  * Returns 0 on success, a negative number on an invalid argument.
- * Tokens [0, T) are split into n_int consecutive intervals of the given lengths
- * (their sum must be T). Every output pointer except `out` may be NULL.
+ * Tokens [0, T) are split into n_int consecutive intervals of the given lengths;
+ * they must cover [0, T), and the last may extend past T when the pairs it
+ * scores (those leaving the window before its end) all exist. Every output
+ * pointer except `out` may be NULL.
  */
 int oracle_run(const oracle_cfg *cfg, int T, const float *q, const float *k, const float *v,
                const float *Wf, int n_int, const int32_t *int_len, const uint8_t *qmask,
@@ -365,12 +367,16 @@ int oracle_run(const oracle_cfg *cfg, int T, const float *q, const float *k, con
     if (!cfg || cfg->Hkv <= 0 || cfg->Hq % cfg->Hkv != 0 || cfg->d <= 0 || cfg->d > 1024 ||
         cfg->D <= 0 || cfg->D % 2 != 0 || cfg->eta < 0 || cfg->lam < 0 || T < 0)
         return -1;
+    /* The intervals cover [0, T); the last one may run past T (a decode
+     * interval that is still open), as long as every pair it scores exists. */
     long tot = 0;
     for (int i = 0; i < n_int; ++i) {
         if (int_len[i] <= 0) return -2;
+        if (tot >= T && T > 0) return -3;
         tot += int_len[i];
+        if (tot - cfg->eta > T) return -4;
     }
-    if (tot != T) return -3;
+    if (tot < T) return -3;
     int Dh = cfg->D / 2;
     double *W = (double *)malloc(sizeof(double) * (size_t)cfg->d * Dh);
     for (int i = 0; i < cfg->d * Dh; ++i) W[i] = Wf[i];

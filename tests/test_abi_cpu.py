@@ -1,0 +1,71 @@
+"""Host-side checks of the C ABI that need no GPU: the library loads, exports
+every symbol include/lola.h declares, sizes workspaces, and rejects bad
+arguments with the documented status codes before touching the device."""
+import ctypes
+
+import pytest
+
+from hybrid_linear_attention_lola_b200 import build as B
+from hybrid_linear_attention_lola_b200 import lola as L
+from hybrid_linear_attention_lola_b200 import workloads as wl
+
+
+@pytest.fixture(scope="module")
+def lib():
+    B.build()
+    return L.load_library()
+
+
+def test_exports_every_header_symbol(lib):
+    names = L.header_symbols()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_state_bytes_for_every_workload(lib):
+    for w in wl.WORKLOADS.values():
+        cfg = L.config_from_workload(w, max_prefill_tokens=min(w.seq_len, 16384))
+        n = L.lola_state_bytes(cfg)
+        assert n > 0 and n % 256 == 0
+
+
+def test_stream_bytes_constant_in_sequence_length(lib):
+    w = wl.WORKLOADS["long-context"]
+    sizes = {L.lola_state_stream_bytes(L.config_from_workload(w, max_prefill_tokens=n))
+             for n in (128, 4096, 65536)}
+    assert len(sizes) == 1
+    # H|s fp32 + cache K/V bf16 + indices + ring K/V bf16 + flags
+    d, D, lam, eta, C = 128, 256, 2048, 64, 128
+    R = eta + C + 1
+    assert sizes.pop() == D * d * 4 + D * 4 + 2 * lam * d * 2 + lam * 4 + 2 * R * d * 2 + C
+
+
+@pytest.mark.parametrize("field,value,code", [
+    ("dtype", 7, 3), ("head_dim", 48, 1), ("feat_dim", 48, 1), ("n_q_heads", 12, 1),
+    ("decode_interval", 70, 1), ("chunk", 0, 1), ("lambda_", -1, 1), ("window", -2, 1),
+    ("max_prefill_tokens", 100, 1), ("eps", -1.0, 1), ("n_q_heads", 80, 1),
+])
+def test_config_validation(lib, field, value, code):
+    cfg = L.config_from_workload(wl.WORKLOADS["prefill-1b"])
+    setattr(cfg, field, value)
+    n = ctypes.c_size_t(0)
+    assert lib.lola_state_bytes(ctypes.byref(cfg), ctypes.byref(n)) == code
+
+
+def test_null_arguments_rejected_without_device(lib):
+    cfg = L.config_from_workload(wl.WORKLOADS["tiny"])
+    h = ctypes.c_void_p(0)
+    assert lib.lola_init_state(ctypes.byref(cfg), None, None, 0, None, ctypes.byref(h)) == 1
+    assert lib.lola_prefill_chunk(None, None, None, None, 64, None, None) == 1
+    assert lib.lola_decode_step(None, None, None, None, None, None) == 1
+    assert lib.lola_sync(None, None) == 1
+    assert lib.lola_state_bytes(None, None) == 1
+    assert lib.lola_position(None) == -1
+    assert lib.lola_free_state(None) == 0
+
+
+def test_status_strings(lib):
+    for code in range(9):
+        assert lib.lola_status_string(code)
+    assert b"unknown" in lib.lola_status_string(99)

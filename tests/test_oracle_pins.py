@@ -324,4 +324,20 @@ def test_qmask_rows_equal_full_run():
 def test_rejects_bad_intervals():
     q, k, v, W = _qkvw(1, 8, 2, 1, 8, 8, 100)
     with pytest.raises(ValueError):
-        oracle.run(q, k, v, W, window=2, lambda_=2, intervals=[4, 3])
+        oracle.run(q, k, v, W, window=2, lambda_=2, intervals=[4, 3])       # short of T
+    with pytest.raises(ValueError):
+        oracle.run(q, k, v, W, window=2, lambda_=2, intervals=[4, 4, 2])    # interval past T
+    with pytest.raises(ValueError):
+        oracle.run(q, k, v, W, window=2, lambda_=2, intervals=[4, 8])       # scores unseen pairs
+
+
+def test_open_last_interval_matches_bruteforce():
+    """A decode interval still open at the end: its candidates are all known
+    (interval length <= eta + 1) and its queries stop at T."""
+    T, eta, lam = 37, 5, 4
+    q, k, v, W = _qkvw(1, T, 4, 2, 8, 8, 101)
+    ints = [4] * 7 + [6, 6]          # covers 40 >= 37, last interval opened at 34
+    r = oracle.run(q, k, v, W, window=eta, lambda_=lam, intervals=ints)
+    out_b, kept_b, _ = brute.run(q, k, v, W, window=eta, lambda_=lam, intervals=ints)
+    np.testing.assert_allclose(r.out, out_b, rtol=1e-10, atol=1e-12)
+    assert [t for t in r.kept[-1, 1] if t >= 0] == kept_b[-1][1]
