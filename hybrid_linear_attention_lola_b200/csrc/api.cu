@@ -1,9 +1,11 @@
 // Host side of the C ABI declared in include/lola.h: argument checks, the
 // workspace layout, and the order in which one prefill call or decode step
 // enqueues its kernels on the caller's stream.
+#include <atomic>
 #include <cstdio>
 #include <cstring>
 #include <new>
+#include <vector>
 
 #include "../../include/lola.h"
 #include "lola_internal.cuh"
@@ -31,11 +33,56 @@ struct lola_state {
     long long sel_cap;
     const int32_t *ovr;
     long long ovr_n;
+    // timing hook
+    bool timing;
+    struct Mark { int phase; cudaEvent_t a, b; };
+    std::vector<Mark> marks;
+    std::vector<cudaEvent_t> pool;
 };
 
 namespace {
 
 using lola::Dims;
+
+std::atomic<long long> g_launches{0};
+void counted(int n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+enum Phase { PH_PHI = 0, PH_CHAIN, PH_ATTN, PH_FINAL, PH_APPEND, PH_UPDATE, PH_DECODE, PH_RESET };
+
+cudaEvent_t take_event(lola_state *st)
+{
+    if (!st->pool.empty()) {
+        cudaEvent_t e = st->pool.back();
+        st->pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Brackets a group of launches with events when the timing hook is on.
+struct PhaseScope {
+    lola_state *st;
+    int phase;
+    cudaStream_t stream;
+    cudaEvent_t a = nullptr;
+    PhaseScope(lola_state *s, int ph, cudaStream_t strm) : st(s), phase(ph), stream(strm)
+    {
+        if (st->timing) {
+            a = take_event(st);
+            cudaEventRecord(a, stream);
+        }
+    }
+    ~PhaseScope()
+    {
+        if (st->timing && a) {
+            cudaEvent_t b = take_event(st);
+            cudaEventRecord(b, stream);
+            st->marks.push_back({phase, a, b});
+        }
+    }
+};
 
 constexpr size_t kAlign = 256;
 
@@ -231,7 +278,9 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->ws_bytes = workspace_bytes;
     layout(dm, (char *)workspace, &st->S, &st->P);
     reset_host(st);
+    st->timing = false;
     lola::launch_init_state(dm, st->S, W, (cudaStream_t)cuda_stream);
+    counted(1);
     r = check_launch();
     if (r != LOLA_OK) {
         delete st;
@@ -245,7 +294,11 @@ lola_status lola_reset_state(lola_state *st, void *cuda_stream)
 {
     if (!st) return LOLA_ERR_INVALID_ARG;
     reset_host(st);
-    lola::launch_init_state(st->dm, st->S, nullptr, (cudaStream_t)cuda_stream);
+    {
+        PhaseScope ps(st, PH_RESET, (cudaStream_t)cuda_stream);
+        lola::launch_init_state(st->dm, st->S, nullptr, (cudaStream_t)cuda_stream);
+        counted(1);
+    }
     return check_launch();
 }
 
@@ -266,9 +319,13 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     const int m = n / dm.C;
     const long long pos0 = st->pos;
 
-    lola::launch_phi_kv(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, 0, st->P.phiK, st->nS,
-                        stream);
-    lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
+    {
+        PhaseScope ps(st, PH_PHI, stream);
+        lola::launch_phi_kv(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, 0, st->P.phiK, st->nS,
+                            stream);
+        lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
+        counted(2);
+    }
 
     lola::ChainArgs ca{};
     ca.mode = 0;
@@ -289,7 +346,11 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     ca.sel_cap = st->sel_cap;
     ca.ovr = st->ovr;
     ca.ovr_n = st->ovr_n;
-    lola::launch_chain(dm, st->S, &st->P, ca, stream);
+    {
+        PhaseScope ps(st, PH_CHAIN, stream);
+        lola::launch_chain(dm, st->S, &st->P, ca, stream);
+        counted(1);
+    }
 
     lola::AttnArgs aa{};
     aa.pos0 = pos0;
@@ -299,10 +360,18 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     aa.kin = k;
     aa.vin = v;
     aa.out = out;
-    lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+    {
+        PhaseScope ps(st, PH_ATTN, stream);
+        lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+        counted(1);
+    }
 
     for (int ci = 0; ci < m; ++ci) advance_interval(st, pos0 + (long long)ci * dm.C, dm.C);
-    lola::launch_finalize_prefill(dm, st->S, st->P, k, v, pos0, n, st->nS, stream);
+    {
+        PhaseScope ps(st, PH_FINAL, stream);
+        lola::launch_finalize_prefill(dm, st->S, st->P, k, v, pos0, n, st->nS, stream);
+        counted(2);
+    }
     st->pos = pos0 + n;
     st->interval_end = st->pos;
     return check_launch();
@@ -317,8 +386,13 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
     const Dims &dm = st->dm;
     cudaStream_t stream = (cudaStream_t)cuda_stream;
     const long long pos = st->pos;
-    lola::launch_decode_append(dm, st->S, k, v, pos, stream);
+    {
+        PhaseScope ps(st, PH_APPEND, stream);
+        lola::launch_decode_append(dm, st->S, k, v, pos, stream);
+        counted(1);
+    }
     if (pos == st->interval_end) {
+        PhaseScope ps(st, PH_UPDATE, stream);
         lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
         lola::ChainArgs ca{};
         ca.mode = 1;
@@ -340,6 +414,7 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
         ca.ovr = st->ovr;
         ca.ovr_n = st->ovr_n;
         lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        counted(2);
         advance_interval(st, pos, dm.Cdec);
         st->t0_open = pos;
         st->interval_end = pos + dm.Cdec;
@@ -354,7 +429,11 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
     da.k = k;
     da.v = v;
     da.out = out;
-    lola::launch_decode_attn(dm, st->S, da, stream);
+    {
+        PhaseScope ps(st, PH_DECODE, stream);
+        lola::launch_decode_attn(dm, st->S, da, stream);
+        counted(3);
+    }
     st->pos = pos + 1;
     return check_launch();
 }
@@ -364,6 +443,7 @@ lola_status lola_get_cache_indices(const lola_state *st, int32_t *dev_idx, int32
 {
     if (!st || !dev_idx) return LOLA_ERR_INVALID_ARG;
     lola::launch_get_indices(st->dm, st->S, st->nS, dev_idx, dev_count, (cudaStream_t)cuda_stream);
+    counted(1);
     return check_launch();
 }
 
@@ -398,8 +478,41 @@ lola_status lola_sync(lola_state *st, void *cuda_stream)
     return LOLA_OK;
 }
 
+lola_status lola_set_timing(lola_state *st, int enable)
+{
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    st->timing = enable != 0;
+    return LOLA_OK;
+}
+
+lola_status lola_timing_read(lola_state *st, double *ms, int64_t *n)
+{
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    lola_status r = LOLA_OK;
+    for (auto &mk : st->marks) {
+        float t = 0.f;
+        if (cudaEventSynchronize(mk.b) != cudaSuccess || cudaEventElapsedTime(&t, mk.a, mk.b) != cudaSuccess)
+            r = LOLA_ERR_CUDA;
+        if (ms && mk.phase < 8) ms[mk.phase] += t;
+        if (n && mk.phase < 8) n[mk.phase] += 1;
+        st->pool.push_back(mk.a);
+        st->pool.push_back(mk.b);
+    }
+    st->marks.clear();
+    if (r != LOLA_OK) check_launch();
+    return r;
+}
+
+int64_t lola_launch_count(void) { return g_launches.load(); }
+
 lola_status lola_free_state(lola_state *st)
 {
+    if (!st) return LOLA_OK;
+    for (auto &mk : st->marks) {
+        st->pool.push_back(mk.a);
+        st->pool.push_back(mk.b);
+    }
+    for (cudaEvent_t e : st->pool) cudaEventDestroy(e);
     delete st;
     return LOLA_OK;
 }

@@ -233,8 +233,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = cnt + tid; i < lam; i += nt) lg[1 + i] = -1;
             if (tid == 0) lg[0] = cnt;
         }
-        if (a.ovr != nullptr && iglob < a.ovr_n) {
-            const int32_t *lst_o = a.ovr + ((size_t)iglob * dm.ns + st) * (lam + 1);
+        const int32_t *lst_o =
+            (a.ovr != nullptr && iglob < a.ovr_n) ? a.ovr + ((size_t)iglob * dm.ns + st) * (lam + 1)
+                                                  : nullptr;
+        if (lst_o != nullptr && lst_o[0] >= 0) {   // a negative count leaves this entry unforced
             const int cnt = lst_o[0];
             if (tid == 0 && cnt != nK) raise_error(S.err, ERR_BOUNDS);
             for (int c = tid; c < nQ; c += nt) {

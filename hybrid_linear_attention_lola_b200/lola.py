@@ -64,6 +64,9 @@ def load_library() -> ctypes.CDLL:
         "lola_sync": (I32, [P, P]),
         "lola_free_state": (I32, [P]),
         "lola_status_string": (ctypes.c_char_p, [I32]),
+        "lola_set_timing": (I32, [P, ctypes.c_int]),
+        "lola_timing_read": (I32, [P, P, P]),
+        "lola_launch_count": (I64, []),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)
@@ -160,6 +163,25 @@ def lola_set_selection_override(h: int, buf: int, n_intervals: int):
 
 def lola_sync(h: int, stream: int):
     _check(load_library().lola_sync(h, stream), "lola_sync")
+
+
+def lola_set_timing(h: int, enable: bool):
+    _check(load_library().lola_set_timing(h, 1 if enable else 0), "lola_set_timing")
+
+
+PHASES = ("phi", "chain", "attn", "finalize", "append", "update", "decode", "reset")
+
+
+def lola_timing_read(h: int) -> dict:
+    """Per-phase (total ms, count) of the events recorded since the last read."""
+    ms = (ctypes.c_double * 8)()
+    n = (ctypes.c_int64 * 8)()
+    _check(load_library().lola_timing_read(h, ms, n), "lola_timing_read")
+    return {PHASES[i]: (ms[i], n[i]) for i in range(8)}
+
+
+def lola_launch_count() -> int:
+    return load_library().lola_launch_count()
 
 
 def lola_free_state(h: int):

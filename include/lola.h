@@ -60,12 +60,12 @@ typedef enum { LOLA_F32 = 0, LOLA_BF16 = 1 } lola_dtype;
 
 typedef struct {
     int32_t batch;              /* B >= 1 */
-    int32_t n_q_heads;          /* multiple of n_kv_heads */
+    int32_t n_q_heads;          /* multiple of n_kv_heads, at most 8 per kv-head */
     int32_t n_kv_heads;         /* >= 1 */
     int32_t head_dim;           /* d: 32, 64 or 128 */
-    int32_t feat_dim;           /* D: even, D/2 in [8, 128] */
+    int32_t feat_dim;           /* D: multiple of 32 in [32, 256] */
     int32_t window;             /* eta >= 0 (0 = no softmax window) */
-    int32_t lambda_;            /* sparse-cache capacity, 0..8192 (0 = no cache) */
+    int32_t lambda_;            /* sparse-cache capacity, 0..4096 (0 = no cache) */
     int32_t chunk;              /* prefill update interval C, 1..256 */
     int32_t decode_interval;    /* decode update interval, 1..min(256, window + 1) */
     int32_t max_prefill_tokens; /* largest n_tokens of one prefill call (multiple of chunk) */
@@ -123,18 +123,34 @@ lola_status lola_state_stream_bytes(const lola_config *cfg, size_t *bytes);
 /* Test hook: log every update interval's kept set. dev_buf is a device int32
  * buffer of capacity * B * n_kv_heads * (lambda_ + 1) entries; interval i
  * (counted from the last init/reset) of stream s writes
- * [count, token ids in slot order, -1 padding] at ((i * streams) + s) * (lambda_ + 1).
+ * [count, kept token ids in no particular order, -1 padding] at
+ * ((i * streams) + s) * (lambda_ + 1).
  * Intervals >= capacity are not logged. NULL disables the log. */
 lola_status lola_set_selection_log(lola_state *st, int32_t *dev_buf, int64_t capacity);
 
 /* Test hook: force the kept set of each interval instead of the one the
  * selection kernel computes (the kernel still runs and still logs its own
- * choice). dev_kept has the selection-log layout with ASCENDING token ids;
- * intervals >= n_intervals are not forced. NULL disables forcing. Used to keep
+ * choice). dev_kept has the selection-log layout with ASCENDING token ids and
+ * must hold n_intervals * B * n_kv_heads * (lambda_ + 1) entries; an entry whose
+ * count is negative leaves that (interval, stream) unforced, and intervals
+ * >= n_intervals are not forced. NULL disables forcing. Used to keep
  * a GPU run on the reference trajectory where the top-lambda choice is
  * numerically ambiguous. */
 lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept,
                                         int64_t n_intervals);
+
+/* Timing hook: when enabled (enable != 0), every entry point brackets each of
+ * its kernel phases with CUDA events recorded on the caller's stream. Phases:
+ * 0 feature map, 1 chain (score/select/fold), 2 attention (prefill), 3 call
+ * finalisation, 4 decode append, 5 decode interval update, 6 decode attention,
+ * 7 state reset. lola_timing_read() waits for the recorded events, adds their
+ * elapsed milliseconds to ms[8] and their count to n[8] (caller-zeroed), and
+ * forgets them. Host memory; NULL pointers skip the output. */
+lola_status lola_set_timing(lola_state *st, int enable);
+lola_status lola_timing_read(lola_state *st, double *ms, int64_t *n);
+
+/* Number of kernels this library has launched in the process so far. */
+int64_t lola_launch_count(void);
 
 /* Waits for the stream work of this state to finish and reports device-side
  * errors recorded since the last lola_sync (LOLA_ERR_DEVICE / LOLA_ERR_TIMEOUT),

@@ -38,12 +38,17 @@ def intervals_for(plan, chunk, decode_interval, pos0=0):
     return ints
 
 
-def override_from(r, lam):
+def override_from(r, lam, ns_gpu=None, stream_map=None):
+    """Engine override buffer [n_int, ns_gpu, lam+1] from an oracle run. Streams
+    the oracle did not run (subset runs) get count -1: not forced."""
     n_int, ns = r.nkept.shape
-    buf = np.full((n_int, ns, lam + 1), -1, np.int32)
-    buf[..., 0] = r.nkept
-    if lam:
-        buf[..., 1:] = r.kept
+    ns_gpu = ns if ns_gpu is None else ns_gpu
+    smap = list(range(ns)) if stream_map is None else stream_map
+    buf = np.full((n_int, ns_gpu, lam + 1), -1, np.int32)
+    for so, sg in enumerate(smap):
+        buf[:, sg, 0] = r.nkept[:, so]
+        if lam:
+            buf[:, sg, 1:] = r.kept[:, so]
     return buf
 
 

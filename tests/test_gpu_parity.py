@@ -61,7 +61,7 @@ def _case(w, plan, *, forced=True, unforced=False, subset=None, qmask_every=None
     res = {}
     runs = []
     if forced:
-        runs.append(("forced", P.override_from(r, w.lambda_)))
+        runs.append(("forced", P.override_from(r, w.lambda_, w.batch * w.n_kv_heads, smap)))
     if unforced:
         runs.append(("unforced", None))
     for name, ovr in runs:
