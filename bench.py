@@ -133,7 +133,7 @@ class ClockSampler:
                 parts = [x.strip() for x in line.split(",")]
                 if len(parts) < 10:
                     continue
-                if self.bus_id and self.bus_id[-12:] not in parts[1].lower():
+                if self.bus_id and self.bus_id not in parts[1].lower():
                     continue
                 rows.append(parts)
         if not rows:
@@ -255,7 +255,10 @@ def run_engine(args, ws, rank, local):
     L.lola_timing_read(S.handle)
     L.lola_set_timing(S.handle, True)
     phase_ms = {}
-    bus = getattr(torch.cuda.get_device_properties(dev), "pci_bus_id", None)
+    props = torch.cuda.get_device_properties(dev)
+    bus = None
+    if isinstance(getattr(props, "pci_bus_id", None), int):
+        bus = f"{props.pci_bus_id:02x}:{getattr(props, 'pci_device_id', 0):02x}."
     clocks = ClockSampler(bus).start() if rank == 0 else None
     barrier(ws)
     torch.cuda.synchronize(dev)

@@ -326,6 +326,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
         counted(2);
     }
+    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
     lola::ChainArgs ca{};
     ca.mode = 0;
@@ -351,6 +352,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         lola::launch_chain(dm, st->S, &st->P, ca, stream);
         counted(1);
     }
+    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
     lola::AttnArgs aa{};
     aa.pos0 = pos0;
@@ -365,6 +367,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
         counted(1);
     }
+    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
     for (int ci = 0; ci < m; ++ci) advance_interval(st, pos0 + (long long)ci * dm.C, dm.C);
     {
@@ -391,6 +394,7 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
         lola::launch_decode_append(dm, st->S, k, v, pos, stream);
         counted(1);
     }
+    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
     if (pos == st->interval_end) {
         PhaseScope ps(st, PH_UPDATE, stream);
         lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
@@ -415,6 +419,7 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
         ca.ovr_n = st->ovr_n;
         lola::launch_chain(dm, st->S, nullptr, ca, stream);
         counted(2);
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
         advance_interval(st, pos, dm.Cdec);
         st->t0_open = pos;
         st->interval_end = pos + dm.Cdec;

@@ -115,11 +115,14 @@ void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long
     const long long rows = (long long)dm.ns * (nS + dm.R + n);
     const int grid = grid_for(rows, 8);
     if (dm.dtype == 0) {
+        cudaFuncSetAttribute(phi_kv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         KVSrc<float> src{(const float *)S.KS, (const float *)S.VS, (const float *)S.KR,
                          (const float *)S.VR, (const float *)kin, nullptr,
                          dm.lam, dm.R, n, dm.Hkv, dm.d, call_start};
         phi_kv_kernel<float><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows, phi_out);
     } else {
+        cudaFuncSetAttribute(phi_kv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
         KVSrc<__nv_bfloat16> src{(const __nv_bfloat16 *)S.KS, (const __nv_bfloat16 *)S.VS,
                                  (const __nv_bfloat16 *)S.KR, (const __nv_bfloat16 *)S.VR,
                                  (const __nv_bfloat16 *)kin, nullptr,
@@ -134,12 +137,16 @@ void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows,
 {
     const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
     const int grid = grid_for(rows, 8);
-    if (dm.dtype == 0)
+    if (dm.dtype == 0) {
+        cudaFuncSetAttribute(phi_q_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         phi_q_kernel<float><<<grid, 256, smem, stream>>>(dm.d, dm.Dh, W, (const float *)q, rows,
                                                          phi_out);
-    else
+    } else {
+        cudaFuncSetAttribute(phi_q_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
         phi_q_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(
             dm.d, dm.Dh, W, (const __nv_bfloat16 *)q, rows, phi_out);
+    }
 }
 
 // ---------------------------------------------------------------- init
