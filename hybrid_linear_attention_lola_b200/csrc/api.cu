@@ -4,6 +4,7 @@
 #include <atomic>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <new>
 #include <vector>
 
@@ -523,3 +524,117 @@ lola_status lola_free_state(lola_state *st)
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- decode step, library-owned scratch
+//
+// lola_decode_step_static runs the same decode step as lola_decode_step, but
+// the per-step temporaries of the split decode attention (the query feature
+// rows and the per-split partial sums) live in the fixed device array below
+// instead of the caller's workspace. It exists for callers that cannot obtain
+// device memory on demand: a host framework that owns all device memory and
+// hands a plugin only its inputs, outputs and persistent state, or code that
+// runs while a CUDA graph is being captured, where cudaMalloc is not allowed.
+// The array is part of the library image, so every GPU that loads the library
+// holds it until the process exits.
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(8) << 20;  // 8 MiB per device
+static __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void *g_static_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up once
+// per device, with that device current, and cached.
+lola_status static_scratch_address(void **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LOLA_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (g_static_ptr[dev] == nullptr) {
+        void *p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress((void **)&p, g_decode_scratch);
+        if (e != cudaSuccess || p == nullptr) {
+            fprintf(stderr, "lola: cudaGetSymbolAddress failed: %s\n", cudaGetErrorString(e));
+            return LOLA_ERR_CUDA;
+        }
+        g_static_ptr[dev] = p;
+    }
+    *out = g_static_ptr[dev];
+    return LOLA_OK;
+}
+
+}  // namespace
+
+extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, const void *k,
+                                               const void *v, void *out, void *cuda_stream)
+{
+    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return LOLA_ERR_INVALID_ARG;
+    const Dims &dm = st->dm;
+    const size_t phiq_bytes = align_up((size_t)dm.B * dm.Hq * dm.D * 4);
+    const size_t part_bytes = align_up((size_t)dm.ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
+    if (phiq_bytes + part_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
+    void *base = nullptr;
+    const lola_status sr = static_scratch_address(&base);
+    if (sr != LOLA_OK) return sr;
+    // Every entry of both regions is written before it is read within one
+    // call, so nothing has to start at zero.
+    lola::DevState Sx = st->S;
+    Sx.phiQd = (float *)base;
+    Sx.part = (float *)((char *)base + phiq_bytes);
+
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    const long long pos = st->pos;
+    {
+        PhaseScope ps(st, PH_APPEND, stream);
+        lola::launch_decode_append(dm, st->S, k, v, pos, stream);
+        counted(1);
+    }
+    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+    if (pos == st->interval_end) {
+        PhaseScope ps(st, PH_UPDATE, stream);
+        lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
+        lola::ChainArgs ca{};
+        ca.mode = 1;
+        ca.pos0 = pos;
+        ca.n_int = 1;
+        ca.ilen = dm.Cdec;
+        ca.nS0 = st->nS;
+        ca.pend_lo = st->pend_lo;
+        ca.pend_n = st->pend_n;
+        ca.iglob0 = st->n_int;
+        ca.phi = st->S.phiV;
+        ca.nvrows = dm.lam + dm.R;
+        ca.sel_log = st->sel_log;
+        ca.sel_cap = st->sel_cap;
+        ca.ovr = st->ovr;
+        ca.ovr_n = st->ovr_n;
+        lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        counted(2);
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+        advance_interval(st, pos, dm.Cdec);
+        st->t0_open = pos;
+        st->interval_end = pos + dm.Cdec;
+    }
+    lola::DecodeArgs da{};
+    da.pos = pos;
+    da.t0 = st->t0_open;
+    da.nS = st->nS;
+    da.L_lo = st->pend_lo;
+    da.L_hi = st->pend_lo + st->pend_n;
+    da.q = q;
+    da.k = k;
+    da.v = v;
+    da.out = out;
+    {
+        PhaseScope ps(st, PH_DECODE, stream);
+        lola::launch_decode_attn(dm, Sx, da, stream);
+        counted(3);
+    }
+    st->pos = pos + 1;
+    return check_launch();
+}

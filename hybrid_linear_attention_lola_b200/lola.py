@@ -57,6 +57,7 @@ def load_library() -> ctypes.CDLL:
         "lola_reset_state": (I32, [P, P]),
         "lola_prefill_chunk": (I32, [P, P, P, P, I64, P, P]),
         "lola_decode_step": (I32, [P, P, P, P, P, P]),
+        "lola_decode_step_static": (I32, [P, P, P, P, P, P]),
         "lola_position": (I64, [P]),
         "lola_get_cache_indices": (I32, [P, P, P, P]),
         "lola_set_selection_log": (I32, [P, P, I64]),
@@ -142,6 +143,13 @@ def lola_prefill_chunk(h: int, q: int, k: int, v: int, n_tokens: int, out: int, 
 
 def lola_decode_step(h: int, q: int, k: int, v: int, out: int, stream: int):
     _check(load_library().lola_decode_step(h, q, k, v, out, stream), "lola_decode_step")
+
+
+def lola_decode_step_static(h: int, q: int, k: int, v: int, out: int, stream: int):
+    """Decode step whose temporaries come from a fixed device array inside the
+    library; for callers that cannot allocate device memory on demand."""
+    _check(load_library().lola_decode_step_static(h, q, k, v, out, stream),
+           "lola_decode_step_static")
 
 
 def lola_position(h: int) -> int:

@@ -107,6 +107,26 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
 lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const void *v,
                              void *out, void *cuda_stream);
 
+/* The same decode step as lola_decode_step, for callers that cannot obtain
+ * device memory on demand -- for example a plugin whose host framework owns
+ * all device memory and passes it only inputs, outputs and persistent state,
+ * or code running while a CUDA graph is being captured, where cudaMalloc is
+ * not allowed. The paper has no counterpart to this call; it only changes
+ * where temporaries live. The per-step scratch of the decode attention (query
+ * features and split partials) is taken from an 8 MiB array inside the
+ * library (a static device array: every GPU that loads the library holds it
+ * until the process exits) instead of the workspace. The call allocates
+ * nothing. Configs whose decode scratch,
+ * B*n_q_heads*feat_dim*4 + streams*splits*(n_q_heads/n_kv_heads)*(2*head_dim+4)*4
+ * bytes (each part rounded up to 256), exceed 8 MiB get LOLA_ERR_WORKSPACE.
+ * The first call on a device looks up the array's device address (once per
+ * device, with the device current); make that first call before any stream
+ * capture. All calls share the one array and leave their contents in it, so
+ * calls whose work overlaps on the GPU (other states, other streams) race:
+ * order them on one stream or synchronise between them. */
+lola_status lola_decode_step_static(lola_state *st, const void *q, const void *k, const void *v,
+                                    void *out, void *cuda_stream);
+
 /* Current position (tokens processed per sequence). */
 int64_t lola_position(const lola_state *st);
 
