@@ -1,0 +1,199 @@
+// Thin helpers around the sm_100a 5th-generation tensor-core instructions
+// (tcgen05.*): shared-memory matrix descriptors for 128-byte-swizzled bf16
+// operands, the instruction descriptor for bf16 x bf16 -> fp32, TMEM
+// allocation, MMA issue/commit, TMEM loads, and mbarrier waits that give up
+// after a bounded number of polls.
+//
+// Operand layouts (bf16, 128-byte swizzle; every tile base 1024-byte aligned):
+//  * K-major tile of R rows (R % 8 == 0) and K columns: atom column kb = k / 64
+//    holds R rows of 128 bytes; rows are grouped by 8 (1024 bytes). Within a
+//    row the 16-byte chunk index is XOR-ed with (row % 8).
+//      offset(r, k) = kb*R*128 + (r/8)*1024 + (r%8)*128 + (((k%64)/8) ^ (r%8))*16 + (k%8)*2
+//    Descriptor: LBO = 16 B, SBO = 1024 B; the 16-element k-step ks starts at
+//    base + (ks/4)*R*128 + (ks%4)*32.
+//  * MN-major tile (N contiguous) of K rows and N columns (N % 64 == 0): atoms
+//    of 8 k-rows x 64 n-elements (1024 bytes), laid out [k/8][n/64][k%8][128 B].
+//      offset(k, n) = (k/8)*(N/64)*1024 + (n/64)*1024 + (k%8)*128 + (((n%64)/8) ^ (k%8))*16 + (n%8)*2
+//    Descriptor: LBO = 1024 B (next 64 n), SBO = (N/64)*1024 B (next 8 k); the
+//    k-step ks starts at base + 2*ks*SBO.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+namespace lola {
+namespace umma {
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p)
+{
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ uint32_t kmajor_offset(int r, int k, int R)
+{
+    const int kb = k >> 6, kk = k & 63;
+    return (uint32_t)(kb * R * 128 + (r >> 3) * 1024 + (r & 7) * 128 +
+                      ((((kk >> 3) ^ (r & 7))) << 4) + ((kk & 7) << 1));
+}
+
+__device__ __forceinline__ uint32_t mnmajor_offset(int k, int n, int N)
+{
+    const int nb = n >> 6, nn = n & 63;
+    return (uint32_t)((k >> 3) * (N >> 6) * 1024 + nb * 1024 + (k & 7) * 128 +
+                      ((((nn >> 3) ^ (k & 7))) << 4) + ((nn & 7) << 1));
+}
+
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1 << 46;   // descriptor version for sm_100
+    d |= (uint64_t)2 << 61;   // 128-byte swizzle
+    return d;
+}
+
+__device__ __forceinline__ uint64_t kmajor_desc(uint32_t base, int ks, int R)
+{
+    return make_desc(base + (uint32_t)((ks >> 2) * R * 128 + (ks & 3) * 32), 16, 1024);
+}
+
+__device__ __forceinline__ uint64_t mnmajor_desc(uint32_t base, int ks, int N)
+{
+    const uint32_t sbo = (uint32_t)(N >> 6) * 1024;
+    return make_desc(base + (uint32_t)(2 * ks) * sbo, 1024, sbo);
+}
+
+// bf16 x bf16 -> fp32, dense; a_mn / b_mn select MN-major operands.
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool a_mn, bool b_mn)
+{
+    return (1u << 4)                     // D format fp32
+           | (1u << 7)                   // A format bf16
+           | (1u << 10)                  // B format bf16
+           | ((a_mn ? 1u : 0u) << 15)    // A major
+           | ((b_mn ? 1u : 0u) << 16)    // B major
+           | ((uint32_t)(N >> 3) << 17)  // N / 8
+           | ((uint32_t)(M >> 4) << 24); // M / 16
+}
+
+// D[tmem] (+)= A[smem desc] * B[smem desc]; issued by one thread.
+__device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t idesc, uint32_t accumulate)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+        :
+        : "r"(d_tmem), "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate));
+}
+
+// Arrive on an mbarrier once all previously issued MMAs of this thread complete.
+__device__ __forceinline__ void mma_commit(uint64_t *mbar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :
+                 : "r"(smem_u32(mbar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void fence_before_sync()
+{
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void fence_after_sync()
+{
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+// Makes generic-proxy shared-memory writes visible to the tensor core.
+__device__ __forceinline__ void fence_async_smem()
+{
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// TMEM allocation by one full warp; the base address lands in *slot (smem).
+__device__ __forceinline__ void tmem_alloc(uint32_t *slot, uint32_t ncols)
+{
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                 :
+                 : "r"(smem_u32(slot)), "r"(ncols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols)
+{
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols)
+                 : "memory");
+}
+
+// 32 lanes x 16 consecutive fp32 columns: thread t of the warp gets lane
+// (lane_base + t), columns [col, col + 16).
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+          "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+
+// 32 lanes x 16 columns store (thread t writes lane lane_base + t).
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
+{
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+        "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+        :
+        : "r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+          "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+          "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+          "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+          "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+          "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15]))
+        : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_init(uint64_t *mbar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(mbar)), "r"(count)
+                 : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Polls the mbarrier phase `parity`; gives up after max_polls and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t max_polls)
+{
+    const uint32_t a = smem_u32(mbar);
+    for (uint32_t i = 0; i < max_polls; ++i) {
+        uint32_t done;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}\n"
+            : "=r"(done)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+
+// 16-byte asynchronous global -> shared copy (L2 only).
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+                 : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+}  // namespace umma
+}  // namespace lola

@@ -68,6 +68,7 @@ def load_library() -> ctypes.CDLL:
         "lola_set_timing": (I32, [P, ctypes.c_int]),
         "lola_timing_read": (I32, [P, P, P]),
         "lola_launch_count": (I64, []),
+        "lola_selftest_umma": (I32, [ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P, P]),
     }
     for name, (res, args) in sigs.items():
         f = getattr(lib, name)

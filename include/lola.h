@@ -169,6 +169,17 @@ lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept,
 lola_status lola_set_timing(lola_state *st, int enable);
 lola_status lola_timing_read(lola_state *st, double *ms, int64_t *n);
 
+/* Test hook for the tensor-core layer: one CTA computes, on the tcgen05 tensor
+ * cores, C[128][N] (fp32, row-major) = A[128][K] * op(B), where A is bf16
+ * row-major, and B is bf16 [N][K] with C = A B^T (layout 0, K-major operand)
+ * or [K][N] with C = A B (layout 1, N-contiguous operand, N % 64 == 0).
+ * 16 <= N, K <= 256, multiples of 16. Device pointers; dev_err is a device
+ * int that receives LOLA's timeout bit if the MMA completion wait gives up.
+ * Not part of the method (the paper has no counterpart); it checks the shared
+ * memory layouts and descriptors the attention and scoring kernels use. */
+lola_status lola_selftest_umma(int layout, const void *A, const void *B, float *C, int N, int K,
+                               int *dev_err, void *cuda_stream);
+
 /* Number of kernels this library has launched in the process so far. */
 int64_t lola_launch_count(void);
 
