@@ -131,7 +131,9 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     if (ns > tiles) ns = tiles;
     if (ns < 1) ns = 1;
     dm->nsplit = (int)ns;
-    if (lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
+    dm->tc_chain = (c->dtype == LOLA_BF16 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
+    if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
+    dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     return LOLA_OK;
 }
@@ -160,15 +162,16 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.VR = take(ns * dm.R * dm.d * e);
     s.pend = (uint8_t *)take(ns * dm.Lmax);
     s.W = (float *)take((size_t)dm.d * dm.Dh * 4);
-    s.phiV = (float *)take(ns * (dm.lam + dm.R) * dm.D * 4);
-    s.phiQd = (float *)take((size_t)dm.B * dm.Hq * dm.D * 4);
+    s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
+    s.phiQd = take((size_t)dm.B * dm.Hq * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     lola::PrefillScratch p{};
     const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
-    p.phiK = (float *)take(ns * nv * dm.D * 4);
-    p.phiQ = (float *)take((size_t)dm.B * dm.Nmax * dm.Hq * dm.D * 4);
-    p.snapH = (float *)take(ns * dm.mmax * dm.D * dm.d * 4);
-    p.snapS = (float *)take(ns * dm.mmax * dm.D * 4);
+    p.phiK = take(ns * nv * dm.D * e);
+    p.phiQ = take((size_t)dm.B * dm.Nmax * dm.Hq * dm.D * e);
+    p.snapH = (float *)take(dm.tc_attn ? 0 : ns * dm.mmax * dm.D * dm.d * 4);
+    p.snapS = (float *)take(dm.tc_attn ? 0 : ns * dm.mmax * dm.D * 4);
+    p.snapImg = dm.tc_chain ? take(ns * dm.mmax * lola::snap_image_bytes(dm)) : nullptr;
     p.logTok = (int *)take(ns * dm.mmax * dm.lam * 4);
     p.logVrow = (int *)take(ns * dm.mmax * dm.lam * 4);
     p.logCount = (int *)take(ns * dm.mmax * 4);
@@ -350,7 +353,9 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     ca.ovr_n = st->ovr_n;
     {
         PhaseScope ps(st, PH_CHAIN, stream);
-        lola::launch_chain(dm, st->S, &st->P, ca, stream);
+        ca.snap_f32 = dm.tc_attn ? 0 : 1;
+        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, stream);
+        else lola::launch_chain(dm, st->S, &st->P, ca, stream);
         counted(1);
     }
     if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
@@ -365,7 +370,8 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     aa.out = out;
     {
         PhaseScope ps(st, PH_ATTN, stream);
-        lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+        if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
+        else lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
         counted(1);
     }
     if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
@@ -418,7 +424,8 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;
         ca.ovr_n = st->ovr_n;
-        lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
+        else lola::launch_chain(dm, st->S, nullptr, ca, stream);
         counted(2);
         if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
         advance_interval(st, pos, dm.Cdec);
@@ -575,7 +582,7 @@ extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, co
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
         return LOLA_ERR_INVALID_ARG;
     const Dims &dm = st->dm;
-    const size_t phiq_bytes = align_up((size_t)dm.B * dm.Hq * dm.D * 4);
+    const size_t phiq_bytes = align_up((size_t)dm.B * dm.Hq * dm.D * elem_bytes(dm));
     const size_t part_bytes = align_up((size_t)dm.ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     if (phiq_bytes + part_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
     void *base = nullptr;
@@ -584,7 +591,7 @@ extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, co
     // Every entry of both regions is written before it is read within one
     // call, so nothing has to start at zero.
     lola::DevState Sx = st->S;
-    Sx.phiQd = (float *)base;
+    Sx.phiQd = base;
     Sx.part = (float *)((char *)base + phiq_bytes);
 
     cudaStream_t stream = (cudaStream_t)cuda_stream;
@@ -613,7 +620,8 @@ extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, co
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;
         ca.ovr_n = st->ovr_n;
-        lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
+        else lola::launch_chain(dm, st->S, nullptr, ca, stream);
         counted(2);
         if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
         advance_interval(st, pos, dm.Cdec);

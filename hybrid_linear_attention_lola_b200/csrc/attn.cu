@@ -68,7 +68,7 @@ __global__ void __launch_bounds__(NW * 32)
     for (int e = tid; e < nrows * D; e += blockDim.x) {
         const int r = e / D, i = e - r * D;
         const long long tok = t0 - a.pos0 + row0 + r;
-        phq[e] = P.phiQ[(((size_t)b * a.n_call + tok) * dm.Hq + hq) * D + i];
+        phq[e] = to_f<T>(((const T *)P.phiQ)[(((size_t)b * a.n_call + tok) * dm.Hq + hq) * D + i]);
     }
 
     RowAcc acc[RPW];
@@ -131,7 +131,8 @@ __global__ void __launch_bounds__(NW * 32)
             for (int e = tid; e < nk * D; e += blockDim.x) {
                 const int j = e / D, i = e - j * D;
                 const int vr = src.tok2vrow(kb + j);
-                phk[j * (D + 1) + i] = P.phiK[((size_t)st * (lam + dm.R + dm.Nmax) + vr) * D + i];
+                phk[j * (D + 1) + i] =
+                    to_f<T>(((const T *)P.phiK)[((size_t)st * (lam + dm.R + dm.Nmax) + vr) * D + i]);
             }
         }
         __syncthreads();

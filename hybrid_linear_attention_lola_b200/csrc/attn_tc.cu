@@ -1,0 +1,373 @@
+// Tensor-core prefill output of a LoLA hybrid-attention layer for bfloat16
+// inputs (gist.science technical summary, "Inferentiestrategie": linear
+// attention + sparse-cache attention + sliding-window attention, combined).
+//
+// One CTA = one update interval of one (batch, kv-head) stream and 128 query
+// rows; row r is (position t0 + mt*128/g + r/g, query head hk*g + r%g), so the
+// rows of a tile are consecutive in q and out. Thread r owns row r (TMEM lane r).
+//   1. O = phi(Q) [H'|s']   (readout of the interval's snapshot; column d of O
+//      carries the linear denominator phi(q).s', so it rescales with O);
+//   2. per 64-key tile: S = Q K^T (and G = phi(Q) phi(K)^T for window tiles that
+//      hold folded leaving pairs) on the tensor cores; thread r turns row r into
+//      P = e^{s-m} (softmax keys) or g e^{-m} (linear keys) with the running
+//      shift m = max(0, max score), rescales its O row in TMEM when m grows, and
+//      writes P (bf16) to shared memory; O += P V.
+//   3. out = O[:, :d] / (sum P + O[:, d] + eps e^{-m}).
+// The key classes follow the method: cached keys are softmax (causal); window
+// keys [t0 - eta, t1) are softmax while inside the window of p, linear once
+// they left it and were folded, and skipped when they were kept (they appear
+// among the cached keys).
+#include "lola_internal.cuh"
+#include "umma.cuh"
+
+namespace lola {
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int kThreads = 128;
+constexpr int KT = 64;                // keys per tile
+constexpr uint32_t kPolls = 1u << 26;
+enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
+
+struct AGeo {
+    int d, D, FP, NB, NBa;
+    uint32_t ncols;
+    size_t off_phq, off_big, off_K, off_V, off_phk, off_P, off_tok, off_info, total;
+};
+
+__host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline AGeo make_ageo(const Dims &dm)
+{
+    AGeo g{};
+    g.d = dm.d;
+    g.D = dm.D;
+    g.FP = (dm.D + 127) / 128 * 128;
+    g.NB = dm.d + 16;
+    g.NBa = (g.NB + 31) / 32 * 32;
+    const uint32_t need = (uint32_t)(g.NBa + 2 * KT);
+    g.ncols = need <= 128 ? 128 : need <= 256 ? 256 : 512;
+    const int dp = (g.d + 63) / 64 * 64;                  // K-major rows span whole atoms
+    size_t o = (size_t)128 * dp * 2;                       // Q
+    g.off_phq = al(o, 1024);
+    o = g.off_phq + (size_t)128 * g.FP * 2;                // phi(Q)
+    g.off_big = al(o, 1024);                               // snapshot image, then key tiles
+    g.off_K = g.off_big;
+    g.off_V = al(g.off_K + (size_t)KT * dp * 2, 1024);
+    g.off_phk = al(g.off_V + (size_t)KT * g.d * 2, 1024);
+    g.off_P = al(g.off_phk + (size_t)KT * g.FP * 2, 1024);
+    size_t tiles_end = g.off_P + (size_t)128 * KT * 2;
+    size_t img_end = g.off_big + (size_t)g.NB * g.FP * 2;
+    o = tiles_end > img_end ? tiles_end : img_end;
+    g.off_tok = al(o, 16);
+    g.off_info = g.off_tok + KT * 4;
+    g.total = g.off_info + KT * 4 + 1024;
+    return g;
+}
+
+__device__ __forceinline__ bool wait_mbar(uint64_t *mbar, uint32_t &phase, int *okflag)
+{
+    if (threadIdx.x == 0) *okflag = umma::mbar_wait(mbar, phase, kPolls) ? 1 : 0;
+    __syncthreads();
+    phase ^= 1u;
+    umma::fence_after_sync();
+    return *okflag != 0;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    attn_tc_kernel(Dims dm, DevState S, PrefillScratch P, AttnArgs a, KVSrc<bf16> src)
+{
+    const AGeo g = make_ageo(dm);
+    const int d = g.d, D = g.D, FP = g.FP, NB = g.NB, eta = dm.eta, lam = dm.lam, gq = dm.g;
+    const int tiles_per_int = (dm.C * gq + 127) / 128;
+    const int ci = blockIdx.x / tiles_per_int, mt = blockIdx.x % tiles_per_int;
+    const int st = blockIdx.y;
+    const int b = st / dm.Hkv, hk = st % dm.Hkv;
+    const long long t0 = a.pos0 + (long long)ci * dm.C, t1 = t0 + dm.C;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int rows_total = dm.C * gq;
+    const int grow = mt * 128 + tid;                 // row within the interval
+    const bool row_ok = grow < rows_total;
+    const long long p = t0 + grow / gq;              // query position of this thread's row
+    const float scale = rsqrtf((float)d);
+
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    __shared__ int okflag;
+    __shared__ int anylin;
+    const uint32_t raw = umma::smem_u32(smraw);
+    uint8_t *base = smraw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *sQ = base, *sPhq = base + g.off_phq, *sImg = base + g.off_big;
+    uint8_t *sK = base + g.off_K, *sV = base + g.off_V, *sPhk = base + g.off_phk, *sP = base + g.off_P;
+    int *ktok = (int *)(base + g.off_tok);
+    int *kinfo = (int *)(base + g.off_info);
+
+    if (tid == 0) umma::mbar_init(&mbar, 1);
+    if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    const uint32_t tm = tslot;
+    const uint32_t tO = tm, tS = tm + (uint32_t)g.NBa, tG = tS + KT;
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    uint32_t phase = 0;
+
+    // ---- stage Q, phi(Q) and the snapshot image
+    const bf16 *q = (const bf16 *)a.q;
+    const bf16 *phiQ = (const bf16 *)P.phiQ;
+    const size_t qrow0 = ((size_t)b * a.n_call + (size_t)(t0 - a.pos0)) * dm.Hq + (size_t)hk * gq;
+    for (int e = tid; e < 128 * (d / 8); e += kThreads) {
+        const int r = e / (d / 8), kc = e % (d / 8);
+        const int gr = mt * 128 + r;
+        uint8_t *dst = sQ + umma::kmajor_offset(r, kc * 8, 128);
+        if (gr < rows_total) {
+            const size_t row = qrow0 + (size_t)(gr / gq) * dm.Hq + gr % gq;
+            umma::cp_async16(dst, q + row * d + kc * 8);
+        } else {
+            *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+        }
+    }
+    for (int e = tid; e < 128 * (FP / 8); e += kThreads) {
+        const int r = e / (FP / 8), kc = e % (FP / 8);
+        const int gr = mt * 128 + r;
+        uint8_t *dst = sPhq + umma::kmajor_offset(r, kc * 8, 128);
+        if (gr < rows_total && kc * 8 < D) {
+            const size_t row = qrow0 + (size_t)(gr / gq) * dm.Hq + gr % gq;
+            umma::cp_async16(dst, phiQ + row * D + kc * 8);
+        } else {
+            *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+        }
+    }
+    {
+        const uint8_t *img = (const uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * NB * FP * 2;
+        for (int e = tid; e < NB * FP * 2 / 16; e += kThreads) umma::cp_async16(sImg + e * 16, img + e * 16);
+    }
+    umma::cp_async_commit();
+    umma::cp_async_wait_all();
+    umma::fence_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+
+    bool ok = true;
+    // ---- 1. O = phi(Q) [H'|s']
+    if (tid == 0) {
+        umma::fence_after_sync();
+        const uint32_t a0 = umma::smem_u32(sPhq), b0 = umma::smem_u32(sImg);
+        const uint32_t id = umma::idesc_bf16(128, NB, false, false);
+        for (int ks = 0; ks < FP / 16; ++ks)
+            umma::mma_ss(tO, umma::kmajor_desc(a0, ks, 128), umma::kmajor_desc(b0, ks, NB), id, ks > 0 ? 1u : 0u);
+        umma::mma_commit(&mbar);
+    }
+    ok = wait_mbar(&mbar, phase, &okflag);
+
+    float m = 0.f, l = 0.f;
+    const size_t lb = (size_t)st * dm.mmax + ci;
+    const int nK = P.logCount[lb];
+    const int *ltok = P.logTok + lb * lam;
+    const int *lvrow = P.logVrow + lb * lam;
+    const uint8_t *llf = P.logLf + lb * dm.Lmax;
+    const long long jlo = t0 - eta > 0 ? t0 - eta : 0;
+    const int nband = (int)(t1 - jlo);
+    const int ntb = (nband + KT - 1) / KT, ntc = (nK + KT - 1) / KT;
+    const uint32_t id_s = umma::idesc_bf16(128, KT, false, false);
+    const uint32_t id_pv = umma::idesc_bf16(128, d, false, true);
+    const bf16 *phiK = (const bf16 *)P.phiK + (size_t)st * (lam + dm.R + dm.Nmax) * D;
+
+    for (int tile = 0; tile < ntb + ntc && ok; ++tile) {
+        const bool band = tile < ntb;
+        const long long kb = band ? jlo + (long long)tile * KT : (long long)(tile - ntb) * KT;
+        const int nk = band ? (int)min((long long)KT, t1 - kb) : min(KT, nK - (int)kb);
+        // key metadata
+        if (tid == 0) anylin = 0;
+        __syncthreads();
+        if (tid < KT) {
+            int tok = -1, info = INFO_SKIP;
+            if (tid < nk) {
+                if (band) {
+                    const long long j = kb + tid;
+                    tok = (int)j;
+                    info = (j < t1 - eta) ? (llf[(int)(j - (t0 - eta))] ? INFO_FOLDED : INFO_SKIP) : INFO_SOFT;
+                    if (info == INFO_FOLDED) anylin = 1;
+                } else {
+                    tok = ltok[kb + tid];
+                    info = INFO_SOFT;
+                }
+            }
+            ktok[tid] = tok;
+            kinfo[tid] = info;
+        }
+        __syncthreads();
+        const bool lin = anylin != 0;
+        // K (K-major [key][d]), V (N-contiguous [key][d]) and, for linear keys, phi(K)
+        for (int e = tid; e < KT * (d / 8); e += kThreads) {
+            const int j = e / (d / 8), kc = e % (d / 8);
+            uint8_t *dk = sK + umma::kmajor_offset(j, kc * 8, KT);
+            uint8_t *dv = sV + umma::mnmajor_offset(j, kc * 8, d);
+            if (j < nk) {
+                const int vr = band ? src.tok2vrow(kb + j) : lvrow[kb + j];
+                umma::cp_async16(dk, src.krow(st, vr) + kc * 8);
+                umma::cp_async16(dv, src.vrow(st, vr) + kc * 8);
+            } else {
+                *(uint4 *)dk = make_uint4(0, 0, 0, 0);
+                *(uint4 *)dv = make_uint4(0, 0, 0, 0);
+            }
+        }
+        if (lin) {
+            for (int e = tid; e < KT * (FP / 8); e += kThreads) {
+                const int j = e / (FP / 8), kc = e % (FP / 8);
+                uint8_t *dst = sPhk + umma::kmajor_offset(j, kc * 8, KT);
+                if (j < nk && kc * 8 < D) umma::cp_async16(dst, phiK + (size_t)src.tok2vrow(kb + j) * D + kc * 8);
+                else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+            }
+        }
+        umma::cp_async_commit();
+        umma::cp_async_wait_all();
+        umma::fence_async_smem();
+        umma::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            umma::fence_after_sync();
+            const uint32_t q0 = umma::smem_u32(sQ), k0 = umma::smem_u32(sK);
+            for (int ks = 0; ks < d / 16; ++ks)
+                umma::mma_ss(tS, umma::kmajor_desc(q0, ks, 128), umma::kmajor_desc(k0, ks, KT), id_s, ks > 0 ? 1u : 0u);
+            if (lin) {
+                const uint32_t pq0 = umma::smem_u32(sPhq), pk0 = umma::smem_u32(sPhk);
+                for (int ks = 0; ks < FP / 16; ++ks)
+                    umma::mma_ss(tG, umma::kmajor_desc(pq0, ks, 128), umma::kmajor_desc(pk0, ks, KT), id_s,
+                                 ks > 0 ? 1u : 0u);
+            }
+            umma::mma_commit(&mbar);
+        }
+        if (!(ok = wait_mbar(&mbar, phase, &okflag))) break;
+
+        // softmax / linear weights of row `tid`
+        float sv[KT];
+#pragma unroll
+        for (int c0 = 0; c0 < KT; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tS + lane_off + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) sv[c0 + i] = v[i] * scale;
+        }
+        float tmax = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < KT; ++j) {
+            const int info = kinfo[j], tok = ktok[j];
+            const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
+            if (soft) tmax = fmaxf(tmax, sv[j]);
+        }
+        if (tmax > m) {
+            const float f = __expf(m - tmax);
+            l *= f;
+            for (int c0 = 0; c0 < NB; c0 += 16) {
+                float v[16];
+                umma::tmem_ld16(tO + lane_off + (uint32_t)c0, v);
+                umma::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] *= f;
+                umma::tmem_st16(tO + lane_off + (uint32_t)c0, v);
+            }
+            umma::tmem_wait_st();
+            m = tmax;
+        }
+        const float em = __expf(-m);
+        float gv[KT];
+        if (lin) {
+#pragma unroll
+            for (int c0 = 0; c0 < KT; c0 += 16) {
+                float v[16];
+                umma::tmem_ld16(tG + lane_off + (uint32_t)c0, v);
+                umma::tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) gv[c0 + i] = v[i];
+            }
+        }
+        float rs = 0.f;
+#pragma unroll
+        for (int j0 = 0; j0 < KT; j0 += 8) {
+            __align__(16) bf16 pk[8];
+#pragma unroll
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = j0 + jj;
+                const int info = kinfo[j], tok = ktok[j];
+                float pw = 0.f;
+                if (info != INFO_SKIP && tok <= p) {
+                    if (info == INFO_FOLDED && tok <= p - eta) pw = lin ? gv[j] * em : 0.f;
+                    else pw = __expf(sv[j] - m);
+                }
+                if (!row_ok) pw = 0.f;
+                const bf16 pb = __float2bfloat16_rn(pw);
+                rs += __bfloat162float(pb);
+                pk[jj] = pb;
+            }
+            *(uint4 *)(sP + umma::kmajor_offset(tid, j0, 128)) = *(const uint4 *)pk;
+        }
+        l += rs;
+        umma::fence_async_smem();
+        umma::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            umma::fence_after_sync();
+            const uint32_t p0 = umma::smem_u32(sP), v0 = umma::smem_u32(sV);
+            for (int ks = 0; ks < KT / 16; ++ks)
+                umma::mma_ss(tO, umma::kmajor_desc(p0, ks, 128), umma::mnmajor_desc(v0, ks, d), id_pv, 1u);
+            umma::mma_commit(&mbar);
+        }
+        if (!(ok = wait_mbar(&mbar, phase, &okflag))) break;
+    }
+
+    if (ok) {
+        // ---- 3. normalise and store
+        float den_lin;
+        {
+            float v[16];
+            umma::tmem_ld16(tO + lane_off + (uint32_t)d, v);
+            umma::tmem_wait_ld();
+            den_lin = v[0];
+        }
+        const float den = l + den_lin + dm.eps * __expf(-m);
+        const float rden = 1.f / den;
+        bf16 *out = (bf16 *)a.out;
+        const size_t orow = qrow0 + (size_t)(grow / gq) * dm.Hq + grow % gq;
+        for (int c0 = 0; c0 < d; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tO + lane_off + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+            if (row_ok) {
+                __align__(16) bf16 o[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) o[i] = __float2bfloat16_rn(v[i] * rden);
+                *(uint4 *)(out + orow * d + c0) = *(const uint4 *)o;
+                *(uint4 *)(out + orow * d + c0 + 8) = *(const uint4 *)(o + 8);
+            }
+        }
+    } else if (tid == 0) {
+        raise_error(S.err, ERR_TIMEOUT);
+        umma::mbar_wait(&mbar, phase ^ 1u, kPolls);
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(tm, g.ncols);
+}
+
+}  // namespace
+
+size_t attn_tc_smem_bytes(const Dims &dm) { return make_ageo(dm).total; }
+
+void launch_attn_tc(const Dims &dm, const DevState &S, const PrefillScratch &P, const AttnArgs &a,
+                    cudaStream_t stream)
+{
+    KVSrc<bf16> src{(const bf16 *)S.KS, (const bf16 *)S.VS, (const bf16 *)S.KR, (const bf16 *)S.VR,
+                    (const bf16 *)a.kin, (const bf16 *)a.vin, dm.lam, dm.R, a.n_call, dm.Hkv, dm.d,
+                    a.pos0};
+    const int tiles_per_int = (dm.C * dm.g + 127) / 128;
+    dim3 grid(a.m * tiles_per_int, dm.ns);
+    const size_t smem = make_ageo(dm).total;
+    cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    attn_tc_kernel<<<grid, kThreads, smem, stream>>>(dm, S, P, a, src);
+}
+
+}  // namespace lola

@@ -68,7 +68,7 @@ __device__ __forceinline__ unsigned long long make_key(float sre, int tok)
 
 // H += sum phi(k_t) v_t^T, s += sum phi(k_t) over the listed virtual rows.
 template <typename T>
-__device__ void fold_rows(const int *lst, int cnt, const float *__restrict__ phi_st,
+__device__ void fold_rows(const int *lst, int cnt, const T *__restrict__ phi_st,
                           const KVSrc<T> &src, int st, float *__restrict__ H,
                           float *__restrict__ s, float *stgPhi, float *stgV, int D, int d)
 {
@@ -77,7 +77,7 @@ __device__ void fold_rows(const int *lst, int cnt, const float *__restrict__ phi
         const int nf = min(kFoldTile, cnt - base);
         for (int e = tid; e < nf * D; e += nt) {
             const int t = e / D, i = e - t * D;
-            stgPhi[t * D + i] = phi_st[(size_t)lst[base + t] * D + i];
+            stgPhi[t * D + i] = to_f<T>(phi_st[(size_t)lst[base + t] * D + i]);
         }
         for (int e = tid; e < nf * d; e += nt) {
             const int t = e / d, c = e - t * d;
@@ -127,7 +127,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     float *H = S.H + (size_t)st * D * d;
     float *s = S.s + (size_t)st * D;
-    const float *phi_st = a.phi + (size_t)st * a.nvrows * D;
+    const T *phi_st = (const T *)a.phi + (size_t)st * a.nvrows * D;
 
     int nS = a.nS0;
     for (int i = tid; i < lam; i += nt) {
@@ -175,13 +175,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         //    Self-Recall Error against the state at the interval start
         const int nDu = D >> 5, ndu = d >> 5;
         for (int c = warp; c < nQ; c += nw) {
-            const float *ph = phi_st + (size_t)cvrow[c] * D;
+            const T *ph = phi_st + (size_t)cvrow[c] * D;
             float phr[8];
             float den = 0.f;
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 if (u < nDu) {
-                    phr[u] = ph[lane + 32 * u];
+                    phr[u] = to_f<T>(ph[lane + 32 * u]);
                     den = fmaf(phr[u], s[lane + 32 * u], den);
                 } else {
                     phr[u] = 0.f;
@@ -287,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // move the new members' rows from the ring into their cache slots
             T *KS = (T *)S.KS + (size_t)st * lam * d;
             T *VS = (T *)S.VS + (size_t)st * lam * d;
-            float *phiV = S.phiV + (size_t)st * a.nvrows * D;
+            T *phiV = (T *)S.phiV + (size_t)st * a.nvrows * D;
             for (int c = warp; c < nL; c += nw) {
                 if (!tmpA[c] || tmpB[c] >= nE + (lam - nS)) continue;
                 const int slot = freeSlot[tmpB[c]];

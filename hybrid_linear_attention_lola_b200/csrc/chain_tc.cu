@@ -1,0 +1,643 @@
+// Tensor-core version of the sequential part of LoLA's update interval
+// (gist.science technical summary, "Inferentiestrategie"; the Self-Recall Error
+// of "Het Self-Recall Error (SRE) Mechanisme") for bfloat16 inputs. One CTA per
+// (batch, kv-head) stream walks the stream's intervals in order.
+//
+// The fp32 state lives in TMEM for the whole call: feature f of block
+// bk = f / 128 is TMEM lane f % 128, columns [bk*NB, bk*NB + d) hold H[f][:],
+// column bk*NB + d holds s[f] (NB = d + 16). Both folds are tcgen05 MMAs that
+// accumulate into it:  H_blk += Phi_F^T [V_F | 1 | 0]  (A = features x tokens,
+// B = [value dims + ones column] x tokens, both K-major over tokens). After each
+// fold a bf16 image of [H | s] is written to shared memory in the K-major
+// layout (rows = value dims + normaliser, K = features); the SRE of 128
+// candidates at a time is then one MMA chain  Phi_Q [H | s]  into TMEM, and one
+// thread per candidate finishes || num / (den + eps) - v ||^2. The kept set is
+// the nK smallest order-preserving keys (SRE bits inverted, token index), found
+// by an 8-pass radix select. Prefill mode stores the image after the eviction
+// fold as the interval's snapshot for the attention kernel.
+#include "lola_internal.cuh"
+#include "umma.cuh"
+
+namespace lola {
+
+namespace {
+
+using bf16 = __nv_bfloat16;
+constexpr int kThreads = 256;
+constexpr int kFoldTok = 64;
+constexpr uint32_t kPolls = 1u << 26;
+
+struct Geo {
+    int D, d, NB, NBa, FP, nblk, lam, Lmax, QC;
+    uint32_t ncols;
+    size_t off_X, off_keys, off_rank, off_lst, off_slotTok, off_slotVrow, off_free, off_keep,
+        off_flag, off_lf, off_hist, off_scal, total;
+};
+
+__host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+__host__ __device__ inline Geo make_geo(const Dims &dm)
+{
+    Geo g{};
+    g.D = dm.D;
+    g.d = dm.d;
+    g.NB = dm.d + 16;
+    g.NBa = (g.NB + 31) / 32 * 32;  // TMEM column stride of each accumulator
+    g.FP = (dm.D + 127) / 128 * 128;
+    g.nblk = g.FP / 128;
+    g.lam = dm.lam;
+    g.Lmax = dm.Lmax;
+    g.QC = dm.lam + dm.Lmax;
+    const uint32_t need = (uint32_t)((g.nblk + 1) * g.NBa);
+    g.ncols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
+    size_t o = (size_t)g.NB * g.FP * 2;                      // Bimg
+    g.off_X = al(o, 1024);
+    const size_t xa = (size_t)128 * g.FP * 2;
+    const size_t xf = (size_t)g.nblk * 128 * kFoldTok * 2 + (size_t)g.NB * kFoldTok * 2;
+    o = g.off_X + (xa > xf ? xa : xf);
+    g.off_keys = al(o, 16);
+    o = g.off_keys + (size_t)g.QC * 8;
+    g.off_rank = o;
+    o += (size_t)g.QC * 4;
+    g.off_lst = o;
+    o += (size_t)g.QC * 4;
+    g.off_slotTok = o;
+    o += (size_t)g.lam * 4;
+    g.off_slotVrow = o;
+    o += (size_t)g.lam * 4;
+    g.off_free = o;
+    o += (size_t)g.lam * 4;
+    g.off_keep = o;
+    o += (size_t)g.QC;
+    g.off_flag = o;
+    o += (size_t)g.QC;
+    g.off_lf = o;
+    o += (size_t)g.Lmax;
+    g.off_hist = al(o, 16);
+    o = g.off_hist + 256 * 4;
+    g.off_scal = o;
+    o += 64 * 4;
+    g.total = o + 1024;  // alignment slack for the 1024-byte aligned base
+    if (g.ncols == 512 && g.total < 116 * 1024) g.total = 116 * 1024;  // one CTA per SM
+    return g;
+}
+
+template <typename F>
+__device__ int scan_excl(const F *in, int *out, int n, int *wsum)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    const int nwarps = nt >> 5;
+    const int per = (n + nt - 1) / nt;
+    const int beg = min(n, tid * per), end = min(n, beg + per);
+    int local = 0;
+    for (int i = beg; i < end; ++i) local += (int)in[i];
+    int x = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) wsum[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int w = lane < nwarps ? wsum[lane] : 0;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += y;
+        }
+        if (lane < nwarps) wsum[lane] = w;
+    }
+    __syncthreads();
+    int run = (warp > 0 ? wsum[warp - 1] : 0) + x - local;
+    for (int i = beg; i < end; ++i) {
+        out[i] = run;
+        run += (int)in[i];
+    }
+    const int total = wsum[nwarps - 1];
+    __syncthreads();
+    return total;
+}
+
+__device__ __forceinline__ unsigned long long make_key(float sre, int tok)
+{
+    const unsigned bits = __float_as_uint(fmaxf(sre, 0.f));
+    return ((unsigned long long)(0xFFFFFFFFu - bits) << 32) | (unsigned)tok;
+}
+
+// The k-th smallest (1-based) of n distinct 64-bit keys, 8 bits per pass.
+__device__ unsigned long long radix_select(const unsigned long long *keys, int n, int k, int *hist,
+                                           int *scal)
+{
+    const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
+    unsigned long long prefix = 0, mask = 0;
+    int rank = k;
+    for (int shift = 56; shift >= 0; shift -= 8) {
+        for (int i = tid; i < 256; i += nt) hist[i] = 0;
+        __syncthreads();
+        for (int c = tid; c < n; c += nt) {
+            const unsigned long long kk = keys[c];
+            if ((kk & mask) == prefix) atomicAdd(&hist[(int)((kk >> shift) & 255u)], 1);
+        }
+        __syncthreads();
+        if (warp == 0) {
+            int loc[8], s = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+                loc[j] = hist[lane * 8 + j];
+                s += loc[j];
+            }
+            int incl = s;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            const int excl = incl - s;
+            if (excl < rank && rank <= incl) {
+                int cum = excl;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    if (cum + loc[j] >= rank) {
+                        scal[0] = lane * 8 + j;
+                        scal[1] = rank - cum;
+                        break;
+                    }
+                    cum += loc[j];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= (unsigned long long)scal[0] << shift;
+        mask |= (unsigned long long)255u << shift;
+        rank = scal[1];
+        __syncthreads();
+    }
+    return prefix;
+}
+
+struct Ctx {
+    Geo g;
+    uint8_t *Bimg, *X;
+    uint32_t tm;           // TMEM base
+    uint64_t *mbar;
+    int *okflag;
+    uint32_t phase;
+};
+
+__device__ __forceinline__ uint32_t tH(const Ctx &c, int bk) { return c.tm + (uint32_t)(bk * c.g.NBa); }
+__device__ __forceinline__ uint32_t tS(const Ctx &c) { return c.tm + (uint32_t)(c.g.nblk * c.g.NBa); }
+
+__device__ bool wait_mma(Ctx &c)
+{
+    if (threadIdx.x == 0) *c.okflag = umma::mbar_wait(c.mbar, c.phase, kPolls) ? 1 : 0;
+    __syncthreads();
+    c.phase ^= 1u;
+    umma::fence_after_sync();
+    return *c.okflag != 0;
+}
+
+// bf16 image of [H | s] (K-major: row n = value dim / normaliser, K = feature).
+__device__ void refresh_image(Ctx &c)
+{
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = warp & 3;
+    for (int bk = warp >> 2; bk < c.g.nblk; bk += kThreads / 128) {
+        const int f = bk * 128 + q * 32 + lane;
+        for (int c0 = 0; c0 < c.g.NB; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tH(c, bk) + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+                *(bf16 *)(c.Bimg + umma::kmajor_offset(c0 + i, f, c.g.NB)) = __float2bfloat16_rn(v[i]);
+        }
+    }
+    umma::fence_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+}
+
+// H += sum phi(k) v^T, s += sum phi(k) over the listed virtual rows, on the tensor cores.
+__device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict__ phi_st,
+                        const KVSrc<bf16> &src, int st)
+{
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = kThreads >> 5;
+    const Geo &g = c.g;
+    uint8_t *Af = c.X;
+    uint8_t *Bf = c.X + (size_t)g.nblk * 128 * kFoldTok * 2;
+    const uint32_t idesc = umma::idesc_bf16(128, g.NB, false, false);
+    for (int base = 0; base < cnt; base += kFoldTok) {
+        const int nt = min(kFoldTok, cnt - base);
+        const int ntp = (nt + 15) & ~15;
+        // zero the padded token columns and the padded feature rows
+        for (int e = tid; e < g.FP * (ntp - nt); e += kThreads) {
+            const int f = e / (ntp - nt), t = nt + e % (ntp - nt);
+            *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 + umma::kmajor_offset(f & 127, t, 128)) =
+                __float2bfloat16_rn(0.f);
+        }
+        for (int e = tid; e < (g.FP - g.D) * nt; e += kThreads) {
+            const int f = g.D + e / nt, t = e % nt;
+            *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 + umma::kmajor_offset(f & 127, t, 128)) =
+                __float2bfloat16_rn(0.f);
+        }
+        for (int e = tid; e < g.NB * (ntp - nt); e += kThreads) {
+            const int n = e / (ntp - nt), t = nt + e % (ntp - nt);
+            *(bf16 *)(Bf + umma::kmajor_offset(n, t, g.NB)) = __float2bfloat16_rn(0.f);
+        }
+        // one warp per token: phi row -> column t of A, [v | 1 | 0] -> column t of B
+        for (int t = warp; t < nt; t += nw) {
+            const int vr = lst[base + t];
+            const bf16 *ph = phi_st + (size_t)vr * g.D;
+            for (int f0 = lane * 8; f0 < g.D; f0 += 256) {
+                const uint4 raw = *(const uint4 *)(ph + f0);
+                const bf16 *pv = (const bf16 *)&raw;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int f = f0 + j;
+                    *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 +
+                              umma::kmajor_offset(f & 127, t, 128)) = pv[j];
+                }
+            }
+            const bf16 *vv = src.vrow(st, vr);
+            for (int c0 = lane * 8; c0 < g.d; c0 += 256) {
+                const uint4 raw = *(const uint4 *)(vv + c0);
+                const bf16 *pv = (const bf16 *)&raw;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) *(bf16 *)(Bf + umma::kmajor_offset(c0 + j, t, g.NB)) = pv[j];
+            }
+            for (int n = g.d + lane; n < g.NB; n += 32)
+                *(bf16 *)(Bf + umma::kmajor_offset(n, t, g.NB)) = __float2bfloat16_rn(n == g.d ? 1.f : 0.f);
+        }
+        umma::fence_async_smem();
+        umma::fence_before_sync();
+        __syncthreads();
+        if (tid == 0) {
+            umma::fence_after_sync();
+            const uint32_t b0 = umma::smem_u32(Bf);
+            for (int bk = 0; bk < g.nblk; ++bk) {
+                const uint32_t a0 = umma::smem_u32(Af + (size_t)bk * 128 * kFoldTok * 2);
+                for (int ks = 0; ks < ntp / 16; ++ks)
+                    umma::mma_ss(tH(c, bk), umma::kmajor_desc(a0, ks, 128),
+                                 umma::kmajor_desc(b0, ks, g.NB), idesc, 1u);
+            }
+            umma::mma_commit(c.mbar);
+        }
+        if (!wait_mma(c)) return false;
+    }
+    return true;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+    chain_tc_kernel(Dims dm, DevState S, PrefillScratch P, ChainArgs a, KVSrc<bf16> src)
+{
+    const int st = blockIdx.x;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const Geo g = make_geo(dm);
+    const int D = g.D, d = g.d, lam = g.lam, eta = dm.eta, Lmax = g.Lmax;
+
+    extern __shared__ uint8_t smraw[];
+    __shared__ uint64_t mbar;
+    __shared__ uint32_t tslot;
+    __shared__ int okflag;
+    const uint32_t raw = umma::smem_u32(smraw);
+    uint8_t *base = smraw + (((raw + 1023u) & ~1023u) - raw);
+    Ctx c;
+    c.g = g;
+    c.Bimg = base;
+    c.X = base + g.off_X;
+    unsigned long long *keys = (unsigned long long *)(base + g.off_keys);
+    int *rank = (int *)(base + g.off_rank);
+    int *lst = (int *)(base + g.off_lst);
+    int *slotTok = (int *)(base + g.off_slotTok);
+    int *slotVrow = (int *)(base + g.off_slotVrow);
+    int *freeSlot = (int *)(base + g.off_free);
+    uint8_t *keep = base + g.off_keep;
+    uint8_t *flag = base + g.off_flag;
+    uint8_t *lf = base + g.off_lf;
+    int *hist = (int *)(base + g.off_hist);
+    int *scal = (int *)(base + g.off_scal);
+    c.mbar = &mbar;
+    c.okflag = &okflag;
+    c.phase = 0;
+
+    if (tid == 0) umma::mbar_init(&mbar, 1);
+    if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
+    umma::fence_before_sync();
+    __syncthreads();
+    umma::fence_after_sync();
+    c.tm = tslot;
+
+    float *Hg = S.H + (size_t)st * D * d;
+    float *sg = S.s + (size_t)st * D;
+    const bf16 *phi_st = (const bf16 *)a.phi + (size_t)st * a.nvrows * D;
+
+    // state -> TMEM (rows past D and columns past d+1 are zero)
+    {
+        const int q = warp & 3;
+        for (int bk = warp >> 2; bk < g.nblk; bk += kThreads / 128) {
+            const int f = bk * 128 + q * 32 + lane;
+            for (int c0 = 0; c0 < g.NB; c0 += 16) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int col = c0 + i;
+                    v[i] = f < D ? (col < d ? Hg[(size_t)f * d + col] : (col == d ? sg[f] : 0.f)) : 0.f;
+                }
+                umma::tmem_st16(tH(c, bk) + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+            }
+        }
+        umma::tmem_wait_st();
+        umma::fence_before_sync();
+        __syncthreads();
+        umma::fence_after_sync();
+    }
+    refresh_image(c);
+
+    int nS = a.nS0;
+    for (int i = tid; i < lam; i += kThreads) {
+        slotTok[i] = i < nS ? S.idxS[(size_t)st * lam + i] : -1;
+        slotVrow[i] = i;
+    }
+    for (int i = tid; i < Lmax; i += kThreads) lf[i] = i < a.pend_n ? S.pend[(size_t)st * Lmax + i] : 0;
+    long long pend_lo = a.pend_lo;
+    int pend_n = a.pend_n;
+    __syncthreads();
+
+    bool ok = true;
+    const uint32_t idesc_sre = umma::idesc_bf16(128, g.NB, false, false);
+    for (int ci = 0; ci < a.n_int && ok; ++ci) {
+        const long long t0 = a.pos0 + (long long)ci * a.ilen;
+        const long long t1 = t0 + a.ilen;
+        const long long iglob = a.iglob0 + ci;
+
+        // 1. fold the previous interval's leaving pairs that were not kept
+        if (pend_n > 0) {
+            const int nf = scan_excl(lf, rank, pend_n, scal);
+            for (int i = tid; i < pend_n; i += kThreads)
+                if (lf[i]) lst[rank[i]] = src.tok2vrow(pend_lo + i);
+            __syncthreads();
+            if (nf > 0) {
+                if (!(ok = fold_tc(c, lst, nf, phi_st, src, st))) break;
+                refresh_image(c);
+            }
+        }
+
+        // 2. score the candidates (cache slots, then pairs leaving in [t0, t1))
+        const long long Llo = t0 - eta > 0 ? t0 - eta : 0;
+        const long long Lhi = t1 - eta > Llo ? t1 - eta : Llo;
+        const int nL = (int)(Lhi - Llo);
+        const int nQ = nS + nL;
+        for (int m0 = 0; m0 < nQ && ok; m0 += 128) {
+            const int nr = min(128, nQ - m0);
+            const int chunks = g.FP / 8;
+            for (int e = tid; e < nr * chunks; e += kThreads) {
+                const int r = e / chunks, kc = e - r * chunks;
+                const int cand = m0 + r;
+                uint8_t *dst = c.X + umma::kmajor_offset(r, kc * 8, 128);
+                if (kc * 8 < D) {
+                    const int vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
+                    umma::cp_async16(dst, phi_st + (size_t)vr * D + kc * 8);
+                } else {
+                    *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+                }
+            }
+            umma::cp_async_commit();
+            umma::cp_async_wait_all();
+            umma::fence_async_smem();
+            umma::fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                umma::fence_after_sync();
+                const uint32_t a0 = umma::smem_u32(c.X), b0 = umma::smem_u32(c.Bimg);
+                for (int ks = 0; ks < g.FP / 16; ++ks)
+                    umma::mma_ss(tS(c), umma::kmajor_desc(a0, ks, 128), umma::kmajor_desc(b0, ks, g.NB),
+                                 idesc_sre, ks > 0 ? 1u : 0u);
+                umma::mma_commit(c.mbar);
+            }
+            if (!(ok = wait_mma(c))) break;
+            if (warp < 4) {
+                const int r = warp * 32 + lane;
+                const int cand = m0 + r;
+                const uint32_t rowaddr = tS(c) + ((uint32_t)(warp * 32) << 16);
+                float v[16];
+                umma::tmem_ld16(rowaddr + (uint32_t)d, v);
+                umma::tmem_wait_ld();
+                const float den = v[0] + dm.eps;
+                float err = 0.f;
+                int vr = 0, tok = 0;
+                if (cand < nQ) {
+                    vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
+                    tok = cand < nS ? slotTok[cand] : (int)(Llo + (cand - nS));
+                }
+                const bf16 *vv = src.vrow(st, vr);
+                for (int c0 = 0; c0 < d; c0 += 16) {
+                    umma::tmem_ld16(rowaddr + (uint32_t)c0, v);
+                    umma::tmem_wait_ld();
+                    if (cand < nQ) {
+                        const uint4 r0 = *(const uint4 *)(vv + c0);
+                        const uint4 r1 = *(const uint4 *)(vv + c0 + 8);
+                        const bf16 *p0 = (const bf16 *)&r0;
+                        const bf16 *p1 = (const bf16 *)&r1;
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float pred = den != 0.f ? v[i] / den : 0.f;
+                            const float diff = pred - __bfloat162float(i < 8 ? p0[i] : p1[i - 8]);
+                            err = fmaf(diff, diff, err);
+                        }
+                    }
+                }
+                if (cand < nQ) keys[cand] = make_key(err, tok);
+            }
+            umma::fence_before_sync();
+            __syncthreads();
+        }
+        if (!ok) break;
+
+        // 3. keep the nK smallest keys (highest SRE, lower token on ties)
+        const int nK = nQ < lam ? nQ : lam;
+        if (nQ > lam) {
+            const unsigned long long thr = radix_select(keys, nQ, nK, hist, scal);
+            for (int i = tid; i < nQ; i += kThreads) keep[i] = keys[i] <= thr ? 1 : 0;
+        } else {
+            for (int i = tid; i < nQ; i += kThreads) keep[i] = 1;
+        }
+        __syncthreads();
+        if (a.sel_log != nullptr && iglob < a.sel_cap) {
+            int32_t *lg = a.sel_log + ((size_t)iglob * dm.ns + st) * (lam + 1);
+            const int cnt = scan_excl(keep, rank, nQ, scal);
+            for (int i = tid; i < nQ; i += kThreads)
+                if (keep[i]) lg[1 + rank[i]] = i < nS ? slotTok[i] : (int)(Llo + (i - nS));
+            for (int i = cnt + tid; i < lam; i += kThreads) lg[1 + i] = -1;
+            if (tid == 0) lg[0] = cnt;
+        }
+        const int32_t *lo_ =
+            (a.ovr != nullptr && iglob < a.ovr_n) ? a.ovr + ((size_t)iglob * dm.ns + st) * (lam + 1) : nullptr;
+        if (lo_ != nullptr && lo_[0] >= 0) {
+            const int cnt = lo_[0];
+            if (tid == 0 && cnt != nK) raise_error(S.err, ERR_BOUNDS);
+            for (int i = tid; i < nQ; i += kThreads) {
+                const int key = i < nS ? slotTok[i] : (int)(Llo + (i - nS));
+                int lo = 0, hi = cnt < lam ? cnt : lam;
+                while (lo < hi) {
+                    const int mid = (lo + hi) >> 1;
+                    if (lo_[1 + mid] < key) lo = mid + 1; else hi = mid;
+                }
+                keep[i] = (lo < cnt && lo < lam && lo_[1 + lo] == key) ? 1 : 0;
+            }
+            __syncthreads();
+        }
+
+        // 4a. evicted cached pairs: fold now (the state this interval's queries read)
+        for (int i = tid; i < nS; i += kThreads) flag[i] = keep[i] ? 0 : 1;
+        __syncthreads();
+        const int nE = scan_excl(flag, rank, nS, scal);
+        for (int i = tid; i < nS; i += kThreads) {
+            if (flag[i]) {
+                lst[rank[i]] = slotVrow[i];
+                freeSlot[rank[i]] = i;
+            }
+        }
+        for (int r = nE + tid; r < nE + (lam - nS); r += kThreads) freeSlot[r] = nS + (r - nE);
+        __syncthreads();
+        if (nE > 0) {
+            if (!(ok = fold_tc(c, lst, nE, phi_st, src, st))) break;
+            refresh_image(c);
+        }
+        if (a.mode == 0 && P.snapImg != nullptr) {
+            uint4 *dst = (uint4 *)((uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * g.NB * g.FP * 2);
+            const uint4 *srcp = (const uint4 *)c.Bimg;
+            const int n16 = g.NB * g.FP * 2 / 16;
+            for (int e = tid; e < n16; e += kThreads) dst[e] = srcp[e];
+        }
+        if (a.mode == 0 && a.snap_f32) {
+            // fp32 (H', s') for the SIMT attention kernel
+            const int q = warp & 3;
+            float *sh = P.snapH + ((size_t)st * dm.mmax + ci) * D * d;
+            float *ss = P.snapS + ((size_t)st * dm.mmax + ci) * D;
+            for (int bk = warp >> 2; bk < g.nblk; bk += kThreads / 128) {
+                const int f = bk * 128 + q * 32 + lane;
+                for (int c0 = 0; c0 < g.NB; c0 += 16) {
+                    float v[16];
+                    umma::tmem_ld16(tH(c, bk) + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+                    umma::tmem_wait_ld();
+                    if (f < D) {
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const int col = c0 + i;
+                            if (col < d) sh[(size_t)f * d + col] = v[i];
+                            else if (col == d) ss[f] = v[i];
+                        }
+                    }
+                }
+            }
+        }
+
+        // 4b. kept leaving pairs take the free slots (eviction slots first, ascending)
+        const int nNew = scan_excl(keep + nS, rank, nL, scal);
+        if (tid == 0 && nNew > nE + (lam - nS)) raise_error(S.err, ERR_BOUNDS);
+        for (int i = tid; i < nL; i += kThreads) {
+            if (keep[nS + i] && rank[i] < nE + (lam - nS)) {
+                const int slot = freeSlot[rank[i]];
+                const long long tok = Llo + i;
+                slotTok[slot] = (int)tok;
+                slotVrow[slot] = a.mode == 0 ? src.tok2vrow(tok) : slot;
+            }
+        }
+        if (a.mode == 1) {
+            bf16 *KS = (bf16 *)S.KS + (size_t)st * lam * d;
+            bf16 *VS = (bf16 *)S.VS + (size_t)st * lam * d;
+            bf16 *phiV = (bf16 *)S.phiV + (size_t)st * a.nvrows * D;
+            for (int i = warp; i < nL; i += kThreads / 32) {
+                if (!keep[nS + i] || rank[i] >= nE + (lam - nS)) continue;
+                const int slot = freeSlot[rank[i]];
+                const int vr = src.tok2vrow(Llo + i);
+                const bf16 *kr = src.krow(st, vr);
+                const bf16 *vv = src.vrow(st, vr);
+                for (int e = lane; e < d; e += 32) {
+                    KS[(size_t)slot * d + e] = kr[e];
+                    VS[(size_t)slot * d + e] = vv[e];
+                }
+                for (int e = lane; e < D; e += 32) phiV[(size_t)slot * D + e] = phiV[(size_t)vr * D + e];
+                if (lane == 0) S.idxS[(size_t)st * lam + slot] = (int)(Llo + i);
+            }
+        }
+        __syncthreads();
+        if (a.mode == 0) {
+            const size_t lb = (size_t)st * dm.mmax + ci;
+            for (int i = tid; i < nK; i += kThreads) {
+                P.logTok[lb * lam + i] = slotTok[i];
+                P.logVrow[lb * lam + i] = slotVrow[i];
+            }
+            for (int i = tid; i < nL; i += kThreads)
+                P.logLf[lb * Lmax + (int)(Llo + i - (t0 - eta))] = keep[nS + i] ? 0 : 1;
+            if (tid == 0) P.logCount[lb] = nK;
+        }
+        __syncthreads();
+        for (int i = tid; i < nL; i += kThreads) lf[i] = keep[nS + i] ? 0 : 1;
+        pend_lo = Llo;
+        pend_n = nL;
+        nS = nK;
+        __syncthreads();
+    }
+
+    if (ok) {
+        // TMEM -> state
+        const int q = warp & 3;
+        for (int bk = warp >> 2; bk < g.nblk; bk += kThreads / 128) {
+            const int f = bk * 128 + q * 32 + lane;
+            for (int c0 = 0; c0 < g.NB; c0 += 16) {
+                float v[16];
+                umma::tmem_ld16(tH(c, bk) + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+                umma::tmem_wait_ld();
+                if (f < D) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int col = c0 + i;
+                        if (col < d) Hg[(size_t)f * d + col] = v[i];
+                        else if (col == d) sg[f] = v[i];
+                    }
+                }
+            }
+        }
+        for (int i = tid; i < Lmax; i += kThreads) S.pend[(size_t)st * Lmax + i] = (uint8_t)(i < pend_n ? lf[i] : 0);
+        if (a.mode == 0) {
+            for (int i = tid; i < lam; i += kThreads) {
+                P.slotTok[(size_t)st * lam + i] = slotTok[i];
+                P.slotVrow[(size_t)st * lam + i] = slotVrow[i];
+            }
+        }
+    } else {
+        if (tid == 0) {
+            raise_error(S.err, ERR_TIMEOUT);
+            umma::mbar_wait(&mbar, c.phase ^ 1u, kPolls);  // let an MMA still in flight drain
+        }
+    }
+    umma::fence_before_sync();
+    __syncthreads();
+    if (warp == 0) umma::tmem_dealloc(c.tm, g.ncols);
+}
+
+}  // namespace
+
+size_t chain_tc_smem_bytes(const Dims &dm) { return make_geo(dm).total; }
+
+size_t snap_image_bytes(const Dims &dm)
+{
+    const Geo g = make_geo(dm);
+    return (size_t)g.NB * g.FP * 2;
+}
+
+void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
+                     cudaStream_t stream)
+{
+    KVSrc<bf16> src{(const bf16 *)S.KS, (const bf16 *)S.VS, (const bf16 *)S.KR, (const bf16 *)S.VR,
+                    (const bf16 *)a.kin, (const bf16 *)a.vin, dm.lam, dm.R, a.n_call, dm.Hkv, dm.d,
+                    a.call_start};
+    const size_t smem = make_geo(dm).total;
+    cudaFuncSetAttribute(chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    PrefillScratch Pv{};
+    if (P) Pv = *P;
+    chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src);
+}
+
+}  // namespace lola

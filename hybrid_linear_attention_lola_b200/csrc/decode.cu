@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(DW * 32)
     }
     for (int e = tid; e < g * D; e += blockDim.x) {
         const int r = e / D, i = e - r * D;
-        phq[e] = S.phiQd[((size_t)b * dm.Hq + hk * g + r) * D + i];
+        phq[e] = to_f<T>(((const T *)S.phiQd)[((size_t)b * dm.Hq + hk * g + r) * D + i]);
     }
 
     const long long p = a.pos;
@@ -81,7 +81,7 @@ __global__ void __launch_bounds__(DW * 32)
     const T *VS = (const T *)S.VS + (size_t)st * lam * d;
     const T *KR = (const T *)S.KR + (size_t)st * R * d;
     const T *VR = (const T *)S.VR + (size_t)st * R * d;
-    const float *phiV = S.phiV + (size_t)st * (lam + R) * D;
+    const T *phiV = (const T *)S.phiV + (size_t)st * (lam + R) * D;
 
     for (long long tile = tb; tile < te; ++tile) {
         __syncthreads();
@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(DW * 32)
         }
         for (int e = tid; e < nk * D; e += blockDim.x) {
             const int j = e / D, i = e - j * D;
-            if (kinfo[j] == 1) phk[j * (D + 1) + i] = phiV[(size_t)krow[j] * D + i];
+            if (kinfo[j] == 1) phk[j * (D + 1) + i] = to_f<T>(phiV[(size_t)krow[j] * D + i]);
         }
         __syncthreads();
         const int mytok = lane < nk ? ktok[lane] : -1;
@@ -226,14 +226,14 @@ __global__ void decode_merge_kernel(Dims dm, DevState S, void *out_)
         }
     }
     // readout phi(q)^T H', phi(q)^T s'
-    const float *pq = S.phiQd + ((size_t)b * dm.Hq + hq) * D;
+    const T *pq = (const T *)S.phiQd + ((size_t)b * dm.Hq + hq) * D;
     const float *H = S.H + (size_t)st * D * d;
     const float *s = S.s + (size_t)st * D;
     float dd = 0.f;
-    for (int i = lane; i < D; i += 32) dd = fmaf(pq[i], s[i], dd);
+    for (int i = lane; i < D; i += 32) dd = fmaf(to_f<T>(pq[i]), s[i], dd);
     LD += warp_sum(dd);
     for (int i = 0; i < D; ++i) {
-        const float f = pq[i];
+        const float f = to_f<T>(pq[i]);
 #pragma unroll
         for (int w = 0; w < 4; ++w)
             if (w < ndu) nln[w] = fmaf(f, H[(size_t)i * d + lane + 32 * w], nln[w]);

@@ -24,6 +24,8 @@ struct Dims {
     int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
     int Nmax, mmax;   // prefill scratch capacity: tokens per call, intervals per call
     int nsplit;       // decode key splits per stream
+    int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
+    int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
     float eps;
 };
 
@@ -37,16 +39,17 @@ struct DevState {
     uint8_t *pend;     // [ns][Lmax]   1 = leaving pair of the last interval that is folded
     float *W;          // [d][Dh]      feature-map matrix, fp32 copy
     int *err;          // [4]          device error words
-    // decode scratch
-    float *phiV;       // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
-    float *phiQd;      // [B][Hq][D]
+    // decode scratch (phi buffers hold the input dtype)
+    void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
+    void *phiQd;       // [B][Hq][D]
     float *part;       // [ns][nsplit][g][2d + 4] split partials
 };
 
 // Per-prefill-call scratch.
 struct PrefillScratch {
-    float *phiK;       // [ns][lam + R + Nmax][D]
-    float *phiQ;       // [B][Nmax][Hq][D]
+    void *phiK;        // [ns][lam + R + Nmax][D]  (input dtype)
+    void *phiQ;        // [B][Nmax][Hq][D]         (input dtype)
+    void *snapImg;     // [ns][mmax][NB x FP] bf16 K-major image of [H'|s'] (tensor-core path)
     float *snapH;      // [ns][mmax][D][d]  H' of each interval (after the cache eviction fold)
     float *snapS;      // [ns][mmax][D]
     int *logTok;       // [ns][mmax][lam]   kept set of each interval (token)
@@ -123,9 +126,9 @@ __device__ __forceinline__ void raise_error(int *err, int code)
 // ---- host launch wrappers (defined in the .cu files) ----
 void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream);
 void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long call_start,
-                   int n, int nvrows, int row_begin_call, float *phi_out, int nS,
+                   int n, int nvrows, int row_begin_call, void *phi_out, int nS,
                    cudaStream_t stream);
-void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, float *phi_out,
+void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, void *phi_out,
                   cudaStream_t stream);
 
 struct ChainArgs {
@@ -139,13 +142,19 @@ struct ChainArgs {
     long long pend_lo;      // pending leaving range of the previous interval
     int pend_n;
     long long iglob0;       // interval counter of the first interval
-    const float *phi;       // [ns][nvrows][D]
+    const void *phi;        // [ns][nvrows][D] (input dtype)
     int nvrows;
     int32_t *sel_log;       // test hook, may be null
     long long sel_cap;
     const int32_t *ovr;     // test hook, may be null
     long long ovr_n;
+    int snap_f32;           // prefill: also write fp32 (H', s') snapshots
 };
+void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
+                     cudaStream_t stream);
+size_t chain_tc_smem_bytes(const Dims &dm);
+size_t attn_tc_smem_bytes(const Dims &dm);
+size_t snap_image_bytes(const Dims &dm);
 void launch_chain(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
                   cudaStream_t stream);
 
@@ -158,6 +167,8 @@ struct AttnArgs {
 };
 void launch_attn_prefill(const Dims &dm, const DevState &S, const PrefillScratch &P,
                          const AttnArgs &a, cudaStream_t stream);
+void launch_attn_tc(const Dims &dm, const DevState &S, const PrefillScratch &P, const AttnArgs &a,
+                    cudaStream_t stream);
 void launch_finalize_prefill(const Dims &dm, const DevState &S, const PrefillScratch &P,
                              const void *kin, const void *vin, long long call_start, int n,
                              int nK, cudaStream_t stream);

@@ -11,7 +11,7 @@ namespace lola {
 template <typename T>
 __device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const float *__restrict__ Ws,
                                              float *__restrict__ xs, int d, int Dh,
-                                             float *__restrict__ out)
+                                             T *__restrict__ out)
 {
     const int lane = threadIdx.x & 31;
     for (int a = lane; a < d; a += 32) xs[a] = to_f<T>(x[a]);
@@ -54,8 +54,8 @@ __device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const floa
     for (int u = 0; u < 4; ++u) {
         const int i = lane + 32 * u;
         if (i < Dh) {
-            out[i] = ep[u] * rp;
-            out[Dh + i] = en[u] * rn;
+            out[i] = from_f<T>(ep[u] * rp);
+            out[Dh + i] = from_f<T>(en[u] * rn);
         }
     }
     __syncwarp();
@@ -64,7 +64,7 @@ __device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const floa
 template <typename T>
 __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, const float *__restrict__ W,
                                                      int nS, int n, int nvrows,
-                                                     float *__restrict__ phi_out)
+                                                     T *__restrict__ phi_out)
 {
     extern __shared__ float sm[];
     float *Ws = sm;                                   // [d][Dh]
@@ -87,7 +87,7 @@ __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, cons
 template <typename T>
 __global__ void __launch_bounds__(256) phi_q_kernel(int d, int Dh, const float *__restrict__ W,
                                                     const T *__restrict__ q, long long rows,
-                                                    float *__restrict__ phi_out)
+                                                    T *__restrict__ phi_out)
 {
     extern __shared__ float sm[];
     float *Ws = sm;
@@ -108,7 +108,7 @@ static int grid_for(long long rows, int warps_per_block)
 }
 
 void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long call_start,
-                   int n, int nvrows, int /*row_begin_call*/, float *phi_out, int nS,
+                   int n, int nvrows, int /*row_begin_call*/, void *phi_out, int nS,
                    cudaStream_t stream)
 {
     const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
@@ -119,7 +119,8 @@ void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long
         KVSrc<float> src{(const float *)S.KS, (const float *)S.VS, (const float *)S.KR,
                          (const float *)S.VR, (const float *)kin, nullptr,
                          dm.lam, dm.R, n, dm.Hkv, dm.d, call_start};
-        phi_kv_kernel<float><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows, phi_out);
+        phi_kv_kernel<float><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows,
+                                                          (float *)phi_out);
     } else {
         cudaFuncSetAttribute(phi_kv_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
@@ -128,11 +129,11 @@ void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long
                                  (const __nv_bfloat16 *)kin, nullptr,
                                  dm.lam, dm.R, n, dm.Hkv, dm.d, call_start};
         phi_kv_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(dm, src, S.W, nS, n, nvrows,
-                                                                  phi_out);
+                                                                  (__nv_bfloat16 *)phi_out);
     }
 }
 
-void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, float *phi_out,
+void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, void *phi_out,
                   cudaStream_t stream)
 {
     const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
@@ -140,12 +141,12 @@ void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows,
     if (dm.dtype == 0) {
         cudaFuncSetAttribute(phi_q_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         phi_q_kernel<float><<<grid, 256, smem, stream>>>(dm.d, dm.Dh, W, (const float *)q, rows,
-                                                         phi_out);
+                                                         (float *)phi_out);
     } else {
         cudaFuncSetAttribute(phi_q_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         phi_q_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(
-            dm.d, dm.Dh, W, (const __nv_bfloat16 *)q, rows, phi_out);
+            dm.d, dm.Dh, W, (const __nv_bfloat16 *)q, rows, (__nv_bfloat16 *)phi_out);
     }
 }
 

@@ -66,13 +66,14 @@ def test_static_decode_matches_decode_step_twice():
 
 
 def test_static_decode_rejects_scratch_beyond_limit():
-    # 64 sequences x 64 query heads x feat_dim 256 need more than the 8 MiB array
-    cfg = L.make_config(batch=64, n_q_heads=64, n_kv_heads=8, head_dim=128, feat_dim=256,
+    # 128 sequences x 64 query heads (8 per kv-head), head_dim 128, feat_dim 256:
+    # query features 4 MiB + split partials 8.5 MB exceed the 8 MiB array
+    cfg = L.make_config(batch=128, n_q_heads=64, n_kv_heads=8, head_dim=128, feat_dim=256,
                         window=1, lambda_=0, chunk=1, decode_interval=1, max_prefill_tokens=1,
                         eps=1e-6, dtype="bf16")
     S = L.LolaState(cfg, torch.zeros(128, 128), torch.device("cuda"))
-    x = torch.zeros((64, 64, 128), dtype=torch.bfloat16, device="cuda")
-    kv = torch.zeros((64, 8, 128), dtype=torch.bfloat16, device="cuda")
+    x = torch.zeros((128, 64, 128), dtype=torch.bfloat16, device="cuda")
+    kv = torch.zeros((128, 8, 128), dtype=torch.bfloat16, device="cuda")
     stream = torch.cuda.current_stream().cuda_stream
     with pytest.raises(L.LolaError) as ei:
         L.lola_decode_step_static(S.handle, x.data_ptr(), kv.data_ptr(), kv.data_ptr(),
