@@ -27,7 +27,7 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int kThreads = 128;
 constexpr int KT = 64;                // keys per tile
-constexpr uint32_t kPolls = 1u << 26;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
 
 struct AGeo {
@@ -66,9 +66,16 @@ __host__ __device__ inline AGeo make_ageo(const Dims &dm)
     return g;
 }
 
-__device__ __forceinline__ bool wait_mbar(uint64_t *mbar, uint32_t &phase, int *okflag)
+// Thread 0 waits for the MMA completion (bounded); a timeout anywhere in the
+// grid sets the device error word, after which every CTA stops waiting.
+__device__ __forceinline__ bool wait_mbar(uint64_t *mbar, uint32_t &phase, int *okflag, int *err)
 {
-    if (threadIdx.x == 0) *okflag = umma::mbar_wait(mbar, phase, kPolls) ? 1 : 0;
+    if (threadIdx.x == 0) {
+        const bool aborted = (*(volatile int *)err & ERR_TIMEOUT) != 0;
+        const bool ok = !aborted && umma::mbar_wait(mbar, phase, kWaitNs);
+        if (!ok) raise_error(err, ERR_TIMEOUT);
+        *okflag = ok ? 1 : 0;
+    }
     __syncthreads();
     phase ^= 1u;
     umma::fence_after_sync();
@@ -160,7 +167,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::mma_ss(tO, umma::kmajor_desc(a0, ks, 128), umma::kmajor_desc(b0, ks, NB), id, ks > 0 ? 1u : 0u);
         umma::mma_commit(&mbar);
     }
-    ok = wait_mbar(&mbar, phase, &okflag);
+    ok = wait_mbar(&mbar, phase, &okflag, S.err);
 
     float m = 0.f, l = 0.f;
     const size_t lb = (size_t)st * dm.mmax + ci;
@@ -240,7 +247,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma::mma_commit(&mbar);
         }
-        if (!(ok = wait_mbar(&mbar, phase, &okflag))) break;
+        if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
 
         // softmax / linear weights of row `tid`
         float sv[KT];
@@ -259,8 +266,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
             if (soft) tmax = fmaxf(tmax, sv[j]);
         }
-        if (tmax > m) {
-            const float f = __expf(m - tmax);
+        // rescale this row's accumulator when its shift grows; TMEM loads and
+        // stores are warp-collective, so the whole warp takes the branch
+        const bool grow_m = tmax > m;
+        if (__any_sync(0xffffffffu, grow_m)) {
+            const float f = grow_m ? __expf(m - tmax) : 1.f;
             l *= f;
             for (int c0 = 0; c0 < NB; c0 += 16) {
                 float v[16];
@@ -271,7 +281,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::tmem_st16(tO + lane_off + (uint32_t)c0, v);
             }
             umma::tmem_wait_st();
-            m = tmax;
+            if (grow_m) m = tmax;
         }
         const float em = __expf(-m);
         float gv[KT];
@@ -316,7 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::mma_ss(tO, umma::kmajor_desc(p0, ks, 128), umma::mnmajor_desc(v0, ks, d), id_pv, 1u);
             umma::mma_commit(&mbar);
         }
-        if (!(ok = wait_mbar(&mbar, phase, &okflag))) break;
+        if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
     }
 
     if (ok) {
@@ -346,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (tid == 0) {
         raise_error(S.err, ERR_TIMEOUT);
-        umma::mbar_wait(&mbar, phase ^ 1u, kPolls);
+        umma::mbar_wait(&mbar, phase ^ 1u, kWaitNs);
     }
     umma::fence_before_sync();
     __syncthreads();

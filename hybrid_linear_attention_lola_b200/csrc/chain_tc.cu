@@ -25,7 +25,7 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int kThreads = 256;
 constexpr int kFoldTok = 64;
-constexpr uint32_t kPolls = 1u << 26;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 
 struct Geo {
     int D, d, NB, NBa, FP, nblk, lam, Lmax, QC;
@@ -182,6 +182,7 @@ struct Ctx {
     uint32_t tm;           // TMEM base
     uint64_t *mbar;
     int *okflag;
+    int *err;              // device error word (timeouts stop every CTA's waits)
     uint32_t phase;
 };
 
@@ -190,7 +191,12 @@ __device__ __forceinline__ uint32_t tS(const Ctx &c) { return c.tm + (uint32_t)(
 
 __device__ bool wait_mma(Ctx &c)
 {
-    if (threadIdx.x == 0) *c.okflag = umma::mbar_wait(c.mbar, c.phase, kPolls) ? 1 : 0;
+    if (threadIdx.x == 0) {
+        const bool aborted = (*(volatile int *)c.err & ERR_TIMEOUT) != 0;
+        const bool ok = !aborted && umma::mbar_wait(c.mbar, c.phase, kWaitNs);
+        if (!ok) raise_error(c.err, ERR_TIMEOUT);
+        *c.okflag = ok ? 1 : 0;
+    }
     __syncthreads();
     c.phase ^= 1u;
     umma::fence_after_sync();
@@ -318,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *scal = (int *)(base + g.off_scal);
     c.mbar = &mbar;
     c.okflag = &okflag;
+    c.err = S.err;
     c.phase = 0;
 
     if (tid == 0) umma::mbar_init(&mbar, 1);
@@ -609,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         if (tid == 0) {
             raise_error(S.err, ERR_TIMEOUT);
-            umma::mbar_wait(&mbar, c.phase ^ 1u, kPolls);  // let an MMA still in flight drain
+            umma::mbar_wait(&mbar, c.phase ^ 1u, kWaitNs);  // let an MMA still in flight drain
         }
     }
     umma::fence_before_sync();

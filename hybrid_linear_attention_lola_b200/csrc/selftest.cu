@@ -9,7 +9,7 @@
 namespace lola {
 namespace {
 
-constexpr uint32_t kPolls = 1u << 22;
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 
 __global__ void __launch_bounds__(128)
     umma_selftest_kernel(int layout, const __nv_bfloat16 *__restrict__ A,
@@ -59,7 +59,7 @@ __global__ void __launch_bounds__(128)
         }
         umma::mma_commit(&mbar);
     }
-    const bool ok = umma::mbar_wait(&mbar, 0, kPolls);
+    const bool ok = umma::mbar_wait(&mbar, 0, kWaitNs);
     if (!ok && lane == 0) atomicOr(err, ERR_TIMEOUT);
     umma::fence_after_sync();
     if (ok) {

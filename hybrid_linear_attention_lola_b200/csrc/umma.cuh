@@ -168,11 +168,20 @@ __device__ __forceinline__ void mbar_init(uint64_t *mbar, uint32_t count)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-// Polls the mbarrier phase `parity`; gives up after max_polls and returns false.
-__device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint32_t max_polls)
+__device__ __forceinline__ uint64_t globaltimer_ns()
+{
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Waits for the mbarrier phase `parity`; gives up after limit_ns nanoseconds of
+// wall time (measured with %globaltimer) and returns false.
+__device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint64_t limit_ns)
 {
     const uint32_t a = smem_u32(mbar);
-    for (uint32_t i = 0; i < max_polls; ++i) {
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
         uint32_t done;
         asm volatile(
             "{\n\t.reg .pred p;\n\t"
@@ -182,8 +191,8 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint3
             : "r"(a), "r"(parity)
             : "memory");
         if (done) return true;
+        if (globaltimer_ns() - start > limit_ns) return false;
     }
-    return false;
 }
 
 // 16-byte asynchronous global -> shared copy (L2 only).
