@@ -158,13 +158,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     bool ok = true;
-    // ---- 1. O = phi(Q) [H'|s']
+    // ---- 1. O = phi(Q) [H'|s']: the snapshot holds H' as an N-contiguous [FP][d]
+    //         operand followed by s' as row 0 of a K-major 16 x FP operand
     if (tid == 0) {
         umma::fence_after_sync();
-        const uint32_t a0 = umma::smem_u32(sPhq), b0 = umma::smem_u32(sImg);
-        const uint32_t id = umma::idesc_bf16(128, NB, false, false);
-        for (int ks = 0; ks < FP / 16; ++ks)
-            umma::mma_ss(tO, umma::kmajor_desc(a0, ks, 128), umma::kmajor_desc(b0, ks, NB), id, ks > 0 ? 1u : 0u);
+        const uint32_t a0 = umma::smem_u32(sPhq), bh = umma::smem_u32(sImg);
+        const uint32_t bs = bh + (uint32_t)(FP * d * 2);
+        const uint32_t id_h = umma::idesc_bf16(128, d, false, true);
+        const uint32_t id_s = umma::idesc_bf16(128, 16, false, false);
+        for (int ks = 0; ks < FP / 16; ++ks) {
+            const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
+            umma::mma_ss(tO, ad, umma::mnmajor_desc(bh, ks, d), id_h, ks > 0 ? 1u : 0u);
+            umma::mma_ss(tO + (uint32_t)d, ad, umma::kmajor_desc(bs, ks, 16), id_s, ks > 0 ? 1u : 0u);
+        }
         umma::mma_commit(&mbar);
     }
     ok = wait_mbar(&mbar, phase, &okflag, S.err);

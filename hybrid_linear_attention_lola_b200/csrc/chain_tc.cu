@@ -4,17 +4,18 @@
 // (batch, kv-head) stream walks the stream's intervals in order.
 //
 // The fp32 state lives in TMEM for the whole call: feature f of block
-// bk = f / 128 is TMEM lane f % 128, columns [bk*NB, bk*NB + d) hold H[f][:],
-// column bk*NB + d holds s[f] (NB = d + 16). Both folds are tcgen05 MMAs that
-// accumulate into it:  H_blk += Phi_F^T [V_F | 1 | 0]  (A = features x tokens,
-// B = [value dims + ones column] x tokens, both K-major over tokens). After each
-// fold a bf16 image of [H | s] is written to shared memory in the K-major
-// layout (rows = value dims + normaliser, K = features); the SRE of 128
-// candidates at a time is then one MMA chain  Phi_Q [H | s]  into TMEM, and one
-// thread per candidate finishes || num / (den + eps) - v ||^2. The kept set is
-// the nK smallest order-preserving keys (SRE bits inverted, token index), found
-// by an 8-pass radix select. Prefill mode stores the image after the eviction
-// fold as the interval's snapshot for the attention kernel.
+// bk = f / 128 is TMEM lane f % 128, columns [bk*NBa, bk*NBa + d) hold H[f][:],
+// column bk*NBa + d holds s[f]. Both folds are tcgen05 MMAs that accumulate into
+// it, H_blk += Phi_F^T V_F and s_blk += Phi_F^T 1, with the tokens' phi rows and
+// value rows used as N-contiguous operands exactly as they are stored. After
+// each fold a bf16 image of the state is written to shared memory: H as an
+// N-contiguous [feature][value dim] operand and s as row 0 of a 16-row K-major
+// operand. The SRE of 128 candidates at a time is then one MMA chain
+// Phi_Q [H | s] into TMEM, and one thread per candidate finishes
+// || num / (den + eps) - v ||^2 with the candidate's value row staged in shared
+// memory. The kept set is the nK smallest order-preserving keys (SRE bits
+// inverted, token index), found by an 8-pass radix select. Prefill mode stores
+// the image after the eviction fold as the interval's snapshot for attention.
 #include "lola_internal.cuh"
 #include "umma.cuh"
 
@@ -28,14 +29,16 @@ constexpr int kFoldTok = 64;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 
 struct Geo {
-    int D, d, NB, NBa, FP, nblk, lam, Lmax, QC;
+    int D, d, NB, NBa, FP, nblk, lam, Lmax, QC, vstride;
     uint32_t ncols;
-    size_t off_X, off_keys, off_rank, off_lst, off_slotTok, off_slotVrow, off_free, off_keep,
-        off_flag, off_lf, off_hist, off_scal, total;
+    size_t off_Bs, off_ones, off_X, off_Vt, off_B1, off_keys, off_rank, off_lst, off_slotTok,
+        off_slotVrow, off_free, off_keep, off_flag, off_lf, off_hist, off_scal, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Shared memory: [H image, N-contiguous FP x d][s image, K-major 16 x FP][ones, K-major 16 x 64]
+// [X: SRE phi tile (K-major 128 x FP) + padded value rows | fold A blocks + value rows][ints]
 __host__ __device__ inline Geo make_geo(const Dims &dm)
 {
     Geo g{};
@@ -48,15 +51,22 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.lam = dm.lam;
     g.Lmax = dm.Lmax;
     g.QC = dm.lam + dm.Lmax;
+    g.vstride = (dm.d + 8) * 2;     // bytes per staged value row (padded against bank conflicts)
     const uint32_t need = (uint32_t)((g.nblk + 1) * g.NBa);
     g.ncols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
-    size_t o = (size_t)g.NB * g.FP * 2;                      // Bimg
+    size_t o = (size_t)g.FP * g.d * 2;                        // H image
+    g.off_Bs = o;                                              // s image
+    o += (size_t)g.FP * 32;
+    g.off_ones = al(o, 1024);
+    o = g.off_ones + 16 * 64 * 2;
     g.off_X = al(o, 1024);
-    const size_t xa = (size_t)128 * g.FP * 2;
-    const size_t xf = (size_t)g.nblk * 128 * kFoldTok * 2 + (size_t)g.NB * kFoldTok * 2;
-    o = g.off_X + (xa > xf ? xa : xf);
+    const size_t xs = (size_t)128 * g.FP * 2 + (size_t)128 * g.vstride;
+    const size_t xf = (size_t)g.nblk * 64 * 128 * 2 + (size_t)64 * g.d * 2;
+    g.off_Vt = g.off_X + (size_t)128 * g.FP * 2;
+    g.off_B1 = g.off_X + (size_t)g.nblk * 64 * 128 * 2;
+    o = g.off_X + (xs > xf ? xs : xf);
     g.off_keys = al(o, 16);
-    o = g.off_keys + (size_t)g.QC * 8;
+    o = g.off_keys + (size_t)g.QC * 4;
     g.off_rank = o;
     o += (size_t)g.QC * 4;
     g.off_lst = o;
@@ -66,7 +76,7 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.off_slotVrow = o;
     o += (size_t)g.lam * 4;
     g.off_free = o;
-    o += (size_t)g.lam * 4;
+    o += (size_t)g.lam * 2;
     g.off_keep = o;
     o += (size_t)g.QC;
     g.off_flag = o;
@@ -74,7 +84,7 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.off_lf = o;
     o += (size_t)g.Lmax;
     g.off_hist = al(o, 16);
-    o = g.off_hist + 256 * 4;
+    o = g.off_hist + 2 * 256 * 4;
     g.off_scal = o;
     o += 64 * 4;
     g.total = o + 1024;  // alignment slack for the 1024-byte aligned base
@@ -119,26 +129,26 @@ __device__ int scan_excl(const F *in, int *out, int n, int *wsum)
     return total;
 }
 
-__device__ __forceinline__ unsigned long long make_key(float sre, int tok)
-{
-    const unsigned bits = __float_as_uint(fmaxf(sre, 0.f));
-    return ((unsigned long long)(0xFFFFFFFFu - bits) << 32) | (unsigned)tok;
-}
-
-// The k-th smallest (1-based) of n distinct 64-bit keys, 8 bits per pass.
-__device__ unsigned long long radix_select(const unsigned long long *keys, int n, int k, int *hist,
+// The k-th smallest (1-based) of n distinct 64-bit keys key(c) = (hi[c] << 32) | tok(c),
+// 8 bits per pass; the two histograms alternate so each pass needs two barriers.
+template <typename TokF>
+__device__ unsigned long long radix_select(const unsigned *hi, TokF tok, int n, int k, int *hist2,
                                            int *scal)
 {
     const int tid = threadIdx.x, nt = blockDim.x, lane = tid & 31, warp = tid >> 5;
     unsigned long long prefix = 0, mask = 0;
     int rank = k;
-    for (int shift = 56; shift >= 0; shift -= 8) {
-        for (int i = tid; i < 256; i += nt) hist[i] = 0;
-        __syncthreads();
+    for (int i = tid; i < 256; i += nt) hist2[i] = 0;
+    __syncthreads();
+    for (int pass = 0; pass < 8; ++pass) {
+        const int shift = 56 - 8 * pass;
+        int *hist = hist2 + (pass & 1) * 256;
+        int *other = hist2 + ((pass + 1) & 1) * 256;
         for (int c = tid; c < n; c += nt) {
-            const unsigned long long kk = keys[c];
+            const unsigned long long kk = ((unsigned long long)hi[c] << 32) | (unsigned)tok(c);
             if ((kk & mask) == prefix) atomicAdd(&hist[(int)((kk >> shift) & 255u)], 1);
         }
+        for (int i = tid; i < 256; i += nt) other[i] = 0;
         __syncthreads();
         if (warp == 0) {
             int loc[8], s = 0;
@@ -171,14 +181,15 @@ __device__ unsigned long long radix_select(const unsigned long long *keys, int n
         prefix |= (unsigned long long)scal[0] << shift;
         mask |= (unsigned long long)255u << shift;
         rank = scal[1];
-        __syncthreads();
     }
+    __syncthreads();
     return prefix;
 }
 
 struct Ctx {
     Geo g;
-    uint8_t *Bimg, *X;
+    uint8_t *Bimg;          // H image (N-contiguous [FP][d]), followed by the s image
+    uint8_t *Bs, *ones, *X;
     uint32_t tm;           // TMEM base
     uint64_t *mbar;
     int *okflag;
@@ -203,88 +214,78 @@ __device__ bool wait_mma(Ctx &c)
     return *c.okflag != 0;
 }
 
-// bf16 image of [H | s] (K-major: row n = value dim / normaliser, K = feature).
+// bf16 images of the state: H as an N-contiguous [feature][value dim] operand
+// (16-byte stores of 8 value dims), s as row 0 of a K-major 16 x FP operand.
 __device__ void refresh_image(Ctx &c)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = warp & 3;
     for (int bk = warp >> 2; bk < c.g.nblk; bk += kThreads / 128) {
         const int f = bk * 128 + q * 32 + lane;
-        for (int c0 = 0; c0 < c.g.NB; c0 += 16) {
+        const uint32_t row = tH(c, bk) + ((uint32_t)(q * 32) << 16);
+        for (int c0 = 0; c0 < c.g.d; c0 += 16) {
             float v[16];
-            umma::tmem_ld16(tH(c, bk) + ((uint32_t)(q * 32) << 16) + (uint32_t)c0, v);
+            umma::tmem_ld16(row + (uint32_t)c0, v);
             umma::tmem_wait_ld();
+            __align__(16) bf16 h[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-                *(bf16 *)(c.Bimg + umma::kmajor_offset(c0 + i, f, c.g.NB)) = __float2bfloat16_rn(v[i]);
+            for (int i = 0; i < 16; ++i) h[i] = __float2bfloat16_rn(v[i]);
+            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0, c.g.d)) = *(const uint4 *)h;
+            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0 + 8, c.g.d)) = *(const uint4 *)(h + 8);
         }
+        float v[16];
+        umma::tmem_ld16(row + (uint32_t)c.g.d, v);
+        umma::tmem_wait_ld();
+        *(bf16 *)(c.Bs + umma::kmajor_offset(0, f, 16)) = __float2bfloat16_rn(v[0]);
     }
     umma::fence_async_smem();
     umma::fence_before_sync();
     __syncthreads();
 }
 
-// H += sum phi(k) v^T, s += sum phi(k) over the listed virtual rows, on the tensor cores.
+// H += sum phi(k) v^T, s += sum phi(k) over the listed virtual rows, on the tensor
+// cores. A = the tokens' phi rows and B = their value rows, both N-contiguous
+// as stored (copied with 16-byte cp.async, no transpose); a second MMA against
+// a ones column accumulates s in column d.
 __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict__ phi_st,
                         const KVSrc<bf16> &src, int st)
 {
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31, nw = kThreads >> 5;
+    const int tid = threadIdx.x;
     const Geo &g = c.g;
-    uint8_t *Af = c.X;
-    uint8_t *Bf = c.X + (size_t)g.nblk * 128 * kFoldTok * 2;
-    const uint32_t idesc = umma::idesc_bf16(128, g.NB, false, false);
+    uint8_t *Af = c.X;                                              // nblk x [64 tokens x 128 features]
+    uint8_t *B1 = c.X + (size_t)g.nblk * 64 * 128 * 2;              // [64 tokens x d]
+    const uint32_t id_h = umma::idesc_bf16(128, g.d, true, true);
+    const uint32_t id_s = umma::idesc_bf16(128, 16, true, false);
+    const int fch = g.FP / 8, vch = g.d / 8;
     for (int base = 0; base < cnt; base += kFoldTok) {
         const int nt = min(kFoldTok, cnt - base);
         const int ntp = (nt + 15) & ~15;
-        // zero the padded token columns and the padded feature rows
-        for (int e = tid; e < g.FP * (ntp - nt); e += kThreads) {
-            const int f = e / (ntp - nt), t = nt + e % (ntp - nt);
-            *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 + umma::kmajor_offset(f & 127, t, 128)) =
-                __float2bfloat16_rn(0.f);
+        for (int e = tid; e < ntp * fch; e += kThreads) {
+            const int t = e / fch, f = (e - t * fch) * 8;
+            uint8_t *dst = Af + (size_t)(f >> 7) * 64 * 128 * 2 + umma::mnmajor_offset(t, f & 127, 128);
+            if (t < nt && f < g.D) umma::cp_async16(dst, phi_st + (size_t)lst[base + t] * g.D + f);
+            else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
         }
-        for (int e = tid; e < (g.FP - g.D) * nt; e += kThreads) {
-            const int f = g.D + e / nt, t = e % nt;
-            *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 + umma::kmajor_offset(f & 127, t, 128)) =
-                __float2bfloat16_rn(0.f);
+        for (int e = tid; e < ntp * vch; e += kThreads) {
+            const int t = e / vch, c0 = (e - t * vch) * 8;
+            uint8_t *dst = B1 + umma::mnmajor_offset(t, c0, g.d);
+            if (t < nt) umma::cp_async16(dst, src.vrow(st, lst[base + t]) + c0);
+            else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
         }
-        for (int e = tid; e < g.NB * (ntp - nt); e += kThreads) {
-            const int n = e / (ntp - nt), t = nt + e % (ntp - nt);
-            *(bf16 *)(Bf + umma::kmajor_offset(n, t, g.NB)) = __float2bfloat16_rn(0.f);
-        }
-        // one warp per token: phi row -> column t of A, [v | 1 | 0] -> column t of B
-        for (int t = warp; t < nt; t += nw) {
-            const int vr = lst[base + t];
-            const bf16 *ph = phi_st + (size_t)vr * g.D;
-            for (int f0 = lane * 8; f0 < g.D; f0 += 256) {
-                const uint4 raw = *(const uint4 *)(ph + f0);
-                const bf16 *pv = (const bf16 *)&raw;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const int f = f0 + j;
-                    *(bf16 *)(Af + (size_t)(f >> 7) * 128 * kFoldTok * 2 +
-                              umma::kmajor_offset(f & 127, t, 128)) = pv[j];
-                }
-            }
-            const bf16 *vv = src.vrow(st, vr);
-            for (int c0 = lane * 8; c0 < g.d; c0 += 256) {
-                const uint4 raw = *(const uint4 *)(vv + c0);
-                const bf16 *pv = (const bf16 *)&raw;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) *(bf16 *)(Bf + umma::kmajor_offset(c0 + j, t, g.NB)) = pv[j];
-            }
-            for (int n = g.d + lane; n < g.NB; n += 32)
-                *(bf16 *)(Bf + umma::kmajor_offset(n, t, g.NB)) = __float2bfloat16_rn(n == g.d ? 1.f : 0.f);
-        }
+        umma::cp_async_commit();
+        umma::cp_async_wait_all();
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t b0 = umma::smem_u32(Bf);
+            const uint32_t b1 = umma::smem_u32(B1), on = umma::smem_u32(c.ones);
             for (int bk = 0; bk < g.nblk; ++bk) {
-                const uint32_t a0 = umma::smem_u32(Af + (size_t)bk * 128 * kFoldTok * 2);
-                for (int ks = 0; ks < ntp / 16; ++ks)
-                    umma::mma_ss(tH(c, bk), umma::kmajor_desc(a0, ks, 128),
-                                 umma::kmajor_desc(b0, ks, g.NB), idesc, 1u);
+                const uint32_t a0 = umma::smem_u32(Af + (size_t)bk * 64 * 128 * 2);
+                for (int ks = 0; ks < ntp / 16; ++ks) {
+                    const uint64_t ad = umma::mnmajor_desc(a0, ks, 128);
+                    umma::mma_ss(tH(c, bk), ad, umma::mnmajor_desc(b1, ks, g.d), id_h, 1u);
+                    umma::mma_ss(tH(c, bk) + (uint32_t)g.d, ad, umma::kmajor_desc(on, ks, 16), id_s, 1u);
+                }
             }
             umma::mma_commit(c.mbar);
         }
@@ -310,13 +311,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     Ctx c;
     c.g = g;
     c.Bimg = base;
+    c.Bs = base + g.off_Bs;
+    c.ones = base + g.off_ones;
     c.X = base + g.off_X;
-    unsigned long long *keys = (unsigned long long *)(base + g.off_keys);
+    unsigned *keys = (unsigned *)(base + g.off_keys);      // high 32 bits of each candidate's key
     int *rank = (int *)(base + g.off_rank);
     int *lst = (int *)(base + g.off_lst);
     int *slotTok = (int *)(base + g.off_slotTok);
     int *slotVrow = (int *)(base + g.off_slotVrow);
-    int *freeSlot = (int *)(base + g.off_free);
+    short *freeSlot = (short *)(base + g.off_free);
     uint8_t *keep = base + g.off_keep;
     uint8_t *flag = base + g.off_flag;
     uint8_t *lf = base + g.off_lf;
@@ -326,6 +329,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     c.okflag = &okflag;
     c.err = S.err;
     c.phase = 0;
+    // constant operands: s image rows 1..15 and the ones column (row 0 of a 16 x 64 tile)
+    for (int e = tid; e < g.FP * 16; e += kThreads) {
+        const int r = e / g.FP, f = e - r * g.FP;
+        if (r > 0) *(bf16 *)(c.Bs + umma::kmajor_offset(r, f, 16)) = __float2bfloat16_rn(0.f);
+    }
+    for (int e = tid; e < 16 * 64; e += kThreads) {
+        const int r = e / 64, k = e - r * 64;
+        *(bf16 *)(c.ones + umma::kmajor_offset(r, k, 16)) = __float2bfloat16_rn(r == 0 ? 1.f : 0.f);
+    }
 
     if (tid == 0) umma::mbar_init(&mbar, 1);
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
@@ -371,7 +383,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     bool ok = true;
-    const uint32_t idesc_sre = umma::idesc_bf16(128, g.NB, false, false);
+    const uint32_t id_sh = umma::idesc_bf16(128, d, false, true);
+    const uint32_t id_ss = umma::idesc_bf16(128, 16, false, false);
+    uint8_t *phiT = c.X, *Vt = base + g.off_Vt;
     for (int ci = 0; ci < a.n_int && ok; ++ci) {
         const long long t0 = a.pos0 + (long long)ci * a.ilen;
         const long long t1 = t0 + a.ilen;
@@ -396,17 +410,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nQ = nS + nL;
         for (int m0 = 0; m0 < nQ && ok; m0 += 128) {
             const int nr = min(128, nQ - m0);
-            const int chunks = g.FP / 8;
+            const int chunks = g.FP / 8, vch = d / 8;
+            // candidates' phi rows (K-major A operand) and value rows (padded, for the epilogue)
             for (int e = tid; e < nr * chunks; e += kThreads) {
                 const int r = e / chunks, kc = e - r * chunks;
                 const int cand = m0 + r;
-                uint8_t *dst = c.X + umma::kmajor_offset(r, kc * 8, 128);
+                uint8_t *dst = phiT + umma::kmajor_offset(r, kc * 8, 128);
                 if (kc * 8 < D) {
                     const int vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
                     umma::cp_async16(dst, phi_st + (size_t)vr * D + kc * 8);
                 } else {
                     *(uint4 *)dst = make_uint4(0, 0, 0, 0);
                 }
+            }
+            for (int e = tid; e < nr * vch; e += kThreads) {
+                const int r = e / vch, cc = e - r * vch;
+                const int cand = m0 + r;
+                const int vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
+                umma::cp_async16(Vt + (size_t)r * g.vstride + cc * 16, src.vrow(st, vr) + cc * 8);
             }
             umma::cp_async_commit();
             umma::cp_async_wait_all();
@@ -415,10 +436,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
             if (tid == 0) {
                 umma::fence_after_sync();
-                const uint32_t a0 = umma::smem_u32(c.X), b0 = umma::smem_u32(c.Bimg);
-                for (int ks = 0; ks < g.FP / 16; ++ks)
-                    umma::mma_ss(tS(c), umma::kmajor_desc(a0, ks, 128), umma::kmajor_desc(b0, ks, g.NB),
-                                 idesc_sre, ks > 0 ? 1u : 0u);
+                const uint32_t a0 = umma::smem_u32(phiT), bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
+                for (int ks = 0; ks < g.FP / 16; ++ks) {
+                    const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
+                    umma::mma_ss(tS(c), ad, umma::mnmajor_desc(bh, ks, d), id_sh, ks > 0 ? 1u : 0u);
+                    umma::mma_ss(tS(c) + (uint32_t)d, ad, umma::kmajor_desc(bs, ks, 16), id_ss, ks > 0 ? 1u : 0u);
+                }
                 umma::mma_commit(c.mbar);
             }
             if (!(ok = wait_mma(c))) break;
@@ -430,19 +453,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::tmem_ld16(rowaddr + (uint32_t)d, v);
                 umma::tmem_wait_ld();
                 const float den = v[0] + dm.eps;
+                const uint8_t *vrow = Vt + (size_t)r * g.vstride;
                 float err = 0.f;
-                int vr = 0, tok = 0;
-                if (cand < nQ) {
-                    vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
-                    tok = cand < nS ? slotTok[cand] : (int)(Llo + (cand - nS));
-                }
-                const bf16 *vv = src.vrow(st, vr);
                 for (int c0 = 0; c0 < d; c0 += 16) {
                     umma::tmem_ld16(rowaddr + (uint32_t)c0, v);
                     umma::tmem_wait_ld();
                     if (cand < nQ) {
-                        const uint4 r0 = *(const uint4 *)(vv + c0);
-                        const uint4 r1 = *(const uint4 *)(vv + c0 + 8);
+                        const uint4 r0 = *(const uint4 *)(vrow + c0 * 2);
+                        const uint4 r1 = *(const uint4 *)(vrow + c0 * 2 + 16);
                         const bf16 *p0 = (const bf16 *)&r0;
                         const bf16 *p1 = (const bf16 *)&r1;
 #pragma unroll
@@ -453,7 +471,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
-                if (cand < nQ) keys[cand] = make_key(err, tok);
+                if (cand < nQ) keys[cand] = 0xFFFFFFFFu - __float_as_uint(fmaxf(err, 0.f));
             }
             umma::fence_before_sync();
             __syncthreads();
@@ -462,9 +480,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
         // 3. keep the nK smallest keys (highest SRE, lower token on ties)
         const int nK = nQ < lam ? nQ : lam;
+        auto tok_of = [&](int i) -> int { return i < nS ? slotTok[i] : (int)(Llo + (i - nS)); };
         if (nQ > lam) {
-            const unsigned long long thr = radix_select(keys, nQ, nK, hist, scal);
-            for (int i = tid; i < nQ; i += kThreads) keep[i] = keys[i] <= thr ? 1 : 0;
+            const unsigned long long thr = radix_select(keys, tok_of, nQ, nK, hist, scal);
+            for (int i = tid; i < nQ; i += kThreads) {
+                const unsigned long long kk = ((unsigned long long)keys[i] << 32) | (unsigned)tok_of(i);
+                keep[i] = kk <= thr ? 1 : 0;
+            }
         } else {
             for (int i = tid; i < nQ; i += kThreads) keep[i] = 1;
         }
@@ -501,10 +523,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = tid; i < nS; i += kThreads) {
             if (flag[i]) {
                 lst[rank[i]] = slotVrow[i];
-                freeSlot[rank[i]] = i;
+                freeSlot[rank[i]] = (short)i;
             }
         }
-        for (int r = nE + tid; r < nE + (lam - nS); r += kThreads) freeSlot[r] = nS + (r - nE);
+        for (int r = nE + tid; r < nE + (lam - nS); r += kThreads) freeSlot[r] = (short)(nS + (r - nE));
         __syncthreads();
         if (nE > 0) {
             if (!(ok = fold_tc(c, lst, nE, phi_st, src, st))) break;

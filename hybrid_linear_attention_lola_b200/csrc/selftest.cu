@@ -26,11 +26,19 @@ __global__ void __launch_bounds__(128)
     uint8_t *sB = base + 128 * Kp * 2;         // K-major [N x Kp] or MN-major [K x N]
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-    for (int e = tid; e < 128 * K; e += blockDim.x) {
-        const int r = e / K, k = e - r * K;
-        *(__nv_bfloat16 *)(sA + umma::kmajor_offset(r, k, 128)) = A[e];
+    const bool a_mn = layout >= 2;            // layouts 2, 3: A given as [K][128], M contiguous
+    if (!a_mn) {
+        for (int e = tid; e < 128 * K; e += blockDim.x) {
+            const int r = e / K, k = e - r * K;
+            *(__nv_bfloat16 *)(sA + umma::kmajor_offset(r, k, 128)) = A[e];
+        }
+    } else {
+        for (int e = tid; e < 128 * K; e += blockDim.x) {
+            const int k = e / 128, m = e - k * 128;
+            *(__nv_bfloat16 *)(sA + umma::mnmajor_offset(k, m, 128)) = A[e];
+        }
     }
-    if (layout == 0) {
+    if (layout == 0 || layout == 3) {
         for (int e = tid; e < N * K; e += blockDim.x) {
             const int n = e / K, k = e - n * K;
             *(__nv_bfloat16 *)(sB + umma::kmajor_offset(n, k, N)) = B[e];
@@ -50,11 +58,12 @@ __global__ void __launch_bounds__(128)
     umma::fence_after_sync();
     const uint32_t taddr = tslot;
     if (tid == 0) {
-        const uint32_t id = umma::idesc_bf16(128, N, false, layout == 1);
+        const bool b_mn = layout == 1 || layout == 2;
+        const uint32_t id = umma::idesc_bf16(128, N, a_mn, b_mn);
         const uint32_t a0 = umma::smem_u32(sA), b0 = umma::smem_u32(sB);
         for (int ks = 0; ks < K / 16; ++ks) {
-            const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
-            const uint64_t bd = layout == 0 ? umma::kmajor_desc(b0, ks, N) : umma::mnmajor_desc(b0, ks, N);
+            const uint64_t ad = a_mn ? umma::mnmajor_desc(a0, ks, 128) : umma::kmajor_desc(a0, ks, 128);
+            const uint64_t bd = b_mn ? umma::mnmajor_desc(b0, ks, N) : umma::kmajor_desc(b0, ks, N);
             umma::mma_ss(taddr, ad, bd, id, ks > 0 ? 1u : 0u);
         }
         umma::mma_commit(&mbar);
@@ -83,11 +92,12 @@ __global__ void __launch_bounds__(128)
 extern "C" lola_status lola_selftest_umma(int layout, const void *A, const void *B, float *C, int N,
                                           int K, int *dev_err, void *cuda_stream)
 {
-    if (!A || !B || !C || !dev_err || (layout != 0 && layout != 1)) return LOLA_ERR_INVALID_ARG;
+    if (!A || !B || !C || !dev_err || layout < 0 || layout > 3) return LOLA_ERR_INVALID_ARG;
     if (N < 16 || N > 256 || N % 16 || K < 16 || K > 256 || K % 16) return LOLA_ERR_INVALID_ARG;
-    if (layout == 1 && N % 64) return LOLA_ERR_INVALID_ARG;
+    if ((layout == 1 || layout == 2) && N % 64) return LOLA_ERR_INVALID_ARG;
+    if (layout >= 2 && K % 8) return LOLA_ERR_INVALID_ARG;
     const size_t Kp = (size_t)(K + 63) / 64 * 64;
-    const size_t smem = 128 * Kp * 2 + (layout == 0 ? (size_t)N * Kp * 2 : (size_t)N * K * 2) + 1024;
+    const size_t smem = 128 * Kp * 2 + ((layout == 0 || layout == 3) ? (size_t)N * Kp * 2 : (size_t)N * K * 2) + 1024;
     cudaFuncSetAttribute(lola::umma_selftest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
     lola::umma_selftest_kernel<<<1, 128, smem, (cudaStream_t)cuda_stream>>>(

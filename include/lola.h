@@ -172,7 +172,9 @@ lola_status lola_timing_read(lola_state *st, double *ms, int64_t *n);
 /* Test hook for the tensor-core layer: one CTA computes, on the tcgen05 tensor
  * cores, C[128][N] (fp32, row-major) = A[128][K] * op(B), where A is bf16
  * row-major, and B is bf16 [N][K] with C = A B^T (layout 0, K-major operand)
- * or [K][N] with C = A B (layout 1, N-contiguous operand, N % 64 == 0).
+ * or [K][N] with C = A B (layout 1, N-contiguous operand, N % 64 == 0);
+ * layouts 2 and 3 take A as [K][128] (M-contiguous operand) with B as in
+ * layouts 1 and 0 respectively.
  * 16 <= N, K <= 256, multiples of 16. Device pointers; dev_err is a device
  * int that receives LOLA's timeout bit if the MMA completion wait gives up.
  * Not part of the method (the paper has no counterpart); it checks the shared

@@ -18,13 +18,17 @@ def _cuda():
 
 
 @pytest.mark.parametrize("layout,N,K", [(0, 80, 128), (0, 144, 256), (0, 128, 64), (0, 16, 16),
-                                        (1, 128, 128), (1, 64, 64), (1, 256, 32), (1, 128, 256)])
+                                        (1, 128, 128), (1, 64, 64), (1, 256, 32), (1, 128, 256),
+                                        (2, 128, 64), (2, 64, 16), (3, 16, 64), (3, 16, 48)])
 def test_umma_matches_matmul(layout, N, K):
     g = torch.Generator().manual_seed(1000 + N + K + layout)
-    A = torch.randn(128, K, generator=g).to(torch.bfloat16)
-    B = torch.randn(N, K, generator=g).to(torch.bfloat16) if layout == 0 else \
+    a_mn = layout >= 2
+    b_kmajor = layout in (0, 3)
+    A = torch.randn(K, 128, generator=g).to(torch.bfloat16) if a_mn else \
+        torch.randn(128, K, generator=g).to(torch.bfloat16)
+    B = torch.randn(N, K, generator=g).to(torch.bfloat16) if b_kmajor else \
         torch.randn(K, N, generator=g).to(torch.bfloat16)
-    want = A.float() @ (B.float().T if layout == 0 else B.float())
+    want = (A.float().T if a_mn else A.float()) @ (B.float().T if b_kmajor else B.float())
     Ad, Bd = A.cuda(), B.cuda()
     C = torch.full((128, N), float("nan"), device="cuda")
     err = torch.zeros(1, dtype=torch.int32, device="cuda")
