@@ -119,7 +119,9 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->C = c->chunk;
     dm->Cdec = c->decode_interval;
     dm->Lmax = c->chunk > c->decode_interval ? c->chunk : c->decode_interval;
-    dm->R = c->window + dm->Lmax + 1;
+    // ring slots: a power of two >= window + longest interval + 1 (slot = token & (R - 1))
+    dm->R = 1;
+    while (dm->R < c->window + dm->Lmax + 1) dm->R <<= 1;
     dm->ns = c->batch * c->n_kv_heads;
     dm->dtype = c->dtype;
     dm->Nmax = nmax;

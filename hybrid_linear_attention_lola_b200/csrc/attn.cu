@@ -292,7 +292,7 @@ __global__ void ring_update_kernel(Dims dm, DevState S, const T *__restrict__ ki
         const int t = first + (int)(r / dm.ns);
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
         const long long tok = call_start + t;
-        const int slot = (int)(tok % dm.R);
+        const int slot = (int)(tok & (dm.R - 1));
         const T *ks = kin + (((size_t)b * n + t) * dm.Hkv + hk) * dm.d;
         const T *vs = vin + (((size_t)b * n + t) * dm.Hkv + hk) * dm.d;
         T *kd = KR + ((size_t)st * dm.R + slot) * dm.d;

@@ -33,7 +33,7 @@ enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
 struct AGeo {
     int d, D, FP, NB, NBa;
     uint32_t ncols;
-    size_t off_phq, off_big, off_K, off_V, off_phk, off_P, off_tok, off_info, total;
+    size_t off_phq, off_big, off_K, off_V, off_phk, off_P, off_tok, off_info, off_vrow, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -62,7 +62,8 @@ __host__ __device__ inline AGeo make_ageo(const Dims &dm)
     o = tiles_end > img_end ? tiles_end : img_end;
     g.off_tok = al(o, 16);
     g.off_info = g.off_tok + KT * 4;
-    g.total = g.off_info + KT * 4 + 1024;
+    g.off_vrow = g.off_info + KT * 4;
+    g.total = g.off_vrow + KT * 4 + 1024;
     return g;
 }
 
@@ -110,6 +111,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t *sK = base + g.off_K, *sV = base + g.off_V, *sPhk = base + g.off_phk, *sP = base + g.off_P;
     int *ktok = (int *)(base + g.off_tok);
     int *kinfo = (int *)(base + g.off_info);
+    int *kvrow = (int *)(base + g.off_vrow);
+    const int lgd = __ffs(d >> 3) - 1, lgf = __ffs(FP >> 3) - 1;   // 16-byte chunks per row (powers of two)
 
     if (tid == 0) umma::mbar_init(&mbar, 1);
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
@@ -125,8 +128,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bf16 *q = (const bf16 *)a.q;
     const bf16 *phiQ = (const bf16 *)P.phiQ;
     const size_t qrow0 = ((size_t)b * a.n_call + (size_t)(t0 - a.pos0)) * dm.Hq + (size_t)hk * gq;
-    for (int e = tid; e < 128 * (d / 8); e += kThreads) {
-        const int r = e / (d / 8), kc = e % (d / 8);
+    for (int e = tid; e < (128 << lgd); e += kThreads) {
+        const int r = e >> lgd, kc = e & ((1 << lgd) - 1);
         const int gr = mt * 128 + r;
         uint8_t *dst = sQ + umma::kmajor_offset(r, kc * 8, 128);
         if (gr < rows_total) {
@@ -136,8 +139,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *(uint4 *)dst = make_uint4(0, 0, 0, 0);
         }
     }
-    for (int e = tid; e < 128 * (FP / 8); e += kThreads) {
-        const int r = e / (FP / 8), kc = e % (FP / 8);
+    for (int e = tid; e < (128 << lgf); e += kThreads) {
+        const int r = e >> lgf, kc = e & ((1 << lgf) - 1);
         const int gr = mt * 128 + r;
         uint8_t *dst = sPhq + umma::kmajor_offset(r, kc * 8, 128);
         if (gr < rows_total && kc * 8 < D) {
@@ -196,30 +199,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) anylin = 0;
         __syncthreads();
         if (tid < KT) {
-            int tok = -1, info = INFO_SKIP;
+            int tok = -1, info = INFO_SKIP, vr = 0;
             if (tid < nk) {
                 if (band) {
                     const long long j = kb + tid;
                     tok = (int)j;
+                    vr = src.tok2vrow(j);
                     info = (j < t1 - eta) ? (llf[(int)(j - (t0 - eta))] ? INFO_FOLDED : INFO_SKIP) : INFO_SOFT;
                     if (info == INFO_FOLDED) anylin = 1;
                 } else {
                     tok = ltok[kb + tid];
+                    vr = lvrow[kb + tid];
                     info = INFO_SOFT;
                 }
             }
             ktok[tid] = tok;
             kinfo[tid] = info;
+            kvrow[tid] = vr;
         }
         __syncthreads();
         const bool lin = anylin != 0;
         // K (K-major [key][d]), V (N-contiguous [key][d]) and, for linear keys, phi(K)
-        for (int e = tid; e < KT * (d / 8); e += kThreads) {
-            const int j = e / (d / 8), kc = e % (d / 8);
+        for (int e = tid; e < (KT << lgd); e += kThreads) {
+            const int j = e >> lgd, kc = e & ((1 << lgd) - 1);
             uint8_t *dk = sK + umma::kmajor_offset(j, kc * 8, KT);
             uint8_t *dv = sV + umma::mnmajor_offset(j, kc * 8, d);
             if (j < nk) {
-                const int vr = band ? src.tok2vrow(kb + j) : lvrow[kb + j];
+                const int vr = kvrow[j];
                 umma::cp_async16(dk, src.krow(st, vr) + kc * 8);
                 umma::cp_async16(dv, src.vrow(st, vr) + kc * 8);
             } else {
@@ -228,10 +234,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         if (lin) {
-            for (int e = tid; e < KT * (FP / 8); e += kThreads) {
-                const int j = e / (FP / 8), kc = e % (FP / 8);
+            for (int e = tid; e < (KT << lgf); e += kThreads) {
+                const int j = e >> lgf, kc = e & ((1 << lgf) - 1);
                 uint8_t *dst = sPhk + umma::kmajor_offset(j, kc * 8, KT);
-                if (j < nk && kc * 8 < D) umma::cp_async16(dst, phiK + (size_t)src.tok2vrow(kb + j) * D + kc * 8);
+                if (j < nk && kc * 8 < D) umma::cp_async16(dst, phiK + (size_t)kvrow[j] * D + kc * 8);
                 else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
             }
         }

@@ -171,6 +171,7 @@ __device__ unsigned long long radix_select(const unsigned *hi, TokF tok, int n, 
                     if (cum + loc[j] >= rank) {
                         scal[0] = lane * 8 + j;
                         scal[1] = rank - cum;
+                        scal[4] = loc[j];          // keys sharing the extended prefix
                         break;
                     }
                     cum += loc[j];
@@ -181,6 +182,18 @@ __device__ unsigned long long radix_select(const unsigned *hi, TokF tok, int n, 
         prefix |= (unsigned long long)scal[0] << shift;
         mask |= (unsigned long long)255u << shift;
         rank = scal[1];
+        if (scal[4] == 1) {
+            // a single key carries this prefix: it is the answer
+            __syncthreads();
+            for (int c = tid; c < n; c += nt) {
+                const unsigned long long kk = ((unsigned long long)hi[c] << 32) | (unsigned)tok(c);
+                if ((kk & mask) == prefix) *(unsigned long long *)(scal + 6) = kk;
+            }
+            __syncthreads();
+            const unsigned long long r = *(const unsigned long long *)(scal + 6);
+            __syncthreads();
+            return r;
+        }
     }
     __syncthreads();
     return prefix;
@@ -255,18 +268,18 @@ __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict_
     uint8_t *B1 = c.X + (size_t)g.nblk * 64 * 128 * 2;              // [64 tokens x d]
     const uint32_t id_h = umma::idesc_bf16(128, g.d, true, true);
     const uint32_t id_s = umma::idesc_bf16(128, 16, true, false);
-    const int fch = g.FP / 8, vch = g.d / 8;
+    const int lgf = __ffs(g.FP >> 3) - 1, lgv = __ffs(g.d >> 3) - 1;  // 16-byte chunks per row
     for (int base = 0; base < cnt; base += kFoldTok) {
         const int nt = min(kFoldTok, cnt - base);
         const int ntp = (nt + 15) & ~15;
-        for (int e = tid; e < ntp * fch; e += kThreads) {
-            const int t = e / fch, f = (e - t * fch) * 8;
+        for (int e = tid; e < (ntp << lgf); e += kThreads) {
+            const int t = e >> lgf, f = (e & ((1 << lgf) - 1)) * 8;
             uint8_t *dst = Af + (size_t)(f >> 7) * 64 * 128 * 2 + umma::mnmajor_offset(t, f & 127, 128);
             if (t < nt && f < g.D) umma::cp_async16(dst, phi_st + (size_t)lst[base + t] * g.D + f);
             else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
         }
-        for (int e = tid; e < ntp * vch; e += kThreads) {
-            const int t = e / vch, c0 = (e - t * vch) * 8;
+        for (int e = tid; e < (ntp << lgv); e += kThreads) {
+            const int t = e >> lgv, c0 = (e & ((1 << lgv) - 1)) * 8;
             uint8_t *dst = B1 + umma::mnmajor_offset(t, c0, g.d);
             if (t < nt) umma::cp_async16(dst, src.vrow(st, lst[base + t]) + c0);
             else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
@@ -408,26 +421,24 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long Lhi = t1 - eta > Llo ? t1 - eta : Llo;
         const int nL = (int)(Lhi - Llo);
         const int nQ = nS + nL;
+        // virtual row of every candidate, once per interval (rank[] is free here)
+        int *cvrow = rank;
+        for (int cnd = tid; cnd < nQ; cnd += kThreads)
+            cvrow[cnd] = cnd < nS ? slotVrow[cnd] : src.tok2vrow(Llo + (cnd - nS));
+        __syncthreads();
+        const int lgc = __ffs(g.FP >> 3) - 1, lgv = __ffs(d >> 3) - 1;   // chunks per row (powers of two)
         for (int m0 = 0; m0 < nQ && ok; m0 += 128) {
             const int nr = min(128, nQ - m0);
-            const int chunks = g.FP / 8, vch = d / 8;
             // candidates' phi rows (K-major A operand) and value rows (padded, for the epilogue)
-            for (int e = tid; e < nr * chunks; e += kThreads) {
-                const int r = e / chunks, kc = e - r * chunks;
-                const int cand = m0 + r;
+            for (int e = tid; e < (nr << lgc); e += kThreads) {
+                const int r = e >> lgc, kc = e & ((1 << lgc) - 1);
                 uint8_t *dst = phiT + umma::kmajor_offset(r, kc * 8, 128);
-                if (kc * 8 < D) {
-                    const int vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
-                    umma::cp_async16(dst, phi_st + (size_t)vr * D + kc * 8);
-                } else {
-                    *(uint4 *)dst = make_uint4(0, 0, 0, 0);
-                }
+                if (kc * 8 < D) umma::cp_async16(dst, phi_st + (size_t)cvrow[m0 + r] * D + kc * 8);
+                else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
             }
-            for (int e = tid; e < nr * vch; e += kThreads) {
-                const int r = e / vch, cc = e - r * vch;
-                const int cand = m0 + r;
-                const int vr = cand < nS ? slotVrow[cand] : src.tok2vrow(Llo + (cand - nS));
-                umma::cp_async16(Vt + (size_t)r * g.vstride + cc * 16, src.vrow(st, vr) + cc * 8);
+            for (int e = tid; e < (nr << lgv); e += kThreads) {
+                const int r = e >> lgv, cc = e & ((1 << lgv) - 1);
+                umma::cp_async16(Vt + (size_t)r * g.vstride + cc * 16, src.vrow(st, cvrow[m0 + r]) + cc * 8);
             }
             umma::cp_async_commit();
             umma::cp_async_wait_all();
@@ -445,33 +456,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::mma_commit(c.mbar);
             }
             if (!(ok = wait_mma(c))) break;
-            if (warp < 4) {
-                const int r = warp * 32 + lane;
-                const int cand = m0 + r;
-                const uint32_t rowaddr = tS(c) + ((uint32_t)(warp * 32) << 16);
+            {
+                // 8 warps: warp w reads lanes 32*(w%4).., value columns half (w/4) of d
+                const int q = warp & 3, half = warp >> 2;
+                const int r = q * 32 + lane;
+                const uint32_t rowaddr = tS(c) + ((uint32_t)(q * 32) << 16);
                 float v[16];
                 umma::tmem_ld16(rowaddr + (uint32_t)d, v);
                 umma::tmem_wait_ld();
                 const float den = v[0] + dm.eps;
+                const float rden = den != 0.f ? 1.f / den : 0.f;
                 const uint8_t *vrow = Vt + (size_t)r * g.vstride;
+                const int cbeg = half * (d >> 1), cend = cbeg + (d >> 1);
                 float err = 0.f;
-                for (int c0 = 0; c0 < d; c0 += 16) {
+                for (int c0 = cbeg; c0 < cend; c0 += 16) {
                     umma::tmem_ld16(rowaddr + (uint32_t)c0, v);
                     umma::tmem_wait_ld();
-                    if (cand < nQ) {
-                        const uint4 r0 = *(const uint4 *)(vrow + c0 * 2);
-                        const uint4 r1 = *(const uint4 *)(vrow + c0 * 2 + 16);
-                        const bf16 *p0 = (const bf16 *)&r0;
-                        const bf16 *p1 = (const bf16 *)&r1;
+                    const uint4 r0 = *(const uint4 *)(vrow + c0 * 2);
+                    const uint4 r1 = *(const uint4 *)(vrow + c0 * 2 + 16);
+                    const bf16 *p0 = (const bf16 *)&r0;
+                    const bf16 *p1 = (const bf16 *)&r1;
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const float pred = den != 0.f ? v[i] / den : 0.f;
-                            const float diff = pred - __bfloat162float(i < 8 ? p0[i] : p1[i - 8]);
-                            err = fmaf(diff, diff, err);
-                        }
+                    for (int i = 0; i < 16; ++i) {
+                        const float diff = v[i] * rden - __bfloat162float(i < 8 ? p0[i] : p1[i - 8]);
+                        err = fmaf(diff, diff, err);
                     }
                 }
-                if (cand < nQ) keys[cand] = 0xFFFFFFFFu - __float_as_uint(fmaxf(err, 0.f));
+                float *part = (float *)(base + g.off_X);   // phi tile no longer needed: reuse for partial sums
+                if (half == 1) part[r] = err;
+                __syncthreads();
+                if (half == 0 && m0 + r < nQ) {
+                    err += part[r];
+                    keys[m0 + r] = 0xFFFFFFFFu - __float_as_uint(fmaxf(err, 0.f));
+                }
             }
             umma::fence_before_sync();
             __syncthreads();

@@ -27,7 +27,7 @@ __global__ void append_kernel(Dims dm, DevState S, const T *__restrict__ k, cons
                               long long pos)
 {
     const int st = blockIdx.x;
-    const int slot = (int)(pos % dm.R);
+    const int slot = (int)(pos & (dm.R - 1));
     T *KR = (T *)S.KR + ((size_t)st * dm.R + slot) * dm.d;
     T *VR = (T *)S.VR + ((size_t)st * dm.R + slot) * dm.d;
     for (int c = threadIdx.x; c < dm.d; c += blockDim.x) {
@@ -98,7 +98,7 @@ __global__ void __launch_bounds__(DW * 32)
                 } else {
                     const long long j = jlo + (kk - a.nS);
                     tok = (int)j;
-                    row = lam + (int)(j % R);
+                    row = lam + (int)(j & (R - 1));
                     if (j >= a.L_lo && j < a.L_hi)
                         info = S.pend[(size_t)st * dm.Lmax + (int)(j - a.L_lo)] ? 1 : 2;
                     else

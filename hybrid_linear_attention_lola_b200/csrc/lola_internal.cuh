@@ -7,7 +7,7 @@
 // places: the state's sparse-cache slots, the state's window ring, and the
 // caller's k/v buffers. The kernels address them through one row index per
 // stream:  [0, lam)            cache slot i
-//          [lam, lam + R)      ring slot (token mod R)
+//          [lam, lam + R)      ring slot (token mod R; R is a power of two)
 //          [lam + R, lam+R+n)  token call_start + (row - lam - R) of the call
 // phi(k) scratch is laid out over the same rows.
 #pragma once
@@ -95,7 +95,7 @@ template <typename T> struct KVSrc {
     __device__ __forceinline__ int tok2vrow(long long tok) const
     {
         if (kin != nullptr && tok >= call_start) return lam + R + (int)(tok - call_start);
-        return lam + (int)(tok % R);
+        return lam + (int)(tok & (R - 1));  // R is a power of two
     }
 };
 

@@ -37,7 +37,7 @@ def test_stream_bytes_constant_in_sequence_length(lib):
     assert len(sizes) == 1
     # H|s fp32 + cache K/V bf16 + indices + ring K/V bf16 + flags
     d, D, lam, eta, C = 128, 256, 2048, 64, 128
-    R = eta + C + 1
+    R = 256                         # power of two >= eta + C + 1
     assert sizes.pop() == D * d * 4 + D * 4 + 2 * lam * d * 2 + lam * 4 + 2 * R * d * 2 + C
 
 
