@@ -4,19 +4,20 @@
 //
 // One CTA = one update interval of one (batch, kv-head) stream and 128 query
 // rows; row r is (position t0 + mt*128/g + r/g, query head hk*g + r%g), so the
-// rows of a tile are consecutive in q and out. Thread r owns row r (TMEM lane r).
+// rows of a tile are consecutive in q and out. Row r is TMEM lane r; threads
+// r and r + 128 (the two halves of the CTA) share it, each exponentiating half
+// of every 64-key tile.
 //   1. O = phi(Q) [H'|s']   (readout of the interval's snapshot; column d of O
 //      carries the linear denominator phi(q).s', so it rescales with O);
 //   2. per 64-key tile: S = Q K^T (and G = phi(Q) phi(K)^T for window tiles that
-//      hold folded leaving pairs) on the tensor cores; thread r turns row r into
-//      P = e^{s-m} (softmax keys) or g e^{-m} (linear keys) with the running
-//      shift m = max(0, max score), rescales its O row in TMEM when m grows, and
-//      writes P (bf16) to shared memory; O += P V.
+//      hold folded leaving pairs) on the tensor cores; P = e^{s-m} for softmax
+//      keys and g e^{-m} for linear keys, with the running shift
+//      m = max(0, max score); O is rescaled in TMEM when m grows; O += P V.
+//      Tile i+1's keys and values are copied while tile i is processed.
 //   3. out = O[:, :d] / (sum P + O[:, d] + eps e^{-m}).
-// The key classes follow the method: cached keys are softmax (causal); window
-// keys [t0 - eta, t1) are softmax while inside the window of p, linear once
-// they left it and were folded, and skipped when they were kept (they appear
-// among the cached keys).
+// Key classes: cached keys are softmax (causal); window keys [t0 - eta, t1)
+// are softmax while inside the window of p, linear once they left it and were
+// folded, and skipped when they were kept (they appear among the cached keys).
 #include "lola_internal.cuh"
 #include "umma.cuh"
 
@@ -25,15 +26,22 @@ namespace lola {
 namespace {
 
 using bf16 = __nv_bfloat16;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int KT = 64;                // keys per tile
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
 
+struct TileMeta {
+    int tok[KT], info[KT], vrow[KT];
+    int lin[2];        // per producing warp: some key is a folded leaving pair
+    int causal[2];     // per producing warp: every key is causal for every row of the CTA
+    int nk, band;
+};
+
 struct AGeo {
     int d, D, FP, NB, NBa;
     uint32_t ncols;
-    size_t off_phq, off_big, off_K, off_V, off_phk, off_P, off_tok, off_info, off_vrow, total;
+    size_t off_phq, off_big, off_K[2], off_V[2], off_phk, off_P, off_meta, off_red, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -53,17 +61,20 @@ __host__ __device__ inline AGeo make_ageo(const Dims &dm)
     g.off_phq = al(o, 1024);
     o = g.off_phq + (size_t)128 * g.FP * 2;                // phi(Q)
     g.off_big = al(o, 1024);                               // snapshot image, then key tiles
-    g.off_K = g.off_big;
-    g.off_V = al(g.off_K + (size_t)KT * dp * 2, 1024);
-    g.off_phk = al(g.off_V + (size_t)KT * g.d * 2, 1024);
+    o = g.off_big;
+    for (int b = 0; b < 2; ++b) {
+        g.off_K[b] = al(o, 1024);
+        g.off_V[b] = al(g.off_K[b] + (size_t)KT * dp * 2, 1024);
+        o = g.off_V[b] + (size_t)KT * g.d * 2;
+    }
+    g.off_phk = al(o, 1024);
     g.off_P = al(g.off_phk + (size_t)KT * g.FP * 2, 1024);
-    size_t tiles_end = g.off_P + (size_t)128 * KT * 2;
-    size_t img_end = g.off_big + (size_t)g.NB * g.FP * 2;
+    const size_t tiles_end = g.off_P + (size_t)128 * KT * 2;
+    const size_t img_end = g.off_big + (size_t)g.FP * (g.d + 16) * 2;
     o = tiles_end > img_end ? tiles_end : img_end;
-    g.off_tok = al(o, 16);
-    g.off_info = g.off_tok + KT * 4;
-    g.off_vrow = g.off_info + KT * 4;
-    g.total = g.off_vrow + KT * 4 + 1024;
+    g.off_meta = al(o, 16);
+    g.off_red = al(g.off_meta + 2 * sizeof(TileMeta), 16);
+    g.total = g.off_red + 128 * 4 + 1024;
     return g;
 }
 
@@ -87,32 +98,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(Dims dm, DevState S, PrefillScratch P, AttnArgs a, KVSrc<bf16> src)
 {
     const AGeo g = make_ageo(dm);
-    const int d = g.d, D = g.D, FP = g.FP, NB = g.NB, eta = dm.eta, lam = dm.lam, gq = dm.g;
+    const int d = g.d, D = g.D, FP = g.FP, eta = dm.eta, lam = dm.lam, gq = dm.g;
     const int tiles_per_int = (dm.C * gq + 127) / 128;
     const int ci = blockIdx.x / tiles_per_int, mt = blockIdx.x % tiles_per_int;
     const int st = blockIdx.y;
     const int b = st / dm.Hkv, hk = st % dm.Hkv;
     const long long t0 = a.pos0 + (long long)ci * dm.C, t1 = t0 + dm.C;
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, half = warp >> 2;
+    const int r = qd * 32 + lane;                    // this thread's row (TMEM lane)
     const int rows_total = dm.C * gq;
-    const int grow = mt * 128 + tid;                 // row within the interval
+    const int grow = mt * 128 + r;
     const bool row_ok = grow < rows_total;
-    const long long p = t0 + grow / gq;              // query position of this thread's row
+    const long long p = t0 + grow / gq;              // query position of the row
+    const long long pmin = t0 + (mt * 128) / gq;     // smallest position in the CTA
     const float scale = rsqrtf((float)d);
+    const int lgd = __ffs(d >> 3) - 1, lgf = __ffs(FP >> 3) - 1;   // 16-byte chunks per row
 
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar;
     __shared__ uint32_t tslot;
     __shared__ int okflag;
-    __shared__ int anylin;
     const uint32_t raw = umma::smem_u32(smraw);
     uint8_t *base = smraw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *sQ = base, *sPhq = base + g.off_phq, *sImg = base + g.off_big;
-    uint8_t *sK = base + g.off_K, *sV = base + g.off_V, *sPhk = base + g.off_phk, *sP = base + g.off_P;
-    int *ktok = (int *)(base + g.off_tok);
-    int *kinfo = (int *)(base + g.off_info);
-    int *kvrow = (int *)(base + g.off_vrow);
-    const int lgd = __ffs(d >> 3) - 1, lgf = __ffs(FP >> 3) - 1;   // 16-byte chunks per row (powers of two)
+    uint8_t *sPhk = base + g.off_phk, *sP = base + g.off_P;
+    TileMeta *meta = (TileMeta *)(base + g.off_meta);
+    float *red = (float *)(base + g.off_red);
 
     if (tid == 0) umma::mbar_init(&mbar, 1);
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
@@ -121,7 +133,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma::fence_after_sync();
     const uint32_t tm = tslot;
     const uint32_t tO = tm, tS = tm + (uint32_t)g.NBa, tG = tS + KT;
-    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     uint32_t phase = 0;
 
     // ---- stage Q, phi(Q) and the snapshot image
@@ -129,9 +141,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bf16 *phiQ = (const bf16 *)P.phiQ;
     const size_t qrow0 = ((size_t)b * a.n_call + (size_t)(t0 - a.pos0)) * dm.Hq + (size_t)hk * gq;
     for (int e = tid; e < (128 << lgd); e += kThreads) {
-        const int r = e >> lgd, kc = e & ((1 << lgd) - 1);
-        const int gr = mt * 128 + r;
-        uint8_t *dst = sQ + umma::kmajor_offset(r, kc * 8, 128);
+        const int rr = e >> lgd, kc = e & ((1 << lgd) - 1);
+        const int gr = mt * 128 + rr;
+        uint8_t *dst = sQ + umma::kmajor_offset(rr, kc * 8, 128);
         if (gr < rows_total) {
             const size_t row = qrow0 + (size_t)(gr / gq) * dm.Hq + gr % gq;
             umma::cp_async16(dst, q + row * d + kc * 8);
@@ -140,9 +152,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     for (int e = tid; e < (128 << lgf); e += kThreads) {
-        const int r = e >> lgf, kc = e & ((1 << lgf) - 1);
-        const int gr = mt * 128 + r;
-        uint8_t *dst = sPhq + umma::kmajor_offset(r, kc * 8, 128);
+        const int rr = e >> lgf, kc = e & ((1 << lgf) - 1);
+        const int gr = mt * 128 + rr;
+        uint8_t *dst = sPhq + umma::kmajor_offset(rr, kc * 8, 128);
         if (gr < rows_total && kc * 8 < D) {
             const size_t row = qrow0 + (size_t)(gr / gq) * dm.Hq + gr % gq;
             umma::cp_async16(dst, phiQ + row * D + kc * 8);
@@ -151,8 +163,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     {
-        const uint8_t *img = (const uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * NB * FP * 2;
-        for (int e = tid; e < NB * FP * 2 / 16; e += kThreads) umma::cp_async16(sImg + e * 16, img + e * 16);
+        const int nb = FP * (d + 16) * 2;
+        const uint8_t *img = (const uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * nb;
+        for (int e = tid; e < nb / 16; e += kThreads) umma::cp_async16(sImg + e * 16, img + e * 16);
     }
     umma::cp_async_commit();
     umma::cp_async_wait_all();
@@ -178,7 +191,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ok = wait_mbar(&mbar, phase, &okflag, S.err);
 
-    float m = 0.f, l = 0.f;
     const size_t lb = (size_t)st * dm.mmax + ci;
     const int nK = P.logCount[lb];
     const int *ltok = P.logTok + lb * lam;
@@ -187,45 +199,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     const long long jlo = t0 - eta > 0 ? t0 - eta : 0;
     const int nband = (int)(t1 - jlo);
     const int ntb = (nband + KT - 1) / KT, ntc = (nK + KT - 1) / KT;
+    const int ntiles = ntb + ntc;
     const uint32_t id_s = umma::idesc_bf16(128, KT, false, false);
     const uint32_t id_pv = umma::idesc_bf16(128, d, false, true);
     const bf16 *phiK = (const bf16 *)P.phiK + (size_t)st * (lam + dm.R + dm.Nmax) * D;
 
-    for (int tile = 0; tile < ntb + ntc && ok; ++tile) {
-        const bool band = tile < ntb;
-        const long long kb = band ? jlo + (long long)tile * KT : (long long)(tile - ntb) * KT;
+    // metadata of tile i (threads 0..63, i.e. warps 0 and 1)
+    auto fill_meta = [&](int i, TileMeta &M) {
+        const bool band = i < ntb;
+        const long long kb = band ? jlo + (long long)i * KT : (long long)(i - ntb) * KT;
         const int nk = band ? (int)min((long long)KT, t1 - kb) : min(KT, nK - (int)kb);
-        // key metadata
-        if (tid == 0) anylin = 0;
-        __syncthreads();
-        if (tid < KT) {
-            int tok = -1, info = INFO_SKIP, vr = 0;
-            if (tid < nk) {
-                if (band) {
-                    const long long j = kb + tid;
-                    tok = (int)j;
-                    vr = src.tok2vrow(j);
-                    info = (j < t1 - eta) ? (llf[(int)(j - (t0 - eta))] ? INFO_FOLDED : INFO_SKIP) : INFO_SOFT;
-                    if (info == INFO_FOLDED) anylin = 1;
-                } else {
-                    tok = ltok[kb + tid];
-                    vr = lvrow[kb + tid];
-                    info = INFO_SOFT;
-                }
+        int tok = -1, info = INFO_SKIP, vr = 0;
+        if (tid < nk) {
+            if (band) {
+                const long long j = kb + tid;
+                tok = (int)j;
+                vr = src.tok2vrow(j);
+                info = (j < t1 - eta) ? (llf[(int)(j - (t0 - eta))] ? INFO_FOLDED : INFO_SKIP) : INFO_SOFT;
+            } else {
+                tok = ltok[kb + tid];
+                vr = lvrow[kb + tid];
+                info = INFO_SOFT;
             }
-            ktok[tid] = tok;
-            kinfo[tid] = info;
-            kvrow[tid] = vr;
         }
-        __syncthreads();
-        const bool lin = anylin != 0;
-        // K (K-major [key][d]), V (N-contiguous [key][d]) and, for linear keys, phi(K)
+        M.tok[tid] = tok;
+        M.info[tid] = info;
+        M.vrow[tid] = vr;
+        const bool l_any = __any_sync(0xffffffffu, info == INFO_FOLDED);
+        const bool c_all = __all_sync(0xffffffffu, tid < nk && tok <= pmin);
+        if (lane == 0) {
+            M.lin[warp] = l_any ? 1 : 0;
+            M.causal[warp] = (!band && c_all) ? 1 : 0;
+        }
+        if (tid == 0) {
+            M.nk = nk;
+            M.band = band ? 1 : 0;
+        }
+    };
+    // copies of tile i's keys, values and (for linear keys) phi(K) into buffer bf
+    auto issue_copies = [&](const TileMeta &M, int bf) {
+        uint8_t *sK = base + g.off_K[bf], *sV = base + g.off_V[bf];
+        const int nk = M.nk;
         for (int e = tid; e < (KT << lgd); e += kThreads) {
             const int j = e >> lgd, kc = e & ((1 << lgd) - 1);
             uint8_t *dk = sK + umma::kmajor_offset(j, kc * 8, KT);
             uint8_t *dv = sV + umma::mnmajor_offset(j, kc * 8, d);
             if (j < nk) {
-                const int vr = kvrow[j];
+                const int vr = M.vrow[j];
                 umma::cp_async16(dk, src.krow(st, vr) + kc * 8);
                 umma::cp_async16(dv, src.vrow(st, vr) + kc * 8);
             } else {
@@ -233,22 +253,34 @@ __global__ void __launch_bounds__(kThreads, 1)
                 *(uint4 *)dv = make_uint4(0, 0, 0, 0);
             }
         }
-        if (lin) {
+        if (M.lin[0] | M.lin[1]) {
             for (int e = tid; e < (KT << lgf); e += kThreads) {
                 const int j = e >> lgf, kc = e & ((1 << lgf) - 1);
                 uint8_t *dst = sPhk + umma::kmajor_offset(j, kc * 8, KT);
-                if (j < nk && kc * 8 < D) umma::cp_async16(dst, phiK + (size_t)kvrow[j] * D + kc * 8);
+                if (j < nk && kc * 8 < D) umma::cp_async16(dst, phiK + (size_t)M.vrow[j] * D + kc * 8);
                 else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
             }
         }
         umma::cp_async_commit();
+    };
+
+    float m = 0.f, lpart = 0.f;
+    if (ntiles > 0 && ok) {
+        if (tid < KT) fill_meta(0, meta[0]);
+        __syncthreads();
+        issue_copies(meta[0], 0);
+    }
+    const int nch = g.NB / 16, split = (nch + 1) / 2;   // O chunks rescaled by half 0 / half 1
+    for (int i = 0; i < ntiles && ok; ++i) {
+        const TileMeta &M = meta[i & 1];
         umma::cp_async_wait_all();
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
+        const bool lin = (M.lin[0] | M.lin[1]) != 0;
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t q0 = umma::smem_u32(sQ), k0 = umma::smem_u32(sK);
+            const uint32_t q0 = umma::smem_u32(sQ), k0 = umma::smem_u32(base + g.off_K[i & 1]);
             for (int ks = 0; ks < d / 16; ++ks)
                 umma::mma_ss(tS, umma::kmajor_desc(q0, ks, 128), umma::kmajor_desc(k0, ks, KT), id_s, ks > 0 ? 1u : 0u);
             if (lin) {
@@ -259,9 +291,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma::mma_commit(&mbar);
         }
+        if (i + 1 < ntiles && tid < KT) fill_meta(i + 1, meta[(i + 1) & 1]);
         if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
+        // tile i+1 loads while tile i is finished (its phi(K) buffer is free: G is done)
+        if (i + 1 < ntiles) issue_copies(meta[(i + 1) & 1], (i + 1) & 1);
 
-        // softmax / linear weights of row `tid`
+        // ---- softmax / linear weights; this half exponentiates keys [32*half, 32*half + 32)
         float sv[KT];
 #pragma unroll
         for (int c0 = 0; c0 < KT; c0 += 16) {
@@ -269,101 +304,128 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::tmem_ld16(tS + lane_off + (uint32_t)c0, v);
             umma::tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 16; ++i) sv[c0 + i] = v[i] * scale;
+            for (int j = 0; j < 16; ++j) sv[c0 + j] = v[j] * scale;
         }
+        const bool fast = (M.causal[0] & M.causal[1]) != 0;
         float tmax = -INFINITY;
+        if (fast) {
 #pragma unroll
-        for (int j = 0; j < KT; ++j) {
-            const int info = kinfo[j], tok = ktok[j];
-            const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
-            if (soft) tmax = fmaxf(tmax, sv[j]);
+            for (int j = 0; j < KT; ++j) tmax = fmaxf(tmax, sv[j]);
+        } else {
+#pragma unroll
+            for (int j = 0; j < KT; ++j) {
+                const int info = M.info[j], tok = M.tok[j];
+                const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
+                if (soft) tmax = fmaxf(tmax, sv[j]);
+            }
         }
-        // rescale this row's accumulator when its shift grows; TMEM loads and
-        // stores are warp-collective, so the whole warp takes the branch
         const bool grow_m = tmax > m;
         if (__any_sync(0xffffffffu, grow_m)) {
+            // TMEM accesses are warp-collective: the whole warp rescales its chunk range
             const float f = grow_m ? __expf(m - tmax) : 1.f;
-            l *= f;
-            for (int c0 = 0; c0 < NB; c0 += 16) {
+            lpart *= f;
+            const int cb = half ? split : 0, ce = half ? nch : split;
+            for (int cc = cb; cc < ce; ++cc) {
                 float v[16];
-                umma::tmem_ld16(tO + lane_off + (uint32_t)c0, v);
+                umma::tmem_ld16(tO + lane_off + (uint32_t)(cc * 16), v);
                 umma::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) v[i] *= f;
-                umma::tmem_st16(tO + lane_off + (uint32_t)c0, v);
+                for (int j = 0; j < 16; ++j) v[j] *= f;
+                umma::tmem_st16(tO + lane_off + (uint32_t)(cc * 16), v);
             }
             umma::tmem_wait_st();
             if (grow_m) m = tmax;
         }
-        const float em = __expf(-m);
-        float gv[KT];
+        float gv[32];
         if (lin) {
 #pragma unroll
-            for (int c0 = 0; c0 < KT; c0 += 16) {
+            for (int c0 = 0; c0 < 32; c0 += 16) {
                 float v[16];
-                umma::tmem_ld16(tG + lane_off + (uint32_t)c0, v);
+                umma::tmem_ld16(tG + lane_off + (uint32_t)(half * 32 + c0), v);
                 umma::tmem_wait_ld();
 #pragma unroll
-                for (int i = 0; i < 16; ++i) gv[c0 + i] = v[i];
+                for (int j = 0; j < 16; ++j) gv[c0 + j] = v[j];
             }
         }
+        const float em = __expf(-m);
         float rs = 0.f;
 #pragma unroll
-        for (int j0 = 0; j0 < KT; j0 += 8) {
-            __align__(16) bf16 pk[8];
+        for (int j0 = 0; j0 < 32; j0 += 8) {
+            float pf[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
-                const int j = j0 + jj;
-                const int info = kinfo[j], tok = ktok[j];
-                float pw = 0.f;
-                if (info != INFO_SKIP && tok <= p) {
-                    if (info == INFO_FOLDED && tok <= p - eta) pw = lin ? gv[j] * em : 0.f;
-                    else pw = __expf(sv[j] - m);
+                const int k = j0 + jj, j = half * 32 + k;
+                const float s = half ? sv[32 + k] : sv[k];   // static indices keep sv in registers
+                float pw;
+                if (fast) {
+                    pw = __expf(s - m);
+                } else {
+                    const int info = M.info[j], tok = M.tok[j];
+                    pw = 0.f;
+                    if (info != INFO_SKIP && tok <= p) {
+                        if (info == INFO_FOLDED && tok <= p - eta) pw = lin ? gv[k] * em : 0.f;
+                        else pw = __expf(s - m);
+                    }
                 }
-                if (!row_ok) pw = 0.f;
-                const bf16 pb = __float2bfloat16_rn(pw);
-                rs += __bfloat162float(pb);
-                pk[jj] = pb;
+                pf[jj] = row_ok ? pw : 0.f;
             }
-            *(uint4 *)(sP + umma::kmajor_offset(tid, j0, 128)) = *(const uint4 *)pk;
+            uint4 pk;
+            pk.x = umma::pack_bf16x2(pf[0], pf[1]);
+            pk.y = umma::pack_bf16x2(pf[2], pf[3]);
+            pk.z = umma::pack_bf16x2(pf[4], pf[5]);
+            pk.w = umma::pack_bf16x2(pf[6], pf[7]);
+            // the row sum uses the rounded weights the tensor core multiplies
+            rs += umma::bf16lo_to_f32(pk.x) + umma::bf16hi_to_f32(pk.x) + umma::bf16lo_to_f32(pk.y) +
+                  umma::bf16hi_to_f32(pk.y) + umma::bf16lo_to_f32(pk.z) + umma::bf16hi_to_f32(pk.z) +
+                  umma::bf16lo_to_f32(pk.w) + umma::bf16hi_to_f32(pk.w);
+            *(uint4 *)(sP + umma::kmajor_offset(r, half * 32 + j0, 128)) = pk;
         }
-        l += rs;
+        lpart += rs;
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t p0 = umma::smem_u32(sP), v0 = umma::smem_u32(sV);
+            const uint32_t p0 = umma::smem_u32(sP), v0 = umma::smem_u32(base + g.off_V[i & 1]);
             for (int ks = 0; ks < KT / 16; ++ks)
                 umma::mma_ss(tO, umma::kmajor_desc(p0, ks, 128), umma::mnmajor_desc(v0, ks, d), id_pv, 1u);
             umma::mma_commit(&mbar);
         }
         if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
     }
+    umma::cp_async_wait_all();
 
     if (ok) {
-        // ---- 3. normalise and store
-        float den_lin;
-        {
-            float v[16];
-            umma::tmem_ld16(tO + lane_off + (uint32_t)d, v);
-            umma::tmem_wait_ld();
-            den_lin = v[0];
-        }
-        const float den = l + den_lin + dm.eps * __expf(-m);
+        // ---- 3. normalise and store; half h writes value columns [h*d/2, (h+1)*d/2)
+        if (half == 1) red[r] = lpart;
+        __syncthreads();
+        const float l = half == 0 ? lpart + red[r] : 0.f;
+        __syncthreads();
+        if (half == 0) red[r] = l;
+        __syncthreads();
+        const float lt = red[r];
+        float v[16];
+        umma::tmem_ld16(tO + lane_off + (uint32_t)d, v);
+        umma::tmem_wait_ld();
+        const float den = lt + v[0] + dm.eps * __expf(-m);
         const float rden = 1.f / den;
         bf16 *out = (bf16 *)a.out;
         const size_t orow = qrow0 + (size_t)(grow / gq) * dm.Hq + grow % gq;
-        for (int c0 = 0; c0 < d; c0 += 16) {
-            float v[16];
+        for (int c0 = half * (d / 2); c0 < (half + 1) * (d / 2); c0 += 16) {
             umma::tmem_ld16(tO + lane_off + (uint32_t)c0, v);
             umma::tmem_wait_ld();
             if (row_ok) {
-                __align__(16) bf16 o[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) o[i] = __float2bfloat16_rn(v[i] * rden);
-                *(uint4 *)(out + orow * d + c0) = *(const uint4 *)o;
-                *(uint4 *)(out + orow * d + c0 + 8) = *(const uint4 *)(o + 8);
+                uint4 o0, o1;
+                o0.x = umma::pack_bf16x2(v[0] * rden, v[1] * rden);
+                o0.y = umma::pack_bf16x2(v[2] * rden, v[3] * rden);
+                o0.z = umma::pack_bf16x2(v[4] * rden, v[5] * rden);
+                o0.w = umma::pack_bf16x2(v[6] * rden, v[7] * rden);
+                o1.x = umma::pack_bf16x2(v[8] * rden, v[9] * rden);
+                o1.y = umma::pack_bf16x2(v[10] * rden, v[11] * rden);
+                o1.z = umma::pack_bf16x2(v[12] * rden, v[13] * rden);
+                o1.w = umma::pack_bf16x2(v[14] * rden, v[15] * rden);
+                *(uint4 *)(out + orow * d + c0) = o0;
+                *(uint4 *)(out + orow * d + c0 + 8) = o1;
             }
         }
     } else if (tid == 0) {

@@ -239,11 +239,17 @@ __device__ void refresh_image(Ctx &c)
             float v[16];
             umma::tmem_ld16(row + (uint32_t)c0, v);
             umma::tmem_wait_ld();
-            __align__(16) bf16 h[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) h[i] = __float2bfloat16_rn(v[i]);
-            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0, c.g.d)) = *(const uint4 *)h;
-            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0 + 8, c.g.d)) = *(const uint4 *)(h + 8);
+            uint4 h0, h1;
+            h0.x = umma::pack_bf16x2(v[0], v[1]);
+            h0.y = umma::pack_bf16x2(v[2], v[3]);
+            h0.z = umma::pack_bf16x2(v[4], v[5]);
+            h0.w = umma::pack_bf16x2(v[6], v[7]);
+            h1.x = umma::pack_bf16x2(v[8], v[9]);
+            h1.y = umma::pack_bf16x2(v[10], v[11]);
+            h1.z = umma::pack_bf16x2(v[12], v[13]);
+            h1.w = umma::pack_bf16x2(v[14], v[15]);
+            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0, c.g.d)) = h0;
+            *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0 + 8, c.g.d)) = h1;
         }
         float v[16];
         umma::tmem_ld16(row + (uint32_t)c.g.d, v);
