@@ -127,12 +127,9 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->Nmax = nmax;
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
+    // decode: 128 keys per CTA over the largest key set (cache + window + interval)
     const long long nkeys = (long long)dm->lam + dm->eta + dm->Cdec;
-    const long long tiles = (nkeys + 31) / 32;
-    long long ns = (296 + dm->ns - 1) / dm->ns;
-    if (ns > tiles) ns = tiles;
-    if (ns < 1) ns = 1;
-    dm->nsplit = (int)ns;
+    dm->nsplit = (int)((nkeys + 127) / 128);
     dm->tc_chain = (c->dtype == LOLA_BF16 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
