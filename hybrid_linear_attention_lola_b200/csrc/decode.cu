@@ -42,6 +42,13 @@ __global__ void append_kernel(Dims dm, DevState S, const T *__restrict__ k, cons
 constexpr int DT = 128;
 constexpr int KPC = 128;
 
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                 ::"r"(static_cast<uint32_t>(__cvta_generic_to_shared(smem))), "l"(gmem)
+                 : "memory");
+}
+
 template <typename T, int DPL>
 __device__ __forceinline__ void load_row(const T *row, int lane, float (&v)[DPL])
 {
@@ -49,23 +56,69 @@ __device__ __forceinline__ void load_row(const T *row, int lane, float (&v)[DPL]
     for (int u = 0; u < DPL; ++u) v[u] = to_f<T>(row[lane * DPL + u]);
 }
 
+template <typename T> struct Vec8;   // 16 bytes of T -> 8 (bf16) or 4 (fp32) floats
+template <> struct Vec8<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ static void load(const void *p, float *f)
+    {
+        const uint4 r = *(const uint4 *)p;
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            f[2 * i] = __uint_as_float(w[i] << 16);
+            f[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+template <> struct Vec8<float> {
+    static constexpr int N = 4;
+    __device__ static void load(const void *p, float *f)
+    {
+        const float4 r = *(const float4 *)p;
+        f[0] = r.x; f[1] = r.y; f[2] = r.z; f[3] = r.w;
+    }
+};
+
+struct DecodeSmem {
+    size_t off_phq, off_rows, off_kv, kstride, vstride, warp_bytes, total;
+};
+
+template <typename T, int DPL>
+__host__ __device__ inline DecodeSmem decode_smem_layout(int D)
+{
+    constexpr int d = 32 * DPL;
+    DecodeSmem L{};
+    L.off_phq = (size_t)8 * d * 4;                                   // queries (fp32)
+    L.off_rows = L.off_phq + (size_t)8 * D * 4;                       // features (fp32)
+    L.off_kv = L.off_rows + 4 * 32 * 4;                               // per-warp key rows
+    L.kstride = (size_t)d * sizeof(T) + 16;                           // padded key row
+    L.vstride = (size_t)d * sizeof(T);
+    L.warp_bytes = 32 * (L.kstride + L.vstride);
+    const size_t kv = 4 * L.warp_bytes;
+    const size_t red = (size_t)4 * 8 * (3 + 2 * d) * 4;               // per-warp partials (aliases kv)
+    L.total = L.off_kv + (kv > red ? kv : red);
+    return L;
+}
+
 template <typename T, int DPL>
 __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, DecodeArgs a, int hpc)
 {
     constexpr int d = 32 * DPL;
+    constexpr int VN = Vec8<T>::N;                   // elements per 16-byte chunk
+    constexpr int CPR = d / VN;                      // 16-byte chunks per row
     const int split = blockIdx.x, st = blockIdx.y;
     const int b = st / dm.Hkv, hk = st % dm.Hkv;
     const int D = dm.D, g = dm.g, lam = dm.lam, R = dm.R;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    __shared__ float qs[8 * d];                  // queries of the group, scaled by 1/sqrt(d)
-    __shared__ float phq[8 * 256];               // their features
-    __shared__ float red[4][8][3 + 2 * d];       // per-warp partials
+    const DecodeSmem L = decode_smem_layout<T, DPL>(D);
+    extern __shared__ __align__(16) uint8_t smd[];
+    float *qs = (float *)smd;                        // [g][d], scaled by 1/sqrt(d)
+    float *phq = (float *)(smd + L.off_phq);         // [g][D]
+    int *rowtab = (int *)(smd + L.off_rows) + warp * 32;
+    uint8_t *wk = smd + L.off_kv + warp * L.warp_bytes;   // this warp's 32 key rows (padded)
+    uint8_t *wv = wk + 32 * L.kstride;                    // and value rows
+    float *red = (float *)(smd + L.off_kv);               // [4][8][3 + 2d], after the keys are done
     const float scale = rsqrtf((float)d);
-    const T *q = (const T *)a.q + ((size_t)b * dm.Hq + (size_t)hk * g) * d;
-    const T *pq = (const T *)S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
-    for (int e = tid; e < g * d; e += DT) qs[e] = to_f<T>(q[e]) * scale;
-    for (int e = tid; e < g * D; e += DT) phq[e] = to_f<T>(pq[e]);
-    __syncthreads();
 
     const long long p = a.pos;
     const long long jlo = a.t0 - dm.eta > 0 ? a.t0 - dm.eta : 0;
@@ -78,6 +131,43 @@ __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, Decode
     const T *VR = (const T *)S.VR + (size_t)st * R * d;
     const T *phiV = (const T *)S.phiV + (size_t)st * (lam + R) * D;
 
+    // this lane's key: class and row (< lam: cache slot, else lam + ring slot)
+    const int kk0 = k0 + warp * 32;
+    const int key = kk0 + lane;
+    const int nvalid = kk0 < k1 ? min(32, k1 - kk0) : 0;     // warp-uniform
+    int cls = 0, row = 0;                                     // cls: 0 skip, 1 softmax, 2 linear
+    if (key < k1) {
+        if (key < a.nS) {
+            row = key;
+            cls = 1;
+        } else {
+            const long long j = jlo + (key - a.nS);
+            row = lam + (int)(j & (R - 1));
+            if (j >= a.L_lo && j < a.L_hi)
+                cls = S.pend[(size_t)st * dm.Lmax + (int)(j - a.L_lo)] ? (j <= p - dm.eta ? 2 : 1) : 0;
+            else
+                cls = 1;
+        }
+    }
+    rowtab[lane] = row;
+    __syncwarp();
+    // stage the warp's key and value rows with coalesced 16-byte copies
+    for (int e = lane; e < nvalid * CPR; e += 32) {
+        const int jj = e / CPR, cc = e - jj * CPR;
+        const int rw = rowtab[jj];
+        const T *ksrc = rw < lam ? KS + (size_t)rw * d : KR + (size_t)(rw - lam) * d;
+        const T *vsrc = rw < lam ? VS + (size_t)rw * d : VR + (size_t)(rw - lam) * d;
+        cp_async16(wk + jj * L.kstride + cc * 16, ksrc + cc * VN);
+        cp_async16(wv + jj * L.vstride + cc * 16, vsrc + cc * VN);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+    const T *qg = (const T *)a.q + ((size_t)b * dm.Hq + (size_t)hk * g) * d;
+    const T *pqg = (const T *)S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
+    for (int e = tid; e < g * d; e += DT) qs[e] = to_f<T>(qg[e]) * scale;
+    for (int e = tid; e < g * D; e += DT) phq[e] = to_f<T>(pqg[e]);
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+
     float m[8], l[8], ld[8], o[8][DPL], lo[8][DPL];
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
@@ -88,42 +178,29 @@ __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, Decode
         for (int u = 0; u < DPL; ++u) o[h][u] = lo[h][u] = 0.f;
     }
 
-    const int kk0 = k0 + warp * 32;
-    if (kk0 < k1) {
-        const int key = kk0 + lane;
-        const bool valid = key < k1;
-        int cls = 0;                    // 0 skip, 1 softmax, 2 linear
-        int row = 0;                    // < lam: cache slot; else lam + ring slot
-        if (valid) {
-            if (key < a.nS) {
-                row = key;
-                cls = 1;
-            } else {
-                const long long j = jlo + (key - a.nS);
-                row = lam + (int)(j & (R - 1));
-                if (j >= a.L_lo && j < a.L_hi)
-                    cls = S.pend[(size_t)st * dm.Lmax + (int)(j - a.L_lo)] ? (j <= p - dm.eta ? 2 : 1) : 0;
-                else
-                    cls = 1;
-            }
-        }
-        const T *krow = row < lam ? KS + (size_t)row * d : KR + (size_t)(row - lam) * d;
-        const T *vrow = row < lam ? VS + (size_t)row * d : VR + (size_t)(row - lam) * d;
-        // scores of this lane's key for every head
+    if (nvalid > 0) {
+        // scores of this lane's key for every head (key row from shared memory)
         float sc[8];
 #pragma unroll
         for (int h = 0; h < 8; ++h) sc[h] = 0.f;
         if (cls == 1) {
-            for (int c0 = 0; c0 < d; c0 += 8) {
-                float kf[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) kf[u] = to_f<T>(krow[c0 + u]);
+            const uint8_t *kr = wk + lane * L.kstride;
+#pragma unroll 4
+            for (int cc = 0; cc < CPR; ++cc) {
+                float kf[VN];
+                Vec8<T>::load(kr + cc * 16, kf);
 #pragma unroll
                 for (int h = 0; h < 8; ++h) {
                     if (h < g) {
-                        const float *qh = qs + h * d + c0;
+                        const float *qh = qs + h * d + cc * VN;
 #pragma unroll
-                        for (int u = 0; u < 8; ++u) sc[h] = fmaf(qh[u], kf[u], sc[h]);
+                        for (int u = 0; u < VN; u += 4) {
+                            const float4 q4 = *(const float4 *)(qh + u);
+                            sc[h] = fmaf(q4.x, kf[u], sc[h]);
+                            sc[h] = fmaf(q4.y, kf[u + 1], sc[h]);
+                            sc[h] = fmaf(q4.z, kf[u + 2], sc[h]);
+                            sc[h] = fmaf(q4.w, kf[u + 3], sc[h]);
+                        }
                     }
                 }
             }
@@ -157,13 +234,12 @@ __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, Decode
                 pw[h] = 0.f;
             }
         }
-        // P V over the warp's keys: lane owns value dims [lane*DPL, lane*DPL + DPL)
-        const int nvalid = min(32, k1 - kk0);
-        const unsigned long long vaddr = (unsigned long long)vrow;
+        // P V: lane owns value dims [lane*DPL, lane*DPL + DPL); rows from shared memory
         for (int jj = 0; jj < nvalid; ++jj) {
-            const T *vr = (const T *)__shfl_sync(0xffffffffu, vaddr, jj);
+            const T *vr = (const T *)(wv + jj * L.vstride);
             float vf[DPL];
-            load_row<T, DPL>(vr, lane, vf);
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) vf[u] = to_f<T>(vr[lane * DPL + u]);
 #pragma unroll
             for (int h = 0; h < 8; ++h) {
                 if (h < g) {
@@ -199,19 +275,21 @@ __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, Decode
             }
         }
     }
+    __syncthreads();   // the staged rows are dead: red[] reuses their space
     // combine the 4 warps, then write this CTA's partial per head
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
         if (h < g) {
+            float *rw = red + (warp * 8 + h) * (3 + 2 * d);
             if (lane == 0) {
-                red[warp][h][0] = m[h];
-                red[warp][h][1] = l[h];
-                red[warp][h][2] = ld[h];
+                rw[0] = m[h];
+                rw[1] = l[h];
+                rw[2] = ld[h];
             }
 #pragma unroll
             for (int u = 0; u < DPL; ++u) {
-                red[warp][h][3 + lane * DPL + u] = o[h][u];
-                red[warp][h][3 + d + lane * DPL + u] = lo[h][u];
+                rw[3 + lane * DPL + u] = o[h][u];
+                rw[3 + d + lane * DPL + u] = lo[h][u];
             }
         }
     }
@@ -219,25 +297,26 @@ __global__ void __launch_bounds__(DT) decode2_kernel(Dims dm, DevState S, Decode
     for (int h = warp; h < g; h += 4) {
         float M = 0.f;
 #pragma unroll
-        for (int w = 0; w < 4; ++w) M = fmaxf(M, red[w][h][0]);
-        float L = 0.f, LD = 0.f, O[DPL], LO[DPL];
+        for (int w = 0; w < 4; ++w) M = fmaxf(M, red[(w * 8 + h) * (3 + 2 * d)]);
+        float Ls = 0.f, LD = 0.f, O[DPL], LO[DPL];
 #pragma unroll
         for (int u = 0; u < DPL; ++u) O[u] = LO[u] = 0.f;
 #pragma unroll
         for (int w = 0; w < 4; ++w) {
-            const float f = __expf(red[w][h][0] - M);
-            L = fmaf(f, red[w][h][1], L);
-            LD += red[w][h][2];
+            const float *rw = red + (w * 8 + h) * (3 + 2 * d);
+            const float f = __expf(rw[0] - M);
+            Ls = fmaf(f, rw[1], Ls);
+            LD += rw[2];
 #pragma unroll
             for (int u = 0; u < DPL; ++u) {
-                O[u] = fmaf(f, red[w][h][3 + lane * DPL + u], O[u]);
-                LO[u] += red[w][h][3 + d + lane * DPL + u];
+                O[u] = fmaf(f, rw[3 + lane * DPL + u], O[u]);
+                LO[u] += rw[3 + d + lane * DPL + u];
             }
         }
         float *pr = S.part + (((size_t)st * dm.nsplit + split) * g + h) * (2 * d + 4);
         if (lane == 0) {
             pr[0] = M;
-            pr[1] = L;
+            pr[1] = Ls;
             pr[2] = LD;
             pr[3] = 0.f;
         }
@@ -314,7 +393,13 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
     launch_phi_q(dm, S.W, a.q, (long long)dm.B * dm.Hq, S.phiQd, stream);
     dim3 grid(dm.nsplit, dm.ns);
     const int hpc = (dm.D + dm.nsplit - 1) / dm.nsplit;
-#define LOLA_DECODE2(T, DPL) decode2_kernel<T, DPL><<<grid, DT, 0, stream>>>(dm, S, a, hpc)
+#define LOLA_DECODE2(T, DPL)                                                                       \
+    do {                                                                                           \
+        const size_t smem = decode_smem_layout<T, DPL>(dm.D).total;                                \
+        cudaFuncSetAttribute(decode2_kernel<T, DPL>, cudaFuncAttributeMaxDynamicSharedMemorySize,  \
+                             (int)smem);                                                           \
+        decode2_kernel<T, DPL><<<grid, DT, smem, stream>>>(dm, S, a, hpc);                         \
+    } while (0)
     if (dm.dtype == 0) {
         if (dm.d == 32) LOLA_DECODE2(float, 1);
         else if (dm.d == 64) LOLA_DECODE2(float, 2);
