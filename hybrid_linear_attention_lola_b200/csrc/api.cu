@@ -127,9 +127,15 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->Nmax = nmax;
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
-    // decode: 128 keys per CTA over the largest key set (cache + window + interval)
+    // decode: 32-key chunks, 4 warps per CTA; enough chunks per warp that the
+    // grid is about four CTAs per SM over the largest key set
     const long long nkeys = (long long)dm->lam + dm->eta + dm->Cdec;
-    dm->nsplit = (int)((nkeys + 127) / 128);
+    const long long chunks = (nkeys + 31) / 32;
+    long long nch = (chunks * dm->ns + 4 * 148 * 4 - 1) / (4 * 148 * 4);
+    if (nch < 1) nch = 1;
+    if (nch > 16) nch = 16;
+    dm->dec_nch = (int)nch;
+    dm->nsplit = (int)((chunks + 4 * nch - 1) / (4 * nch));
     dm->tc_chain = (c->dtype == LOLA_BF16 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
@@ -164,6 +170,7 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
     s.phiQd = take((size_t)dm.B * dm.Hq * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
+    s.dec_cnt = (int *)take(ns * 4);
     lola::PrefillScratch p{};
     const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
     p.phiK = take(ns * nv * dm.D * e);

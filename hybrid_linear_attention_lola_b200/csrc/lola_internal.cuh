@@ -23,7 +23,8 @@ enum : int { ERR_BOUNDS = 1, ERR_TIMEOUT = 2 };
 struct Dims {
     int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
     int Nmax, mmax;   // prefill scratch capacity: tokens per call, intervals per call
-    int nsplit;       // decode key splits per stream
+    int nsplit;       // decode key splits (CTAs) per stream
+    int dec_nch;      // decode: 32-key chunks per warp (4 warps per CTA)
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
     float eps;
@@ -43,6 +44,7 @@ struct DevState {
     void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
     void *phiQd;       // [B][Hq][D]
     float *part;       // [ns][nsplit][g][2d + 4] split partials
+    int *dec_cnt;      // [ns] finished decode CTAs per stream (reset by the last one)
 };
 
 // Per-prefill-call scratch.

@@ -171,6 +171,7 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
     if (W != nullptr)
         for (long long e = tid; e < (long long)dm.d * dm.Dh; e += stride) S.W[e] = to_f<T>(W[e]);
     if (tid < 4) S.err[tid] = 0;
+    for (long long e = tid; e < dm.ns; e += stride) S.dec_cnt[e] = 0;
 }
 
 void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream)
