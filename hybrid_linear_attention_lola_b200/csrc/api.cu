@@ -30,6 +30,13 @@ struct lola_state {
     long long pend_lo;       // leaving pairs of the last interval: [pend_lo, pend_lo + pend_n)
     int pend_n;
     long long n_int;         // update intervals run since init/reset
+    bool phiV_valid;         // phi rows of the cache slots and the ring are current
+    // prefill segments: chain on a high-priority library stream, attention on the caller's
+    static constexpr int kMaxSeg = 64;
+    int seg_len;                     // intervals per segment (0: the whole call)
+    cudaStream_t chain_stream;
+    cudaEvent_t ev_fork;
+    cudaEvent_t ev_seg[kMaxSeg];
     int32_t *sel_log;
     long long sel_cap;
     const int32_t *ovr;
@@ -127,19 +134,12 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->Nmax = nmax;
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
-    // decode: 32-key chunks, 4 warps per CTA; enough chunks per warp that the
-    // grid is about four CTAs per SM over the largest key set
-    const long long nkeys = (long long)dm->lam + dm->eta + dm->Cdec;
-    const long long chunks = (nkeys + 31) / 32;
-    long long nch = (chunks * dm->ns + 4 * 148 * 4 - 1) / (4 * 148 * 4);
-    if (nch < 1) nch = 1;
-    if (nch > 16) nch = 16;
-    dm->dec_nch = (int)nch;
-    dm->nsplit = (int)((chunks + 4 * nch - 1) / (4 * nch));
+    if (!lola::decode_plan(dm)) return LOLA_ERR_INVALID_ARG;
     dm->tc_chain = (c->dtype == LOLA_BF16 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
+    if (c->dtype == LOLA_BF16 && lola::phi_tc_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     return LOLA_OK;
 }
 
@@ -167,14 +167,14 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.VR = take(ns * dm.R * dm.d * e);
     s.pend = (uint8_t *)take(ns * dm.Lmax);
     s.W = (float *)take((size_t)dm.d * dm.Dh * 4);
+    s.Wt = take((size_t)dm.d * dm.Dh * e);
     s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
-    s.phiQd = take((size_t)dm.B * dm.Hq * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     s.dec_cnt = (int *)take(ns * 4);
     lola::PrefillScratch p{};
     const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
     p.phiK = take(ns * nv * dm.D * e);
-    p.phiQ = take((size_t)dm.B * dm.Nmax * dm.Hq * dm.D * e);
+    p.phiQ = dm.tc_attn ? nullptr : take((size_t)dm.B * dm.Nmax * dm.Hq * dm.D * e);
     p.snapH = (float *)take(dm.tc_attn ? 0 : ns * dm.mmax * dm.D * dm.d * 4);
     p.snapS = (float *)take(dm.tc_attn ? 0 : ns * dm.mmax * dm.D * 4);
     p.snapImg = dm.tc_chain ? take(ns * dm.mmax * lola::snap_image_bytes(dm)) : nullptr;
@@ -210,6 +210,7 @@ void reset_host(lola_state *st)
     st->pend_lo = 0;
     st->pend_n = 0;
     st->n_int = 0;
+    st->phiV_valid = false;
 }
 
 // Host mirror of one interval's bookkeeping (identical for every stream).
@@ -226,6 +227,84 @@ void advance_interval(lola_state *st, long long t0, int len)
     st->pend_lo = lo;
     st->pend_n = nL;
     st->n_int += 1;
+}
+
+// One decode step. `part` receives the split partials of the decode attention.
+lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const void *v, void *out,
+                             void *cuda_stream, float *part)
+{
+    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+        return LOLA_ERR_INVALID_ARG;
+    const Dims &dm = st->dm;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    const long long pos = st->pos;
+    int do_append = 1;
+    if (pos == st->interval_end) {
+        // an update interval opens: the new pair joins the ring first (it may
+        // already be a leaving pair), then score / select / fold
+        {
+            PhaseScope ps(st, PH_APPEND, stream);
+            lola::launch_decode_append(dm, st->S, k, v, pos, st->phiV_valid ? 1 : 0, stream);
+            counted(1);
+        }
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+        do_append = 0;
+        PhaseScope ps(st, PH_UPDATE, stream);
+        if (!st->phiV_valid) {
+            if (dm.dtype == LOLA_BF16)
+                lola::launch_phi_kv_tc(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, st->S.phiV, st->nS, stream);
+            else
+                lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
+            counted(1);
+        }
+        lola::ChainArgs ca{};
+        ca.mode = 1;
+        ca.pos0 = pos;
+        ca.n_int = 1;
+        ca.ilen = dm.Cdec;
+        ca.call_start = 0;
+        ca.n_call = 0;
+        ca.kin = nullptr;
+        ca.vin = nullptr;
+        ca.nS0 = st->nS;
+        ca.pend_lo = st->pend_lo;
+        ca.pend_n = st->pend_n;
+        ca.iglob0 = st->n_int;
+        ca.phi = st->S.phiV;
+        ca.nvrows = dm.lam + dm.R;
+        ca.sel_log = st->sel_log;
+        ca.sel_cap = st->sel_cap;
+        ca.ovr = st->ovr;
+        ca.ovr_n = st->ovr_n;
+        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
+        else lola::launch_chain(dm, st->S, nullptr, ca, stream);
+        counted(1);
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+        st->phiV_valid = true;
+        advance_interval(st, pos, dm.Cdec);
+        st->t0_open = pos;
+        st->interval_end = pos + dm.Cdec;
+    }
+    lola::DecodeArgs da{};
+    da.pos = pos;
+    da.t0 = st->t0_open;
+    da.nS = st->nS;
+    da.L_lo = st->pend_lo;
+    da.L_hi = st->pend_lo + st->pend_n;
+    da.q = q;
+    da.k = k;
+    da.v = v;
+    da.out = out;
+    lola::DevState Sx = st->S;
+    Sx.part = part;
+    {
+        PhaseScope ps(st, PH_DECODE, stream);
+        lola::launch_decode_attn(dm, Sx, da, do_append, stream);
+        counted(1);
+    }
+    st->pos = pos + 1;
+    return check_launch();
 }
 
 }  // namespace
@@ -289,6 +368,26 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     layout(dm, (char *)workspace, &st->S, &st->P);
     reset_host(st);
     st->timing = false;
+    st->seg_len = 0;
+    st->chain_stream = nullptr;
+    if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
+        // segments of at least 4 intervals, at most kMaxSeg of them per call
+        int len = dm.mmax / 32;
+        if (len < 4) len = 4;
+        while ((dm.mmax + len - 1) / len > lola_state::kMaxSeg) ++len;
+        int lo = 0, hi = 0;
+        bool okc = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
+                   cudaStreamCreateWithPriority(&st->chain_stream, cudaStreamNonBlocking, hi) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&st->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+        for (int i = 0; okc && i < lola_state::kMaxSeg; ++i)
+            okc = cudaEventCreateWithFlags(&st->ev_seg[i], cudaEventDisableTiming) == cudaSuccess;
+        if (!okc) {
+            cudaGetLastError();
+            delete st;
+            return LOLA_ERR_CUDA;
+        }
+        st->seg_len = len;
+    }
     lola::launch_init_state(dm, st->S, W, (cudaStream_t)cuda_stream);
     counted(1);
     r = check_launch();
@@ -330,59 +429,94 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     const long long pos0 = st->pos;
 
     {
+        // phi of the keys (cache slots, ring, call tokens); phi of the queries is
+        // computed inside the tensor-core attention kernel
         PhaseScope ps(st, PH_PHI, stream);
-        lola::launch_phi_kv(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, 0, st->P.phiK, st->nS,
-                            stream);
-        lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
-        counted(2);
+        if (dm.dtype == LOLA_BF16) {
+            lola::launch_phi_kv_tc(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, st->P.phiK, st->nS,
+                                   stream);
+            counted(1);
+            if (!dm.tc_attn) {
+                lola::launch_phi_q_tc(dm, st->S, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
+                counted(1);
+            }
+        } else {
+            lola::launch_phi_kv(dm, st->S, k, pos0, n, dm.lam + dm.R + dm.Nmax, 0, st->P.phiK, st->nS,
+                                stream);
+            lola::launch_phi_q(dm, st->S.W, q, (long long)dm.B * n * dm.Hq, st->P.phiQ, stream);
+            counted(2);
+        }
     }
     if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
-    lola::ChainArgs ca{};
-    ca.mode = 0;
-    ca.pos0 = pos0;
-    ca.n_int = m;
-    ca.ilen = dm.C;
-    ca.call_start = pos0;
-    ca.n_call = n;
-    ca.kin = k;
-    ca.vin = v;
-    ca.nS0 = st->nS;
-    ca.pend_lo = st->pend_lo;
-    ca.pend_n = st->pend_n;
-    ca.iglob0 = st->n_int;
-    ca.phi = st->P.phiK;
-    ca.nvrows = dm.lam + dm.R + dm.Nmax;
-    ca.sel_log = st->sel_log;
-    ca.sel_cap = st->sel_cap;
-    ca.ovr = st->ovr;
-    ca.ovr_n = st->ovr_n;
-    {
-        PhaseScope ps(st, PH_CHAIN, stream);
-        ca.snap_f32 = dm.tc_attn ? 0 : 1;
-        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, stream);
-        else lola::launch_chain(dm, st->S, &st->P, ca, stream);
-        counted(1);
+    // The call's intervals run in segments. The chain of a segment (sequential per
+    // stream, a few SMs) runs on the library's high-priority stream; the attention
+    // of the segment follows on the caller's stream once that chain is done, so it
+    // overlaps the chain of the next segments on the other SMs.
+    const int seg = st->seg_len > 0 ? st->seg_len : m;
+    const int nseg = (m + seg - 1) / seg;
+    const bool fork = nseg > 1 && st->chain_stream != nullptr;
+    cudaStream_t cs = fork ? st->chain_stream : stream;
+    if (fork) {
+        cudaEventRecord(st->ev_fork, stream);
+        cudaStreamWaitEvent(cs, st->ev_fork, 0);
     }
-    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+    for (int sg = 0; sg < nseg; ++sg) {
+        const int ci0 = sg * seg;
+        const int ms = m - ci0 < seg ? m - ci0 : seg;
+        lola::ChainArgs ca{};
+        ca.mode = 0;
+        ca.pos0 = pos0 + (long long)ci0 * dm.C;
+        ca.n_int = ms;
+        ca.ilen = dm.C;
+        ca.call_start = pos0;
+        ca.n_call = n;
+        ca.kin = k;
+        ca.vin = v;
+        ca.nS0 = st->nS;
+        ca.pend_lo = st->pend_lo;
+        ca.pend_n = st->pend_n;
+        ca.iglob0 = st->n_int;
+        ca.phi = st->P.phiK;
+        ca.nvrows = dm.lam + dm.R + dm.Nmax;
+        ca.sel_log = st->sel_log;
+        ca.sel_cap = st->sel_cap;
+        ca.ovr = st->ovr;
+        ca.ovr_n = st->ovr_n;
+        ca.ci0 = ci0;
+        ca.cont = sg > 0 ? 1 : 0;
+        {
+            PhaseScope ps(st, PH_CHAIN, cs);
+            ca.snap_f32 = dm.tc_attn ? 0 : 1;
+            if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, cs);
+            else lola::launch_chain(dm, st->S, &st->P, ca, cs);
+            counted(1);
+        }
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+        if (fork) {
+            cudaEventRecord(st->ev_seg[sg], cs);
+            cudaStreamWaitEvent(stream, st->ev_seg[sg], 0);
+        }
+        for (int ci = 0; ci < ms; ++ci) advance_interval(st, pos0 + (long long)(ci0 + ci) * dm.C, dm.C);
 
-    lola::AttnArgs aa{};
-    aa.pos0 = pos0;
-    aa.m = m;
-    aa.n_call = n;
-    aa.q = q;
-    aa.kin = k;
-    aa.vin = v;
-    aa.out = out;
-    {
-        PhaseScope ps(st, PH_ATTN, stream);
-        if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
-        else lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
-        counted(1);
+        lola::AttnArgs aa{};
+        aa.pos0 = pos0;
+        aa.m = ms;
+        aa.ci0 = ci0;
+        aa.n_call = n;
+        aa.q = q;
+        aa.kin = k;
+        aa.vin = v;
+        aa.out = out;
+        {
+            PhaseScope ps(st, PH_ATTN, stream);
+            if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
+            else lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+            counted(1);
+        }
+        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
     }
-    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
-    for (int ci = 0; ci < m; ++ci) advance_interval(st, pos0 + (long long)ci * dm.C, dm.C);
     {
         PhaseScope ps(st, PH_FINAL, stream);
         lola::launch_finalize_prefill(dm, st->S, st->P, k, v, pos0, n, st->nS, stream);
@@ -390,71 +524,15 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     }
     st->pos = pos0 + n;
     st->interval_end = st->pos;
+    st->phiV_valid = false;   // cache slots and ring rows changed outside the decode path
     return check_launch();
 }
 
 lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const void *v,
                              void *out, void *cuda_stream)
 {
-    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-        return LOLA_ERR_INVALID_ARG;
-    const Dims &dm = st->dm;
-    cudaStream_t stream = (cudaStream_t)cuda_stream;
-    const long long pos = st->pos;
-    {
-        PhaseScope ps(st, PH_APPEND, stream);
-        lola::launch_decode_append(dm, st->S, k, v, pos, stream);
-        counted(1);
-    }
-    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
-    if (pos == st->interval_end) {
-        PhaseScope ps(st, PH_UPDATE, stream);
-        lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
-        lola::ChainArgs ca{};
-        ca.mode = 1;
-        ca.pos0 = pos;
-        ca.n_int = 1;
-        ca.ilen = dm.Cdec;
-        ca.call_start = 0;
-        ca.n_call = 0;
-        ca.kin = nullptr;
-        ca.vin = nullptr;
-        ca.nS0 = st->nS;
-        ca.pend_lo = st->pend_lo;
-        ca.pend_n = st->pend_n;
-        ca.iglob0 = st->n_int;
-        ca.phi = st->S.phiV;
-        ca.nvrows = dm.lam + dm.R;
-        ca.sel_log = st->sel_log;
-        ca.sel_cap = st->sel_cap;
-        ca.ovr = st->ovr;
-        ca.ovr_n = st->ovr_n;
-        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
-        else lola::launch_chain(dm, st->S, nullptr, ca, stream);
-        counted(2);
-        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
-        advance_interval(st, pos, dm.Cdec);
-        st->t0_open = pos;
-        st->interval_end = pos + dm.Cdec;
-    }
-    lola::DecodeArgs da{};
-    da.pos = pos;
-    da.t0 = st->t0_open;
-    da.nS = st->nS;
-    da.L_lo = st->pend_lo;
-    da.L_hi = st->pend_lo + st->pend_n;
-    da.q = q;
-    da.k = k;
-    da.v = v;
-    da.out = out;
-    {
-        PhaseScope ps(st, PH_DECODE, stream);
-        lola::launch_decode_attn(dm, st->S, da, stream);
-        counted(3);
-    }
-    st->pos = pos + 1;
-    return check_launch();
+    if (!st) return LOLA_ERR_INVALID_ARG;
+    return decode_step_impl(st, q, k, v, out, cuda_stream, st->S.part);
 }
 
 lola_status lola_get_cache_indices(const lola_state *st, int32_t *dev_idx, int32_t *dev_count,
@@ -532,6 +610,12 @@ lola_status lola_free_state(lola_state *st)
         st->pool.push_back(mk.b);
     }
     for (cudaEvent_t e : st->pool) cudaEventDestroy(e);
+    if (st->chain_stream != nullptr) {
+        cudaStreamSynchronize(st->chain_stream);
+        cudaStreamDestroy(st->chain_stream);
+        cudaEventDestroy(st->ev_fork);
+        for (int i = 0; i < lola_state::kMaxSeg; ++i) cudaEventDestroy(st->ev_seg[i]);
+    }
     delete st;
     return LOLA_OK;
 }
@@ -541,8 +625,8 @@ lola_status lola_free_state(lola_state *st)
 // ---------------------------------------------------------------- decode step, library-owned scratch
 //
 // lola_decode_step_static runs the same decode step as lola_decode_step, but
-// the per-step temporaries of the split decode attention (the query feature
-// rows and the per-split partial sums) live in the fixed device array below
+// the per-step temporaries of the split decode attention (the per-split
+// partial sums of a stream's CTAs) live in the fixed device array below
 // instead of the caller's workspace. It exists for callers that cannot obtain
 // device memory on demand: a host framework that owns all device memory and
 // hands a plugin only its inputs, outputs and persistent state, or code that
@@ -584,71 +668,14 @@ lola_status static_scratch_address(void **out)
 extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, const void *k,
                                                const void *v, void *out, void *cuda_stream)
 {
-    if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
-        return LOLA_ERR_INVALID_ARG;
+    if (!st) return LOLA_ERR_INVALID_ARG;
     const Dims &dm = st->dm;
-    const size_t phiq_bytes = align_up((size_t)dm.B * dm.Hq * dm.D * elem_bytes(dm));
     const size_t part_bytes = align_up((size_t)dm.ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
-    if (phiq_bytes + part_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
+    if (part_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
     void *base = nullptr;
     const lola_status sr = static_scratch_address(&base);
     if (sr != LOLA_OK) return sr;
-    // Every entry of both regions is written before it is read within one
-    // call, so nothing has to start at zero.
-    lola::DevState Sx = st->S;
-    Sx.phiQd = base;
-    Sx.part = (float *)((char *)base + phiq_bytes);
-
-    cudaStream_t stream = (cudaStream_t)cuda_stream;
-    const long long pos = st->pos;
-    {
-        PhaseScope ps(st, PH_APPEND, stream);
-        lola::launch_decode_append(dm, st->S, k, v, pos, stream);
-        counted(1);
-    }
-    if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
-    if (pos == st->interval_end) {
-        PhaseScope ps(st, PH_UPDATE, stream);
-        lola::launch_phi_kv(dm, st->S, nullptr, 0, 0, dm.lam + dm.R, 0, st->S.phiV, st->nS, stream);
-        lola::ChainArgs ca{};
-        ca.mode = 1;
-        ca.pos0 = pos;
-        ca.n_int = 1;
-        ca.ilen = dm.Cdec;
-        ca.nS0 = st->nS;
-        ca.pend_lo = st->pend_lo;
-        ca.pend_n = st->pend_n;
-        ca.iglob0 = st->n_int;
-        ca.phi = st->S.phiV;
-        ca.nvrows = dm.lam + dm.R;
-        ca.sel_log = st->sel_log;
-        ca.sel_cap = st->sel_cap;
-        ca.ovr = st->ovr;
-        ca.ovr_n = st->ovr_n;
-        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
-        else lola::launch_chain(dm, st->S, nullptr, ca, stream);
-        counted(2);
-        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
-        advance_interval(st, pos, dm.Cdec);
-        st->t0_open = pos;
-        st->interval_end = pos + dm.Cdec;
-    }
-    lola::DecodeArgs da{};
-    da.pos = pos;
-    da.t0 = st->t0_open;
-    da.nS = st->nS;
-    da.L_lo = st->pend_lo;
-    da.L_hi = st->pend_lo + st->pend_n;
-    da.q = q;
-    da.k = k;
-    da.v = v;
-    da.out = out;
-    {
-        PhaseScope ps(st, PH_DECODE, stream);
-        lola::launch_decode_attn(dm, Sx, da, stream);
-        counted(3);
-    }
-    st->pos = pos + 1;
-    return check_launch();
+    // Every partial is written before it is read within one call, so nothing
+    // has to start at zero.
+    return decode_step_impl(st, q, k, v, out, cuda_stream, (float *)base);
 }

@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(NW * 32)
 {
     const int d = dm.d, D = dm.D, eta = dm.eta, lam = dm.lam;
     const int qsplit = (dm.C + QR - 1) / QR;
-    const int ci = blockIdx.x / qsplit, qp = blockIdx.x % qsplit;
+    const int ci = a.ci0 + blockIdx.x / qsplit, qp = blockIdx.x % qsplit;
     const int hq = blockIdx.y, b = blockIdx.z;
     const int hk = hq / dm.g, st = b * dm.Hkv + hk;
     const long long t0 = a.pos0 + (long long)ci * dm.C, t1 = t0 + dm.C;

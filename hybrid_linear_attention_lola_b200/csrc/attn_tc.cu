@@ -41,7 +41,7 @@ struct TileMeta {
 struct AGeo {
     int d, D, FP, NB, NBa;
     uint32_t ncols;
-    size_t off_phq, off_big, off_K[2], off_V[2], off_phk, off_P, off_meta, off_red, total;
+    size_t off_phq, off_big, off_K[2], off_V[2], off_phk, off_P, off_wt, off_meta, off_red, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -71,7 +71,10 @@ __host__ __device__ inline AGeo make_ageo(const Dims &dm)
     g.off_P = al(g.off_phk + (size_t)KT * g.FP * 2, 1024);
     const size_t tiles_end = g.off_P + (size_t)128 * KT * 2;
     const size_t img_end = g.off_big + (size_t)g.FP * (g.d + 16) * 2;
-    o = tiles_end > img_end ? tiles_end : img_end;
+    // W^T (K-major, Dh rows) behind the snapshot image: both are dead once the key tiles load
+    g.off_wt = al(img_end, 1024);
+    const size_t wt_end = g.off_wt + (size_t)(g.D / 2) * dp * 2;
+    o = tiles_end > wt_end ? tiles_end : wt_end;
     g.off_meta = al(o, 16);
     g.off_red = al(g.off_meta + 2 * sizeof(TileMeta), 16);
     g.total = g.off_red + 128 * 4 + 1024;
@@ -100,7 +103,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const AGeo g = make_ageo(dm);
     const int d = g.d, D = g.D, FP = g.FP, eta = dm.eta, lam = dm.lam, gq = dm.g;
     const int tiles_per_int = (dm.C * gq + 127) / 128;
-    const int ci = blockIdx.x / tiles_per_int, mt = blockIdx.x % tiles_per_int;
+    const int ci = a.ci0 + blockIdx.x / tiles_per_int, mt = blockIdx.x % tiles_per_int;
     const int st = blockIdx.y;
     const int b = st / dm.Hkv, hk = st % dm.Hkv;
     const long long t0 = a.pos0 + (long long)ci * dm.C, t1 = t0 + dm.C;
@@ -136,9 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
     uint32_t phase = 0;
 
-    // ---- stage Q, phi(Q) and the snapshot image
+    // ---- stage Q, W^T and the snapshot image
     const bf16 *q = (const bf16 *)a.q;
-    const bf16 *phiQ = (const bf16 *)P.phiQ;
+    const int Dh = D / 2;
+    uint8_t *sWt = base + g.off_wt;
     const size_t qrow0 = ((size_t)b * a.n_call + (size_t)(t0 - a.pos0)) * dm.Hq + (size_t)hk * gq;
     for (int e = tid; e < (128 << lgd); e += kThreads) {
         const int rr = e >> lgd, kc = e & ((1 << lgd) - 1);
@@ -151,15 +155,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             *(uint4 *)dst = make_uint4(0, 0, 0, 0);
         }
     }
-    for (int e = tid; e < (128 << lgf); e += kThreads) {
-        const int rr = e >> lgf, kc = e & ((1 << lgf) - 1);
-        const int gr = mt * 128 + rr;
-        uint8_t *dst = sPhq + umma::kmajor_offset(rr, kc * 8, 128);
-        if (gr < rows_total && kc * 8 < D) {
-            const size_t row = qrow0 + (size_t)(gr / gq) * dm.Hq + gr % gq;
-            umma::cp_async16(dst, phiQ + row * D + kc * 8);
-        } else {
-            *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+    {
+        const bf16 *Wt = (const bf16 *)S.Wt;
+        for (int e = tid; e < (Dh << lgd); e += kThreads) {
+            const int rr = e >> lgd, kc = e & ((1 << lgd) - 1);
+            umma::cp_async16(sWt + umma::kmajor_offset(rr, kc * 8, Dh), Wt + (size_t)rr * d + kc * 8);
         }
     }
     {
@@ -174,9 +174,69 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     bool ok = true;
+    // ---- 0. phi(Q) = [softmax(Q W), softmax(-Q W)]: Z = Q W on the tensor cores (into the
+    //         score columns), then each row's two softmaxes; half 0 of the CTA writes the
+    //         first Dh features, half 1 the last Dh, as bf16 into the K-major phi(Q) tile
+    if (tid == 0) {
+        umma::fence_after_sync();
+        const uint32_t q0 = umma::smem_u32(sQ), w0 = umma::smem_u32(sWt);
+        const uint32_t id_z = umma::idesc_bf16(128, Dh, false, false);
+        for (int ks = 0; ks < d / 16; ++ks)
+            umma::mma_ss(tS, umma::kmajor_desc(q0, ks, 128), umma::kmajor_desc(w0, ks, Dh), id_z,
+                         ks > 0 ? 1u : 0u);
+        umma::mma_commit(&mbar);
+    }
+    ok = wait_mbar(&mbar, phase, &okflag, S.err);
+    if (ok) {
+        float zmax = -INFINITY, zmin = INFINITY;
+        for (int c0 = 0; c0 < Dh; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tS + lane_off + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+                zmax = fmaxf(zmax, v[j]);
+                zmin = fminf(zmin, v[j]);
+            }
+        }
+        float ssum = 0.f;
+        for (int c0 = 0; c0 < Dh; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tS + lane_off + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; ++j) ssum += half ? __expf(zmin - v[j]) : __expf(v[j] - zmax);
+        }
+        const float rs_ = 1.f / ssum;
+        for (int c0 = 0; c0 < Dh; c0 += 16) {
+            float v[16];
+            umma::tmem_ld16(tS + lane_off + (uint32_t)c0, v);
+            umma::tmem_wait_ld();
+#pragma unroll
+            for (int j = 0; j < 16; j += 8) {
+                float f[8];
+#pragma unroll
+                for (int t = 0; t < 8; ++t)
+                    f[t] = (half ? __expf(zmin - v[j + t]) : __expf(v[j + t] - zmax)) * rs_;
+                uint4 pk;
+                pk.x = umma::pack_bf16x2(f[0], f[1]);
+                pk.y = umma::pack_bf16x2(f[2], f[3]);
+                pk.z = umma::pack_bf16x2(f[4], f[5]);
+                pk.w = umma::pack_bf16x2(f[6], f[7]);
+                *(uint4 *)(sPhq + umma::kmajor_offset(r, half * Dh + c0 + j, 128)) = pk;
+            }
+        }
+        if (half == 1)
+            for (int c = D; c < FP; c += 8)
+                *(uint4 *)(sPhq + umma::kmajor_offset(r, c, 128)) = make_uint4(0, 0, 0, 0);
+    }
+    umma::fence_async_smem();
+    umma::fence_before_sync();
+    __syncthreads();
+
     // ---- 1. O = phi(Q) [H'|s']: the snapshot holds H' as an N-contiguous [FP][d]
     //         operand followed by s' as row 0 of a K-major 16 x FP operand
-    if (tid == 0) {
+    if (tid == 0 && ok) {
         umma::fence_after_sync();
         const uint32_t a0 = umma::smem_u32(sPhq), bh = umma::smem_u32(sImg);
         const uint32_t bs = bh + (uint32_t)(FP * d * 2);
@@ -189,7 +249,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         umma::mma_commit(&mbar);
     }
-    ok = wait_mbar(&mbar, phase, &okflag, S.err);
+    if (ok) ok = wait_mbar(&mbar, phase, &okflag, S.err);
 
     const size_t lb = (size_t)st * dm.mmax + ci;
     const int nK = P.logCount[lb];

@@ -393,8 +393,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     int nS = a.nS0;
     for (int i = tid; i < lam; i += kThreads) {
-        slotTok[i] = i < nS ? S.idxS[(size_t)st * lam + i] : -1;
-        slotVrow[i] = i;
+        if (a.mode == 0 && a.cont) {
+            slotTok[i] = P.slotTok[(size_t)st * lam + i];
+            slotVrow[i] = P.slotVrow[(size_t)st * lam + i];
+        } else {
+            slotTok[i] = i < nS ? S.idxS[(size_t)st * lam + i] : -1;
+            slotVrow[i] = i;
+        }
     }
     for (int i = tid; i < Lmax; i += kThreads) lf[i] = i < a.pend_n ? S.pend[(size_t)st * Lmax + i] : 0;
     long long pend_lo = a.pend_lo;
@@ -556,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             refresh_image(c);
         }
         if (a.mode == 0 && P.snapImg != nullptr) {
-            uint4 *dst = (uint4 *)((uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * g.NB * g.FP * 2);
+            uint4 *dst = (uint4 *)((uint8_t *)P.snapImg + ((size_t)st * dm.mmax + a.ci0 + ci) * g.NB * g.FP * 2);
             const uint4 *srcp = (const uint4 *)c.Bimg;
             const int n16 = g.NB * g.FP * 2 / 16;
             for (int e = tid; e < n16; e += kThreads) dst[e] = srcp[e];
@@ -564,8 +569,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (a.mode == 0 && a.snap_f32) {
             // fp32 (H', s') for the SIMT attention kernel
             const int q = warp & 3;
-            float *sh = P.snapH + ((size_t)st * dm.mmax + ci) * D * d;
-            float *ss = P.snapS + ((size_t)st * dm.mmax + ci) * D;
+            float *sh = P.snapH + ((size_t)st * dm.mmax + a.ci0 + ci) * D * d;
+            float *ss = P.snapS + ((size_t)st * dm.mmax + a.ci0 + ci) * D;
             for (int bk = warp >> 2; bk < g.nblk; bk += kThreads / 128) {
                 const int f = bk * 128 + q * 32 + lane;
                 for (int c0 = 0; c0 < g.NB; c0 += 16) {
@@ -615,7 +620,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
         if (a.mode == 0) {
-            const size_t lb = (size_t)st * dm.mmax + ci;
+            const size_t lb = (size_t)st * dm.mmax + a.ci0 + ci;
             for (int i = tid; i < nK; i += kThreads) {
                 P.logTok[lb * lam + i] = slotTok[i];
                 P.logVrow[lb * lam + i] = slotVrow[i];

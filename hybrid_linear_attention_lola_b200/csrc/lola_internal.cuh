@@ -23,8 +23,10 @@ enum : int { ERR_BOUNDS = 1, ERR_TIMEOUT = 2 };
 struct Dims {
     int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
     int Nmax, mmax;   // prefill scratch capacity: tokens per call, intervals per call
-    int nsplit;       // decode key splits (CTAs) per stream
-    int dec_nch;      // decode: 32-key chunks per warp (4 warps per CTA)
+    int nsplit;       // decode: CTAs per stream
+    int dec_nw;       // decode: warps per CTA
+    int dec_nst;      // decode: staging buffers per warp
+    int dec_sb;       // decode: bytes per staging buffer
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
     float eps;
@@ -39,10 +41,10 @@ struct DevState {
     void *KR, *VR;     // [ns][R][d]   window ring (slot = token mod R)
     uint8_t *pend;     // [ns][Lmax]   1 = leaving pair of the last interval that is folded
     float *W;          // [d][Dh]      feature-map matrix, fp32 copy
+    void *Wt;          // [Dh][d]      W transposed, in the input dtype (tensor-core operand)
     int *err;          // [4]          device error words
     // decode scratch (phi buffers hold the input dtype)
     void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
-    void *phiQd;       // [B][Hq][D]
     float *part;       // [ns][nsplit][g][2d + 4] split partials
     int *dec_cnt;      // [ns] finished decode CTAs per stream (reset by the last one)
 };
@@ -120,6 +122,61 @@ __device__ __forceinline__ float warp_min(float x)
     return x;
 }
 
+// phi(x) = [softmax(x W), softmax(-x W)] of one row, computed by one warp. W (fp32, [d][Dh]) sits in shared memory; lane l owns
+// features l, l + 32, ... The row max / min shift is exact in real arithmetic.
+template <typename T>
+__device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const float *__restrict__ Ws,
+                                             float *__restrict__ xs, int d, int Dh,
+                                             T *__restrict__ out)
+{
+    const int lane = threadIdx.x & 31;
+    for (int a = lane; a < d; a += 32) xs[a] = to_f<T>(x[a]);
+    __syncwarp();
+    float z[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) z[u] = 0.f;
+    for (int a = 0; a < d; ++a) {
+        const float xa = xs[a];
+        const float *wr = Ws + (size_t)a * Dh;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int i = lane + 32 * u;
+            if (i < Dh) z[u] = fmaf(xa, wr[i], z[u]);
+        }
+    }
+    float zmax = -INFINITY, zmin = INFINITY;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        if (lane + 32 * u < Dh) {
+            zmax = fmaxf(zmax, z[u]);
+            zmin = fminf(zmin, z[u]);
+        }
+    }
+    zmax = warp_max(zmax);
+    zmin = warp_min(zmin);
+    float ep[4], en[4], sp = 0.f, sn = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const bool ok = lane + 32 * u < Dh;
+        ep[u] = ok ? __expf(z[u] - zmax) : 0.f;
+        en[u] = ok ? __expf(zmin - z[u]) : 0.f;
+        sp += ep[u];
+        sn += en[u];
+    }
+    sp = warp_sum(sp);
+    sn = warp_sum(sn);
+    const float rp = 1.f / sp, rn = 1.f / sn;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int i = lane + 32 * u;
+        if (i < Dh) {
+            out[i] = from_f<T>(ep[u] * rp);
+            out[Dh + i] = from_f<T>(en[u] * rn);
+        }
+    }
+    __syncwarp();
+}
+
 __device__ __forceinline__ void raise_error(int *err, int code)
 {
     if (err) atomicOr(err, code);
@@ -132,6 +189,12 @@ void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long
                    cudaStream_t stream);
 void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows, void *phi_out,
                   cudaStream_t stream);
+// bfloat16 tensor-core versions of the two above
+void launch_phi_kv_tc(const Dims &dm, const DevState &S, const void *kin, long long call_start, int n,
+                      int nvrows, void *phi_out, int nS, cudaStream_t stream);
+void launch_phi_q_tc(const Dims &dm, const DevState &S, const void *q, long long rows, void *phi_out,
+                     cudaStream_t stream);
+size_t phi_tc_smem_bytes(const Dims &dm);
 
 struct ChainArgs {
     int mode;               // 0 = prefill call, 1 = decode interval
@@ -151,6 +214,9 @@ struct ChainArgs {
     const int32_t *ovr;     // test hook, may be null
     long long ovr_n;
     int snap_f32;           // prefill: also write fp32 (H', s') snapshots
+    int ci0;                // prefill: index of the first interval within the call
+    int cont;               // prefill: the call's earlier intervals ran in an earlier launch
+                            // (slot contents come from the scratch, not the state)
 };
 void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
                      cudaStream_t stream);
@@ -162,7 +228,8 @@ void launch_chain(const Dims &dm, const DevState &S, const PrefillScratch *P, co
 
 struct AttnArgs {
     long long pos0;         // first token of the call
-    int m;                  // chunks in the call
+    int m;                  // chunks in this launch
+    int ci0;                // index of this launch's first chunk within the call
     int n_call;
     const void *q, *kin, *vin;
     void *out;
@@ -184,9 +251,16 @@ struct DecodeArgs {
     const void *q, *k, *v;
     void *out;
 };
+// Decode launch shape: splits per stream, warps per CTA, staging buffers and
+// their size (fills dm.nsplit, dec_nw, dec_nst, dec_sb); returns false if no
+// shape fits in shared memory.
+bool decode_plan(Dims *dm);
+size_t decode_smem_bytes(const Dims &dm);
+// with_phi: also compute phi(k) of the appended token into the phi rows.
 void launch_decode_append(const Dims &dm, const DevState &S, const void *k, const void *v,
-                          long long pos, cudaStream_t stream);
-void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a,
+                          long long pos, int with_phi, cudaStream_t stream);
+// do_append: the kernel also appends the step's k, v (and phi(k)) to the window ring.
+void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, int do_append,
                         cudaStream_t stream);
 void launch_get_indices(const Dims &dm, const DevState &S, int nS, int32_t *idx, int32_t *cnt,
                         cudaStream_t stream);

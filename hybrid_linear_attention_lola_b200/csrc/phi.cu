@@ -6,61 +6,6 @@
 
 namespace lola {
 
-// One warp maps one row. W (fp32, [d][Dh]) sits in shared memory; lane l owns
-// features l, l + 32, ... The row max / min shift is exact in real arithmetic.
-template <typename T>
-__device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const float *__restrict__ Ws,
-                                             float *__restrict__ xs, int d, int Dh,
-                                             T *__restrict__ out)
-{
-    const int lane = threadIdx.x & 31;
-    for (int a = lane; a < d; a += 32) xs[a] = to_f<T>(x[a]);
-    __syncwarp();
-    float z[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) z[u] = 0.f;
-    for (int a = 0; a < d; ++a) {
-        const float xa = xs[a];
-        const float *wr = Ws + (size_t)a * Dh;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int i = lane + 32 * u;
-            if (i < Dh) z[u] = fmaf(xa, wr[i], z[u]);
-        }
-    }
-    float zmax = -INFINITY, zmin = INFINITY;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        if (lane + 32 * u < Dh) {
-            zmax = fmaxf(zmax, z[u]);
-            zmin = fminf(zmin, z[u]);
-        }
-    }
-    zmax = warp_max(zmax);
-    zmin = warp_min(zmin);
-    float ep[4], en[4], sp = 0.f, sn = 0.f;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const bool ok = lane + 32 * u < Dh;
-        ep[u] = ok ? __expf(z[u] - zmax) : 0.f;
-        en[u] = ok ? __expf(zmin - z[u]) : 0.f;
-        sp += ep[u];
-        sn += en[u];
-    }
-    sp = warp_sum(sp);
-    sn = warp_sum(sn);
-    const float rp = 1.f / sp, rn = 1.f / sn;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-        const int i = lane + 32 * u;
-        if (i < Dh) {
-            out[i] = from_f<T>(ep[u] * rp);
-            out[Dh + i] = from_f<T>(en[u] * rn);
-        }
-    }
-    __syncwarp();
-}
-
 template <typename T>
 __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, const float *__restrict__ W,
                                                      int nS, int n, int nvrows,
@@ -168,8 +113,14 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
         KR[e] = from_f<T>(0.f);
         VR[e] = from_f<T>(0.f);
     }
-    if (W != nullptr)
-        for (long long e = tid; e < (long long)dm.d * dm.Dh; e += stride) S.W[e] = to_f<T>(W[e]);
+    if (W != nullptr) {
+        T *Wt = (T *)S.Wt;
+        for (long long e = tid; e < (long long)dm.d * dm.Dh; e += stride) {
+            S.W[e] = to_f<T>(W[e]);
+            const long long a = e / dm.Dh, i = e - a * dm.Dh;
+            Wt[i * dm.d + a] = W[e];
+        }
+    }
     if (tid < 4) S.err[tid] = 0;
     for (long long e = tid; e < dm.ns; e += stride) S.dec_cnt[e] = 0;
 }

@@ -1,8 +1,8 @@
 // Thin helpers around the sm_100a 5th-generation tensor-core instructions
 // (tcgen05.*): shared-memory matrix descriptors for 128-byte-swizzled bf16
 // operands, the instruction descriptor for bf16 x bf16 -> fp32, TMEM
-// allocation, MMA issue/commit, TMEM loads, and mbarrier waits that give up
-// after a bounded number of polls.
+// allocation, MMA issue/commit, TMEM loads, bulk (TMA) global -> shared
+// copies, and mbarrier waits that give up after a bounded time.
 //
 // Operand layouts (bf16, 128-byte swizzle; every tile base 1024-byte aligned):
 //  * K-major tile of R rows (R % 8 == 0) and K columns: atom column kb = k / 64
@@ -193,6 +193,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint6
         if (done) return true;
         if (globaltimer_ns() - start > limit_ns) return false;
     }
+}
+
+// Expects `bytes` more transaction bytes on the mbarrier and arrives once.
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(mbar)), "r"(bytes)
+                 : "memory");
+}
+
+// Bulk (TMA, non-tensor) global -> shared copy of `bytes` (a multiple of 16;
+// both addresses 16-byte aligned); completion is counted on the mbarrier.
+__device__ __forceinline__ void bulk_g2s(void *smem_dst, const void *gmem_src, uint32_t bytes, uint64_t *mbar)
+{
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        :
+        : "r"(smem_u32(smem_dst)), "l"(gmem_src), "r"(bytes), "r"(smem_u32(mbar))
+        : "memory");
 }
 
 // Two fp32 -> one register holding two bf16 (round to nearest even); lo in bits 0..15.

@@ -112,13 +112,14 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
  * all device memory and passes it only inputs, outputs and persistent state,
  * or code running while a CUDA graph is being captured, where cudaMalloc is
  * not allowed. The paper has no counterpart to this call; it only changes
- * where temporaries live. The per-step scratch of the decode attention (query
- * features and split partials) is taken from an 8 MiB array inside the
- * library (a static device array: every GPU that loads the library holds it
- * until the process exits) instead of the workspace. The call allocates
- * nothing. Configs whose decode scratch,
- * B*n_q_heads*feat_dim*4 + streams*splits*(n_q_heads/n_kv_heads)*(2*head_dim+4)*4
- * bytes (each part rounded up to 256), exceed 8 MiB get LOLA_ERR_WORKSPACE.
+ * where temporaries live. The per-step scratch of the decode attention (the
+ * partial sums of the CTAs that share a stream) is taken from an 8 MiB array
+ * inside the library (a static device array: every GPU that loads the library
+ * holds it until the process exits) instead of the workspace. The call
+ * allocates nothing. Configs whose decode scratch,
+ * streams*splits*(n_q_heads/n_kv_heads)*(2*head_dim+4)*4 bytes (rounded up to
+ * 256; splits = CTAs per stream, chosen by the library), exceed 8 MiB get
+ * LOLA_ERR_WORKSPACE.
  * The first call on a device looks up the array's device address (once per
  * device, with the device current); make that first call before any stream
  * capture. All calls share the one array and leave their contents in it, so
