@@ -170,6 +170,7 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.Wt = take((size_t)dm.d * dm.Dh * e);
     s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
+    s.phiQd = (float *)take(dm.dtype == LOLA_BF16 ? (size_t)dm.B * dm.Hq * dm.D * 4 : 0);
     s.dec_cnt = (int *)take(ns * 4);
     lola::PrefillScratch p{};
     const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
@@ -231,7 +232,7 @@ void advance_interval(lola_state *st, long long t0, int len)
 
 // One decode step. `part` receives the split partials of the decode attention.
 lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const void *v, void *out,
-                             void *cuda_stream, float *part)
+                             void *cuda_stream, float *part, float *phiq)
 {
     if (!st || !q || !k || !v || !out) return LOLA_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
@@ -298,6 +299,7 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
     da.out = out;
     lola::DevState Sx = st->S;
     Sx.part = part;
+    Sx.phiQd = phiq;
     {
         PhaseScope ps(st, PH_DECODE, stream);
         lola::launch_decode_attn(dm, Sx, da, do_append, stream);
@@ -532,7 +534,7 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
                              void *out, void *cuda_stream)
 {
     if (!st) return LOLA_ERR_INVALID_ARG;
-    return decode_step_impl(st, q, k, v, out, cuda_stream, st->S.part);
+    return decode_step_impl(st, q, k, v, out, cuda_stream, st->S.part, st->S.phiQd);
 }
 
 lola_status lola_get_cache_indices(const lola_state *st, int32_t *dev_idx, int32_t *dev_count,
@@ -625,8 +627,9 @@ lola_status lola_free_state(lola_state *st)
 // ---------------------------------------------------------------- decode step, library-owned scratch
 //
 // lola_decode_step_static runs the same decode step as lola_decode_step, but
-// the per-step temporaries of the split decode attention (the per-split
-// partial sums of a stream's CTAs) live in the fixed device array below
+// the per-step temporaries of the decode attention (the partial sums of the
+// warps or CTAs that share a stream, and the query features) live in the
+// fixed device array below
 // instead of the caller's workspace. It exists for callers that cannot obtain
 // device memory on demand: a host framework that owns all device memory and
 // hands a plugin only its inputs, outputs and persistent state, or code that
@@ -671,11 +674,13 @@ extern "C" lola_status lola_decode_step_static(lola_state *st, const void *q, co
     if (!st) return LOLA_ERR_INVALID_ARG;
     const Dims &dm = st->dm;
     const size_t part_bytes = align_up((size_t)dm.ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
-    if (part_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
+    const size_t phiq_bytes = dm.dtype == LOLA_BF16 ? align_up((size_t)dm.B * dm.Hq * dm.D * 4) : 0;
+    if (part_bytes + phiq_bytes > kStaticScratchBytes) return LOLA_ERR_WORKSPACE;
     void *base = nullptr;
     const lola_status sr = static_scratch_address(&base);
     if (sr != LOLA_OK) return sr;
-    // Every partial is written before it is read within one call, so nothing
-    // has to start at zero.
-    return decode_step_impl(st, q, k, v, out, cuda_stream, (float *)base);
+    // Every partial and query feature is written before it is read within one
+    // call, so nothing has to start at zero.
+    return decode_step_impl(st, q, k, v, out, cuda_stream, (float *)base,
+                            phiq_bytes ? (float *)((char *)base + part_bytes) : nullptr);
 }

@@ -29,17 +29,17 @@ constexpr int kFoldTok = 64;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 
 struct Geo {
-    int D, d, NB, NBa, FP, nblk, lam, Lmax, QC, vstride;
+    int D, d, NB, NBa, FP, nblk, lam, Lmax, QC, nbuf;
     uint32_t ncols;
-    size_t off_Bs, off_ones, off_X, off_Vt, off_B1, off_keys, off_rank, off_lst, off_slotTok,
+    size_t off_Bs, off_ones, off_X, off_X1, off_B1, off_part, off_keys, off_rank, off_lst, off_slotTok,
         off_slotVrow, off_free, off_keep, off_flag, off_lf, off_hist, off_scal, total;
 };
 
 __host__ __device__ inline size_t al(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 // Shared memory: [H image, N-contiguous FP x d][s image, K-major 16 x FP][ones, K-major 16 x 64]
-// [X: SRE phi tile (K-major 128 x FP) + padded value rows | fold A blocks + value rows][ints]
-__host__ __device__ inline Geo make_geo(const Dims &dm)
+// [X: nbuf SRE phi tiles (K-major 128 x FP) | fold A blocks + value rows][partial sums][ints]
+__host__ __device__ inline Geo make_geo_n(const Dims &dm, int nbuf)
 {
     Geo g{};
     g.D = dm.D;
@@ -51,7 +51,7 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.lam = dm.lam;
     g.Lmax = dm.Lmax;
     g.QC = dm.lam + dm.Lmax;
-    g.vstride = (dm.d + 8) * 2;     // bytes per staged value row (padded against bank conflicts)
+    g.nbuf = nbuf;
     const uint32_t need = (uint32_t)((g.nblk + 1) * g.NBa);
     g.ncols = need <= 32 ? 32 : need <= 64 ? 64 : need <= 128 ? 128 : need <= 256 ? 256 : 512;
     size_t o = (size_t)g.FP * g.d * 2;                        // H image
@@ -60,11 +60,14 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.off_ones = al(o, 1024);
     o = g.off_ones + 16 * 64 * 2;
     g.off_X = al(o, 1024);
-    const size_t xs = (size_t)128 * g.FP * 2 + (size_t)128 * g.vstride;
+    const size_t tile = (size_t)128 * g.FP * 2;
+    g.off_X1 = g.off_X + tile;
+    const size_t xs = (size_t)nbuf * tile;
     const size_t xf = (size_t)g.nblk * 64 * 128 * 2 + (size_t)64 * g.d * 2;
-    g.off_Vt = g.off_X + (size_t)128 * g.FP * 2;
     g.off_B1 = g.off_X + (size_t)g.nblk * 64 * 128 * 2;
     o = g.off_X + (xs > xf ? xs : xf);
+    g.off_part = al(o, 16);
+    o = g.off_part + 128 * 4;
     g.off_keys = al(o, 16);
     o = g.off_keys + (size_t)g.QC * 4;
     g.off_rank = o;
@@ -90,6 +93,13 @@ __host__ __device__ inline Geo make_geo(const Dims &dm)
     g.total = o + 1024;  // alignment slack for the 1024-byte aligned base
     if (g.ncols == 512 && g.total < 116 * 1024) g.total = 116 * 1024;  // one CTA per SM
     return g;
+}
+
+// Two SRE tile buffers (the next tile loads while this one is scored) when they fit.
+__host__ __device__ inline Geo make_geo(const Dims &dm)
+{
+    const Geo g2 = make_geo_n(dm, 2);
+    return g2.total <= 227 * 1024 - 64 ? g2 : make_geo_n(dm, 1);
 }
 
 template <typename F>
@@ -232,6 +242,9 @@ __device__ bool wait_mma(Ctx &c)
 __device__ void refresh_image(Ctx &c)
 {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, q = warp & 3;
+    // the last snapshot store must have read the image before it is overwritten
+    if (threadIdx.x == 0) umma::bulk_wait_read();
+    __syncthreads();
     for (int bk = warp >> 2; bk < c.g.nblk; bk += kThreads / 128) {
         const int f = bk * 128 + q * 32 + lane;
         const uint32_t row = tH(c, bk) + ((uint32_t)(q * 32) << 16);
@@ -409,7 +422,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const uint32_t id_sh = umma::idesc_bf16(128, d, false, true);
     const uint32_t id_ss = umma::idesc_bf16(128, 16, false, false);
-    uint8_t *phiT = c.X, *Vt = base + g.off_Vt;
     for (int ci = 0; ci < a.n_int && ok; ++ci) {
         const long long t0 = a.pos0 + (long long)ci * a.ilen;
         const long long t1 = t0 + a.ilen;
@@ -437,28 +449,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cnd = tid; cnd < nQ; cnd += kThreads)
             cvrow[cnd] = cnd < nS ? slotVrow[cnd] : src.tok2vrow(Llo + (cnd - nS));
         __syncthreads();
-        const int lgc = __ffs(g.FP >> 3) - 1, lgv = __ffs(d >> 3) - 1;   // chunks per row (powers of two)
-        for (int m0 = 0; m0 < nQ && ok; m0 += 128) {
-            const int nr = min(128, nQ - m0);
-            // candidates' phi rows (K-major A operand) and value rows (padded, for the epilogue)
+        const int lgc = __ffs(g.FP >> 3) - 1;   // 16-byte chunks per phi row (power of two)
+        const int ntile = (nQ + 127) / 128;
+        // phi rows of tile t (K-major A operand) into buffer t % nbuf; one cp.async group
+        auto load_tile = [&](int t) {
+            uint8_t *dstT = base + (t % g.nbuf ? g.off_X1 : g.off_X);
+            const int m0 = t * 128, nr = min(128, nQ - m0);
             for (int e = tid; e < (nr << lgc); e += kThreads) {
                 const int r = e >> lgc, kc = e & ((1 << lgc) - 1);
-                uint8_t *dst = phiT + umma::kmajor_offset(r, kc * 8, 128);
+                uint8_t *dst = dstT + umma::kmajor_offset(r, kc * 8, 128);
                 if (kc * 8 < D) umma::cp_async16(dst, phi_st + (size_t)cvrow[m0 + r] * D + kc * 8);
                 else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
             }
-            for (int e = tid; e < (nr << lgv); e += kThreads) {
-                const int r = e >> lgv, cc = e & ((1 << lgv) - 1);
-                umma::cp_async16(Vt + (size_t)r * g.vstride + cc * 16, src.vrow(st, cvrow[m0 + r]) + cc * 8);
-            }
             umma::cp_async_commit();
-            umma::cp_async_wait_all();
+        };
+        if (ntile > 0) load_tile(0);
+        if (g.nbuf == 2 && ntile > 1) load_tile(1);
+        const int q = warp & 3, half = warp >> 2;
+        const int r = q * 32 + lane;                      // this thread's row of the tile
+        const int hd = d >> 1;                            // value dims per thread
+        for (int t = 0; t < ntile && ok; ++t) {
+            const int m0 = t * 128, nr = min(128, nQ - m0);
+            if (g.nbuf == 2 && t + 1 < ntile) umma::cp_async_wait_1();
+            else umma::cp_async_wait_all();
             umma::fence_async_smem();
             umma::fence_before_sync();
             __syncthreads();
             if (tid == 0) {
                 umma::fence_after_sync();
-                const uint32_t a0 = umma::smem_u32(phiT), bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
+                const uint32_t a0 = umma::smem_u32(base + (t % g.nbuf ? g.off_X1 : g.off_X));
+                const uint32_t bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
                 for (int ks = 0; ks < g.FP / 16; ++ks) {
                     const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
                     umma::mma_ss(tS(c), ad, umma::mnmajor_desc(bh, ks, d), id_sh, ks > 0 ? 1u : 0u);
@@ -466,37 +486,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 umma::mma_commit(c.mbar);
             }
+            // this thread's half of its candidate's value row, fetched while the MMA runs
+            uint4 vr4[8];
+            if (r < nr) {
+                const uint4 *vsrc = (const uint4 *)(src.vrow(st, cvrow[m0 + r]) + half * hd);
+#pragma unroll
+                for (int i = 0; i < 8; ++i)
+                    if (i * 8 < hd) vr4[i] = vsrc[i];
+            }
             if (!(ok = wait_mma(c))) break;
+            if (g.nbuf == 1 && t + 1 < ntile) load_tile(t + 1);         // the tile buffer is free
+            if (g.nbuf == 2 && t + 2 < ntile) load_tile(t + 2);
             {
-                // 8 warps: warp w reads lanes 32*(w%4).., value columns half (w/4) of d
-                const int q = warp & 3, half = warp >> 2;
-                const int r = q * 32 + lane;
                 const uint32_t rowaddr = tS(c) + ((uint32_t)(q * 32) << 16);
                 float v[16];
                 umma::tmem_ld16(rowaddr + (uint32_t)d, v);
                 umma::tmem_wait_ld();
                 const float den = v[0] + dm.eps;
                 const float rden = den != 0.f ? 1.f / den : 0.f;
-                const uint8_t *vrow = Vt + (size_t)r * g.vstride;
-                const int cbeg = half * (d >> 1), cend = cbeg + (d >> 1);
                 float err = 0.f;
-                for (int c0 = cbeg; c0 < cend; c0 += 16) {
-                    umma::tmem_ld16(rowaddr + (uint32_t)c0, v);
-                    umma::tmem_wait_ld();
-                    const uint4 r0 = *(const uint4 *)(vrow + c0 * 2);
-                    const uint4 r1 = *(const uint4 *)(vrow + c0 * 2 + 16);
-                    const bf16 *p0 = (const bf16 *)&r0;
-                    const bf16 *p1 = (const bf16 *)&r1;
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const float diff = v[i] * rden - __bfloat162float(i < 8 ? p0[i] : p1[i - 8]);
-                        err = fmaf(diff, diff, err);
+                for (int i2 = 0; i2 < 4; ++i2) {
+                    if (i2 * 16 < hd) {
+                        umma::tmem_ld16(rowaddr + (uint32_t)(half * hd + i2 * 16), v);
+                        umma::tmem_wait_ld();
+                        const bf16 *p0 = (const bf16 *)&vr4[2 * i2];
+                        const bf16 *p1 = (const bf16 *)&vr4[2 * i2 + 1];
+#pragma unroll
+                        for (int i = 0; i < 16; ++i) {
+                            const float diff = v[i] * rden - __bfloat162float(i < 8 ? p0[i] : p1[i - 8]);
+                            err = fmaf(diff, diff, err);
+                        }
                     }
                 }
-                float *part = (float *)(base + g.off_X);   // phi tile no longer needed: reuse for partial sums
+                float *part = (float *)(base + g.off_part);
                 if (half == 1) part[r] = err;
                 __syncthreads();
-                if (half == 0 && m0 + r < nQ) {
+                if (half == 0 && r < nr) {
                     err += part[r];
                     keys[m0 + r] = 0xFFFFFFFFu - __float_as_uint(fmaxf(err, 0.f));
                 }
@@ -560,11 +586,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = fold_tc(c, lst, nE, phi_st, src, st))) break;
             refresh_image(c);
         }
-        if (a.mode == 0 && P.snapImg != nullptr) {
-            uint4 *dst = (uint4 *)((uint8_t *)P.snapImg + ((size_t)st * dm.mmax + a.ci0 + ci) * g.NB * g.FP * 2);
-            const uint4 *srcp = (const uint4 *)c.Bimg;
-            const int n16 = g.NB * g.FP * 2 / 16;
-            for (int e = tid; e < n16; e += kThreads) dst[e] = srcp[e];
+        if (a.mode == 0 && P.snapImg != nullptr && tid == 0) {
+            // the image (written and proxy-fenced by refresh_image) goes out as one bulk store
+            uint8_t *dst = (uint8_t *)P.snapImg + ((size_t)st * dm.mmax + a.ci0 + ci) * g.NB * g.FP * 2;
+            umma::bulk_s2g(dst, c.Bimg, (uint32_t)(g.NB * g.FP * 2));
         }
         if (a.mode == 0 && a.snap_f32) {
             // fp32 (H', s') for the SIMT attention kernel
@@ -669,6 +694,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::mbar_wait(&mbar, c.phase ^ 1u, kWaitNs);  // let an MMA still in flight drain
         }
     }
+    if (tid == 0) umma::bulk_wait_all();
     umma::fence_before_sync();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(c.tm, g.ncols);

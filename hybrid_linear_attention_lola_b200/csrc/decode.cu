@@ -31,6 +31,7 @@ namespace {
 constexpr int kMaxG = 8;
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per staging-buffer wait
 constexpr int kSMs = 148;
+constexpr int kMinPer = 8;   // items per warp of the streaming kernel, at least
 
 // ---------------------------------------------------------------- shared memory plan
 
@@ -110,13 +111,13 @@ template <int VN> __device__ __forceinline__ int qidx(int x) { return qoff<VN>(x
 //   [0, nkc)            32 softmax keys: cache slots [0, nS), then window tokens [wlo, p]
 //   [nkc, nkc + nlc)    16 linear-band tokens of [jlo, lhi) (left the window this
 //                       interval; folded ones are linear, kept ones are skipped)
-//   [nkc + nlc, ni)     32 feature rows of the state (H, s)
+//   [nkc + nlc, ni)     hrows feature rows of the state (H, s)
 struct Items {
     long long jlo, wlo, lhi;
     int nsoft, nkc, nlc, ni;
 };
 
-__device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a)
+__device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a, int hrows)
 {
     Items it;
     const long long p = a.pos;
@@ -127,7 +128,7 @@ __device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a)
     it.nsoft = a.nS + (int)(p - it.wlo + 1);
     it.nkc = (it.nsoft + 31) / 32;
     it.nlc = (int)((it.lhi - it.jlo + 15) / 16);
-    it.ni = it.nkc + it.nlc + dm.D / 32;
+    it.ni = it.nkc + it.nlc + dm.D / hrows;
     return it;
 }
 
@@ -146,7 +147,7 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
     const int D = dm.D, Dh = dm.Dh, g = dm.g, lam = dm.lam, R = dm.R;
     const long long p = a.pos;
     const int nS = a.nS;
-    const Items IT = make_items(dm, a);
+    const Items IT = make_items(dm, a, 32);
     const int gw = split * nw + warp, wstride = dm.nsplit * nw;
     const int nmine = gw < IT.ni ? (IT.ni - gw + wstride - 1) / wstride : 0;
     const DecLayout L = dec_layout(dm);
@@ -627,6 +628,493 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
     if (tid == 0) S.dec_cnt[st] = 0;
 }
 
+
+// ---------------------------------------------------------------- bfloat16: warp-level MMA
+//
+// Same items and pipeline as above, staged with 16-byte cp.async into a
+// 128-byte XOR-swizzled row layout (conflict-free ldmatrix). For a chunk of 32
+// keys, S = Q K^T and O += P V run as mma.sync m16n8k16 (bf16 in, fp32
+// accumulate) with the group's heads as the M rows (padded to 16); the score
+// fragments become the P operand directly. Linear-band and state items use the
+// SIMT code of the kernel above.
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
+{
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+                 : "r"(addr));
+}
+// C[16x8] += A[16x16] B[16x8]; rows 8..15 of A are zero (a1 = a3 = 0)
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1)
+{
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a0), "r"(0u), "r"(a2), "r"(0u), "r"(b0), "r"(b1));
+}
+// 16-byte async copy; src_bytes = 0 writes zeros
+__device__ __forceinline__ void cpa16(uint32_t dst, const void *src, int src_bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void cpa_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cpa_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+__device__ __forceinline__ uint32_t pack2(float lo, float hi)
+{
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+// byte offset of 16-byte chunk c of row r in a [32 rows][CPR chunks] swizzled tile
+template <int CPR> __device__ __forceinline__ uint32_t swz(int r, int c)
+{
+    return (uint32_t)((c >> 3) * 32 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
+}
+
+// Step preparation (bfloat16 path): phi(q) of every query row into an fp32
+// scratch, and, when the step appends, the new pair into the window ring with
+// phi(k) of it in the phi rows. One warp per row; W (fp32) in shared memory.
+template <typename T>
+__global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, DecodeArgs a, int do_append)
+{
+    extern __shared__ float smp[];
+    const int d = dm.d, Dh = dm.Dh, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    float *Ws = smp;
+    float *xs = smp + d * Dh + warp * d;
+    {
+        // 16-byte copies, all in flight at once (d * Dh is a multiple of 4)
+        const float4 *w4 = (const float4 *)S.W;
+        float4 *s4 = (float4 *)Ws;
+        const int n4 = d * Dh / 4;
+#pragma unroll 4
+        for (int e = threadIdx.x; e < n4; e += blockDim.x) s4[e] = __ldg(w4 + e);
+    }
+    __syncthreads();
+    const int nq = dm.B * dm.Hq, nk = do_append ? dm.ns : 0;
+    const int slot = (int)(a.pos & (dm.R - 1));
+    for (int r = blockIdx.x * 8 + warp; r < nq + nk; r += gridDim.x * 8) {
+        if (r < nq) {
+            phi_row_warp<T, float>((const T *)a.q + (size_t)r * d, Ws, xs, d, Dh, S.phiQd + (size_t)r * dm.D);
+        } else {
+            const int st = r - nq;
+            const T *k = (const T *)a.k + (size_t)st * d, *v = (const T *)a.v + (size_t)st * d;
+            T *kr = (T *)S.KR + ((size_t)st * dm.R + slot) * d, *vr = (T *)S.VR + ((size_t)st * dm.R + slot) * d;
+            for (int c = lane; c < d; c += 32) {
+                kr[c] = k[c];
+                vr[c] = v[c];
+            }
+            phi_row_warp<T, T>(k, Ws, xs, d, Dh, (T *)S.phiV + ((size_t)st * (dm.lam + dm.R) + dm.lam + slot) * dm.D);
+        }
+    }
+}
+
+// Streaming decode (bfloat16 path). A persistent grid; the work items of all
+// streams form one list (stream-major, see make_items) and every warp takes a
+// contiguous range of it, flowing its items through its own ring of three
+// shared-memory buffers (16-byte cp.async, 128-byte XOR-swizzled key/value
+// rows). For a chunk of 32 keys, S = Q K^T and O += P V run as mma.sync
+// m16n8k16 (bf16 in, fp32 accumulate) with the group's heads as the M rows
+// (padded to 16); the score fragments become the P operand directly. Linear
+// band and state items run on the SIMT units. When a warp leaves a stream it
+// writes its partial (m, l, linear den, softmax num, linear num per head); the
+// warp that writes a stream's last partial merges them (a per-stream counter).
+template <int DPL, int G>
+__global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S, DecodeArgs a, int per, int wbytes)
+{
+    using T = __nv_bfloat16;
+    constexpr int d = 32 * DPL;
+    constexpr int E = 2;
+    constexpr int VN = 8;
+    constexpr int CPR = d / 8;                         // 16-byte chunks per key row
+    constexpr int KS_ = d / 16;                        // k-steps of Q K^T
+    constexpr int ND = d / 8;                          // n-tiles of P V (8 value dims each)
+    constexpr int HR = 16;                             // state rows per item
+    constexpr int NST = 3;                             // staging buffers per warp
+    constexpr int RS = d * E + 16;                     // padded row stride of key / value tiles
+    constexpr int KTB = 32 * RS;                       // bytes of a 32-row tile
+    const int SB = dm.dec_sb;
+    const int nw = blockDim.x >> 5;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int gq = lane >> 2, tig = lane & 3;          // fragment row (head) and column pair
+    const int D = dm.D, g = dm.g, lam = dm.lam, R = dm.R;
+    const long long p = a.pos;
+    const int nS = a.nS;
+    const Items IT = make_items(dm, a, HR);
+    const int ni = IT.ni;
+    const long long total = (long long)dm.ns * ni;
+    const long long gw = (long long)blockIdx.x * nw + warp;
+    const long long i0 = gw * per;
+    if (i0 >= total) return;                            // warp-uniform; no CTA-wide barriers below
+    const int nmine = (int)min((long long)per, total - i0);
+    const int PS = D + D / 8;                           // padded phi(q) row (floats)
+    const int CPD = D / VN;
+    const int XMD = CPD >= 16 ? 7 : (CPD >> 1) - 1;
+    const float scale = rsqrtf((float)d);
+
+    extern __shared__ __align__(128) uint8_t smd[];
+    uint8_t *wbase = smd + (size_t)warp * wbytes;
+    uint8_t *ring = wbase;
+    float *phq = (float *)(wbase + NST * SB);            // [G][PS]
+    float *pws = phq + G * PS;                           // [G][32]
+    uint8_t *fate = (uint8_t *)(pws + G * 32);           // [Lmax]
+    uint64_t *mb = (uint64_t *)(fate + 256);             // [NST]
+
+    // ---- copies of item k of this warp into buffer s: bulk (TMA) copies, completion
+    //      counted on the buffer's mbarrier. Key chunks: one copy per key row and per
+    //      value row into padded rows (stride RS: conflict-free ldmatrix), invalid rows
+    //      zeroed. Linear-band and state items: contiguous row runs, plain layout.
+    auto issue = [&](int k, int s) {
+        if (k >= nmine) return;
+        const long long gi = i0 + k;
+        const int st = (int)(gi / ni), it = (int)(gi % ni);
+        uint8_t *buf = ring + (size_t)s * SB;
+        uint64_t *bar = &mb[s];
+        if (it < IT.nkc) {
+            const int k0 = it * 32;
+            const int nv = min(32, IT.nsoft - k0);
+            if (lane == 0) umma::mbar_arrive_expect_tx(bar, (uint32_t)nv * 2 * d * E);
+            __syncwarp();
+            uint8_t *kd = buf + (size_t)lane * RS, *vd = buf + KTB + (size_t)lane * RS;
+            const int key = k0 + lane;
+            if (lane < nv) {
+                const T *kr, *vr;
+                if (key < nS) {
+                    kr = (const T *)S.KS + ((size_t)st * lam + key) * d;
+                    vr = (const T *)S.VS + ((size_t)st * lam + key) * d;
+                } else {
+                    const long long j = IT.wlo + (key - nS);
+                    kr = (const T *)S.KR + ((size_t)st * R + (j & (R - 1))) * d;
+                    vr = (const T *)S.VR + ((size_t)st * R + (j & (R - 1))) * d;
+                }
+                umma::bulk_g2s(kd, kr, (uint32_t)(d * E), bar);
+                umma::bulk_g2s(vd, vr, (uint32_t)(d * E), bar);
+            } else {
+#pragma unroll
+                for (int c = 0; c < CPR; ++c) {
+                    *(uint4 *)(kd + c * 16) = make_uint4(0, 0, 0, 0);
+                    *(uint4 *)(vd + c * 16) = make_uint4(0, 0, 0, 0);
+                }
+            }
+        } else if (lane == 0) {
+            if (it < IT.nkc + IT.nlc) {
+                const long long j0 = IT.jlo + (long long)(it - IT.nkc) * 16;
+                const int nl = (int)min(16LL, IT.lhi - j0);
+                const uint32_t fb = (uint32_t)(D * E), rb = (uint32_t)(d * E);
+                umma::mbar_arrive_expect_tx(bar, (uint32_t)nl * (fb + rb));
+                const T *phiR = (const T *)S.phiV + ((size_t)st * (lam + R) + lam) * D;
+                const T *VR = (const T *)S.VR + (size_t)st * R * d;
+                uint8_t *fd = buf, *vd = buf + 16 * fb;
+                long long j = j0;
+                int n = nl;
+                while (n > 0) {
+                    const int slot = (int)(j & (R - 1));
+                    const int m = min(n, R - slot);
+                    umma::bulk_g2s(fd, phiR + (size_t)slot * D, (uint32_t)m * fb, bar);
+                    umma::bulk_g2s(vd, VR + (size_t)slot * d, (uint32_t)m * rb, bar);
+                    fd += (size_t)m * fb;
+                    vd += (size_t)m * rb;
+                    j += m;
+                    n -= m;
+                }
+            } else {
+                const int r0 = (it - IT.nkc - IT.nlc) * HR;
+                umma::mbar_arrive_expect_tx(bar, (uint32_t)(HR * d * 4 + HR * 4));
+                umma::bulk_g2s(buf, S.H + ((size_t)st * D + r0) * d, (uint32_t)(HR * d * 4), bar);
+                umma::bulk_g2s(buf + HR * d * 4, S.s + (size_t)st * D + r0, (uint32_t)(HR * 4), bar);
+            }
+        }
+    };
+    if (lane == 0)
+        for (int i = 0; i < NST; ++i) umma::mbar_init(&mb[i], 1);
+    __syncwarp();
+    for (int k = 0; k < NST; ++k) issue(k, k);
+
+    // ---- per-stream state of this warp
+    int cur = -1;
+    uint32_t qa0[KS_], qa2[KS_];
+    float mrow = 0.f, lrow = 0.f;
+    float oc[ND][4];
+    float ld[G], lo[G][DPL];
+    auto begin = [&](int st) {
+        const int b = st / dm.Hkv, hk = st % dm.Hkv;
+        const T *qg = (const T *)a.q + ((size_t)b * dm.Hq + (size_t)hk * g) * d;
+        const bool hv = gq < g;
+#pragma unroll
+        for (int ks = 0; ks < KS_; ++ks) {
+            qa0[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + tig * 2) : 0u;
+            qa2[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + 8 + tig * 2) : 0u;
+        }
+        const float *pg = S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
+        for (int e = lane; e < g * D; e += 32) {
+            const int h = e / D, f = e - h * D;
+            phq[h * PS + qidx<VN>(f)] = pg[e];
+        }
+        const int nL = (int)(a.L_hi - a.L_lo);
+        for (int i = lane; i < nL; i += 32) fate[i] = S.pend[(size_t)st * dm.Lmax + i];
+        mrow = 0.f;
+        lrow = 0.f;
+#pragma unroll
+        for (int n = 0; n < ND; ++n) oc[n][0] = oc[n][1] = oc[n][2] = oc[n][3] = 0.f;
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            ld[h] = 0.f;
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) lo[h][u] = 0.f;
+        }
+        __syncwarp();
+    };
+    const size_t rec = 2 * d + 4;
+    auto flush = [&](int st) {
+        const long long first = ((long long)st * ni) / per;            // first warp with items of st
+        const long long last = ((long long)st * ni + ni - 1) / per;
+        const int nparts = (int)(last - first + 1), pi = (int)(gw - first);
+        float lq = lrow + __shfl_xor_sync(0xffffffffu, lrow, 1);
+        lq += __shfl_xor_sync(0xffffffffu, lq, 2);
+        float *base = S.part + (size_t)st * dm.nsplit * g * rec;
+        if (gq < g) {
+            float *pr = base + ((size_t)pi * g + gq) * rec;
+            if (tig == 0) {
+                pr[0] = mrow;
+                pr[1] = lq;
+                pr[3] = 0.f;
+            }
+#pragma unroll
+            for (int n = 0; n < ND; ++n) {
+                pr[4 + n * 8 + tig * 2] = oc[n][0];
+                pr[4 + n * 8 + tig * 2 + 1] = oc[n][1];
+            }
+        }
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            if (h < g) {
+                float *pr = base + ((size_t)pi * g + h) * rec;
+                if (lane == 0) pr[2] = ld[h];
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) pr[4 + d + lane * DPL + u] = lo[h][u];
+            }
+        }
+        __threadfence();
+        __syncwarp();
+        int prev = 0;
+        if (lane == 0) prev = atomicAdd(&S.dec_cnt[st], 1);
+        prev = __shfl_sync(0xffffffffu, prev, 0);
+        if (prev != nparts - 1) return;
+        // this warp wrote the stream's last partial: merge (online-softmax identity) and write out
+        __threadfence();
+        const int b = st / dm.Hkv, hk = st % dm.Hkv;
+        for (int h = 0; h < g; ++h) {
+            float M = 0.f;
+            for (int q2 = 0; q2 < nparts; ++q2) M = fmaxf(M, __ldcg(base + ((size_t)q2 * g + h) * rec));
+            float Ls = 0.f, LD = 0.f, O[DPL], LO[DPL];
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) O[u] = LO[u] = 0.f;
+            for (int q2 = 0; q2 < nparts; ++q2) {
+                const float *pr = base + ((size_t)q2 * g + h) * rec;
+                const float f = __expf(__ldcg(pr) - M);
+                Ls = fmaf(f, __ldcg(pr + 1), Ls);
+                LD += __ldcg(pr + 2);
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) {
+                    O[u] = fmaf(f, __ldcg(pr + 4 + lane * DPL + u), O[u]);
+                    LO[u] += __ldcg(pr + 4 + d + lane * DPL + u);
+                }
+            }
+            const float em = __expf(-M);
+            const float rden = 1.f / (Ls + em * (LD + dm.eps));
+            T *out = (T *)a.out + ((size_t)b * dm.Hq + (size_t)hk * g + h) * d;
+#pragma unroll
+            for (int u = 0; u < DPL; ++u) out[lane * DPL + u] = from_f<T>((O[u] + em * LO[u]) * rden);
+        }
+        if (lane == 0) S.dec_cnt[st] = 0;
+    };
+
+    for (int k = 0; k < nmine; ++k) {
+        const int s = k % NST;
+        const long long gi = i0 + k;
+        const int st = (int)(gi / ni), it = (int)(gi % ni);
+        if (st != cur) {
+            if (cur >= 0) flush(cur);
+            begin(st);
+            cur = st;
+        }
+        bool got = true;
+        if (lane == 0) {
+            const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
+            got = !aborted && umma::mbar_wait(&mb[s], (uint32_t)((k / NST) & 1), kWaitNs);
+            if (!got) raise_error(S.err, ERR_TIMEOUT);
+        }
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
+            // give up on the step (the error word is set): let copies in flight land
+            if (lane == 0)
+                for (int k2 = k + 1; k2 < k + NST && k2 < nmine; ++k2)
+                    umma::mbar_wait(&mb[k2 % NST], (uint32_t)((k2 / NST) & 1), kWaitNs);
+            return;
+        }
+        const uint8_t *buf = ring + (size_t)s * SB;
+        if (it < IT.nkc) {
+            const int k0 = it * 32;
+            const int key = k0 + lane;
+            bool soft = key < IT.nsoft;
+            if (soft && key >= nS) {
+                const long long j = IT.wlo + (key - nS);
+                if (j >= a.L_lo && j < a.L_hi && fate[(int)(j - a.L_lo)] == 0) soft = false;   // kept: a cache slot
+            }
+            const unsigned smask = __ballot_sync(0xffffffffu, soft);
+            const uint32_t kb = umma::smem_u32(buf), vb = kb + KTB;
+            float sc[4][4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+            const int mi = lane >> 3, rr = lane & 7;
+#pragma unroll
+            for (int np = 0; np < 2; ++np) {
+#pragma unroll
+                for (int kp = 0; kp < KS_; ++kp) {
+                    const int krow = np * 16 + (mi >> 1) * 8 + rr;
+                    const int kch = kp * 2 + (mi & 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4(kb + (uint32_t)(krow * RS + kch * 16), b0, b1, b2, b3);
+                    mma16816(sc[np * 2], qa0[kp], qa2[kp], b0, b1);
+                    mma16816(sc[np * 2 + 1], qa0[kp], qa2[kp], b2, b3);
+                }
+            }
+            float cmax = 0.f;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+                for (int e = 0; e < 2; ++e) {
+                    sc[nt][e] *= scale;
+                    if ((smask >> (nt * 8 + tig * 2 + e)) & 1u) cmax = fmaxf(cmax, sc[nt][e]);
+                }
+            cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 1));
+            cmax = fmaxf(cmax, __shfl_xor_sync(0xffffffffu, cmax, 2));
+            const float mn = fmaxf(mrow, cmax);
+            const float f = __expf(mrow - mn);
+            mrow = mn;
+            lrow *= f;
+#pragma unroll
+            for (int n = 0; n < ND; ++n) {
+                oc[n][0] *= f;
+                oc[n][1] *= f;
+            }
+            uint32_t pa[4];
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+                const float p0 = ((smask >> (nt * 8 + tig * 2)) & 1u) ? __expf(sc[nt][0] - mn) : 0.f;
+                const float p1 = ((smask >> (nt * 8 + tig * 2 + 1)) & 1u) ? __expf(sc[nt][1] - mn) : 0.f;
+                pa[nt] = pack2(p0, p1);
+                lrow += umma::bf16lo_to_f32(pa[nt]) + umma::bf16hi_to_f32(pa[nt]);
+            }
+#pragma unroll
+            for (int kk = 0; kk < 2; ++kk) {
+#pragma unroll
+                for (int n = 0; n < ND; n += 2) {
+                    const int vrow = kk * 16 + (mi & 1) * 8 + rr;
+                    const int vch = n + (mi >> 1);
+                    uint32_t b0, b1, b2, b3;
+                    ldsm_x4_t(vb + (uint32_t)(vrow * RS + vch * 16), b0, b1, b2, b3);
+                    mma16816(oc[n], pa[kk * 2], pa[kk * 2 + 1], b0, b1);
+                    mma16816(oc[n + 1], pa[kk * 2], pa[kk * 2 + 1], b2, b3);
+                }
+            }
+        } else if (it < IT.nkc + IT.nlc) {
+            const long long j0 = IT.jlo + (long long)(it - IT.nkc) * 16;
+            const int nl = (int)min(16LL, IT.lhi - j0);
+            const int kk = lane & 15, hf = lane >> 4;
+            const bool lin = kk < nl && fate[(int)(j0 + kk - a.L_lo)] != 0;
+            float gl[G];
+#pragma unroll
+            for (int h = 0; h < G; ++h) gl[h] = 0.f;
+            if (lin) {
+                const uint8_t *fr = buf + (size_t)kk * D * E;
+                const int cb = hf * (CPD >> 1);
+                for (int c = 0; c < (CPD >> 1); ++c) {
+                    const int c2 = cb + (c ^ (kk & XMD));
+                    float ff[VN];
+                    Chunk<T>::load(fr + c2 * 16, ff);
+#pragma unroll
+                    for (int h = 0; h < G; ++h) {
+                        if (h < g) {
+                            const float *ph = phq + h * PS + qoff<VN>(c2, 0);
+#pragma unroll
+                            for (int u = 0; u < VN; u += 4) {
+                                const float4 q4 = *(const float4 *)(ph + u);
+                                gl[h] = fmaf(q4.x, ff[u], gl[h]);
+                                gl[h] = fmaf(q4.y, ff[u + 1], gl[h]);
+                                gl[h] = fmaf(q4.z, ff[u + 2], gl[h]);
+                                gl[h] = fmaf(q4.w, ff[u + 3], gl[h]);
+                            }
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int h = 0; h < G; ++h) {
+                if (h < g) {
+                    gl[h] += __shfl_xor_sync(0xffffffffu, gl[h], 16);
+                    if (hf == 0) pws[h * 32 + kk] = lin ? gl[h] : 0.f;
+                }
+            }
+            __syncwarp();
+            const uint8_t *vbp = buf + (size_t)16 * D * E;
+            for (int jj = 0; jj < nl; ++jj) {
+                const T *vr = (const T *)(vbp + (size_t)jj * d * E);
+                float vf[DPL];
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) vf[u] = to_f<T>(vr[lane * DPL + u]);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    if (h < g) {
+                        const float wv = pws[h * 32 + jj];
+#pragma unroll
+                        for (int u = 0; u < DPL; ++u) lo[h][u] = fmaf(wv, vf[u], lo[h][u]);
+                        ld[h] += wv;
+                    }
+                }
+            }
+        } else {
+            const int r0 = (it - IT.nkc - IT.nlc) * HR;
+            const float *Hs = (const float *)buf;
+            const float *ss = (const float *)(buf + HR * d * 4);
+#pragma unroll 4
+            for (int i = 0; i < HR; ++i) {
+                float hv[DPL];
+#pragma unroll
+                for (int u = 0; u < DPL; ++u) hv[u] = Hs[i * d + lane * DPL + u];
+                const float si = ss[i];
+                const int fi = qidx<VN>(r0 + i);
+#pragma unroll
+                for (int h = 0; h < G; ++h) {
+                    if (h < g) {
+                        const float fq = phq[h * PS + fi];
+#pragma unroll
+                        for (int u = 0; u < DPL; ++u) lo[h][u] = fmaf(fq, hv[u], lo[h][u]);
+                        ld[h] = fmaf(fq, si, ld[h]);
+                    }
+                }
+            }
+        }
+        __syncwarp();
+        fence_proxy_async();   // this buffer's reads are done before the copies overwrite it
+        issue(k + NST, s);
+    }
+    flush(cur);
+}
+
+// bytes of shared memory per warp of decode_stream_kernel
+inline int stream_warp_bytes(const Dims &dm, int G)
+{
+    const size_t b = (size_t)3 * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
+    return (int)((b + 127) / 128 * 128);
+}
+
 // Appends the step's key/value to the window ring (one CTA per stream) and,
 // with with_phi, writes phi(k) of it into the phi rows (warp 0).
 template <typename T>
@@ -643,7 +1131,7 @@ __global__ void append_kernel(Dims dm, DevState S, const T *__restrict__ k, cons
         VR[c] = v[(size_t)st * dm.d + c];
     }
     if (with_phi && threadIdx.x < 32)
-        phi_row_warp<T>(k + (size_t)st * dm.d, S.W, xs, dm.d, dm.Dh,
+        phi_row_warp<T, T>(k + (size_t)st * dm.d, S.W, xs, dm.d, dm.Dh,
                         (T *)S.phiV + ((size_t)st * (dm.lam + dm.R) + dm.lam + slot) * dm.D);
 }
 
@@ -665,16 +1153,48 @@ size_t decode_smem_bytes(const Dims &dm) { return dec_layout(dm).total; }
 
 bool decode_plan(Dims *dm)
 {
-    const int e = dm->dtype == 0 ? 4 : 2;
+    if (dm->dtype != 0) {
+        // streaming kernel: 3 buffers per warp of key chunks (2 swizzled 32-row tiles),
+        // linear-band items (16 phi rows + 16 value rows) or state items (16 H rows + s)
+        const size_t sb_keys = (size_t)2 * 32 * (dm->d * 2 + 16);
+        const size_t sb_lin = (size_t)16 * (dm->D + dm->d) * 2;
+        const size_t sb_h = (size_t)16 * dm->d * 4 + 64;
+        size_t sb = sb_keys > sb_h ? sb_keys : sb_h;
+        if (sb_lin > sb) sb = sb_lin;
+        dm->dec_sb = (int)((sb + 127) / 128 * 128);
+        dm->dec_nst = 3;
+        const int G = dm->g <= 1 ? 1 : dm->g <= 2 ? 2 : dm->g <= 4 ? 4 : 8;
+        // warps per CTA: the most resident warps per SM (shared memory, ~160 registers per thread)
+        const size_t wb = (size_t)stream_warp_bytes(*dm, G);
+        int best = 0;
+        dm->dec_nw = 0;
+        for (int nw = 4; nw >= 1; --nw) {
+            if ((size_t)nw * wb > 227 * 1024) continue;
+            int res = (int)((228 * 1024) / (nw * wb + 1280));
+            const int rlim = 65536 / (nw * 32 * 160);
+            if (res > rlim) res = rlim;
+            if (res * nw > best) {
+                best = res * nw;
+                dm->dec_nw = nw;
+            }
+        }
+        if (dm->dec_nw == 0) return false;
+        const long long nkeys = (long long)dm->lam + dm->eta + 1;
+        const long long items = (nkeys + 31) / 32 + (dm->Cdec + 15) / 16 + dm->D / 16;
+        dm->nsplit = (int)((items + kMinPer - 1) / kMinPer + 1);
+        return true;
+    }
+    const int e = 4;
+    const int hrows = 32;
     const size_t sb_keys = (size_t)32 * 2 * dm->d * e;
     const size_t sb_lin = (size_t)16 * (dm->D + dm->d) * e;
-    const size_t sb_h = (size_t)32 * dm->d * 4 + 128;
+    const size_t sb_h = (size_t)hrows * dm->d * 4 + (size_t)hrows * 4;
     size_t sb = sb_keys > sb_h ? sb_keys : sb_h;
     if (sb_lin > sb) sb = sb_lin;
     dm->dec_sb = (int)((sb + 127) / 128 * 128);
     // shape with the most staging bytes in flight per SM (buffers beyond the one
     // being worked on), at up to 228 KB of shared memory per SM
-    const int shapes[6][2] = {{2, 3}, {4, 3}, {4, 2}, {2, 2}, {1, 3}, {1, 2}};
+    const int shapes[6][2] = {{4, 3}, {2, 3}, {4, 2}, {2, 2}, {1, 3}, {1, 2}};
     long long best = -1;
     int bw = 0, bs = 0, bres = 1;
     for (auto &sh : shapes) {
@@ -682,8 +1202,8 @@ bool decode_plan(Dims *dm)
         dm->dec_nst = sh[1];
         const size_t tot = dec_layout(*dm).total;
         if (tot > 200 * 1024) continue;
-        int res = (int)((228 * 1024) / (tot + 1024));
-        if (res > 16 / sh[0]) res = 16 / sh[0];       // registers: ~170 per thread
+        int res = (int)((228 * 1024) / (tot + 1024 + 256));   // + driver and static shared memory
+        if (res > 16 / sh[0]) res = 16 / sh[0];                 // registers
         const long long fly = (long long)res * sh[0] * (sh[1] - 1) * dm->dec_sb;
         if (fly > best) {
             best = fly;
@@ -697,7 +1217,7 @@ bool decode_plan(Dims *dm)
     dm->dec_nst = bs;
     // about two waves of resident CTAs, at least one item per warp
     const long long nkeys = (long long)dm->lam + dm->eta + 1;
-    const long long items = (nkeys + 31) / 32 + (dm->Cdec + 15) / 16 + dm->D / 32;
+    const long long items = (nkeys + 31) / 32 + (dm->Cdec + 15) / 16 + dm->D / hrows;
     const long long want = 2LL * kSMs * bres;
     long long nsp = (want + dm->ns - 1) / dm->ns;
     const long long cap = (items + bw - 1) / bw;
@@ -718,9 +1238,74 @@ void launch_decode_append(const Dims &dm, const DevState &S, const void *k, cons
             dm, S, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, pos, with_phi);
 }
 
+// Items of one stream at this step (the host mirror of make_items).
+static long long host_items(const Dims &dm, const DecodeArgs &a, int hrows)
+{
+    const long long p = a.pos;
+    const long long jlo = a.t0 - dm.eta > 0 ? a.t0 - dm.eta : 0;
+    const long long wlo = p - dm.eta + 1 > jlo ? p - dm.eta + 1 : jlo;
+    long long lhi = a.L_hi < wlo ? a.L_hi : wlo;
+    if (lhi < jlo) lhi = jlo;
+    const long long nsoft = a.nS + (p - wlo + 1);
+    return (nsoft + 31) / 32 + (lhi - jlo + 15) / 16 + dm.D / hrows;
+}
+
+
 void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, int do_append,
                         cudaStream_t stream)
 {
+    if (dm.dtype != 0) {
+        // bfloat16: preparation, then the persistent streaming kernel
+        const size_t psm = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
+        {
+            static size_t attr = 0;
+            if (psm > attr) {
+                cudaFuncSetAttribute(decode_prep_kernel<__nv_bfloat16>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
+                attr = psm;
+            }
+            const int rows = dm.B * dm.Hq + (do_append ? dm.ns : 0);
+            int grid = (rows + 7) / 8;
+            if (grid > kSMs * 4) grid = kSMs * 4;
+            decode_prep_kernel<__nv_bfloat16><<<grid, 256, psm, stream>>>(dm, S, a, do_append);
+        }
+        const int G = dm.g <= 1 ? 1 : dm.g <= 2 ? 2 : dm.g <= 4 ? 4 : 8;
+        const int wb = stream_warp_bytes(dm, G);
+        const int nw = dm.dec_nw;
+        const size_t smem = (size_t)nw * wb;
+        int res = (int)((228 * 1024) / (smem + 1280));
+        if (res < 1) res = 1;
+        if (res > 65536 / (nw * 32 * 160)) res = 65536 / (nw * 32 * 160);
+        const long long total = (long long)dm.ns * host_items(dm, a, 16);
+        const long long warps_cap = (long long)kSMs * res * nw;
+        long long per = (total + warps_cap - 1) / warps_cap;
+        if (per < kMinPer) per = kMinPer;
+        const long long nwarps = (total + per - 1) / per;
+        const int grid = (int)((nwarps + nw - 1) / nw);
+#define LOLA_STREAM(DPL, GG)                                                                       \
+    do {                                                                                           \
+        static size_t attr = 0;                                                                    \
+        if (smem > attr) {                                                                         \
+            cudaFuncSetAttribute(decode_stream_kernel<DPL, GG>,                                    \
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);          \
+            attr = smem;                                                                           \
+        }                                                                                          \
+        decode_stream_kernel<DPL, GG><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb);    \
+    } while (0)
+#define LOLA_STREAM_G(DPL)                                                                         \
+    do {                                                                                           \
+        if (G == 1) LOLA_STREAM(DPL, 1);                                                           \
+        else if (G == 2) LOLA_STREAM(DPL, 2);                                                      \
+        else if (G == 4) LOLA_STREAM(DPL, 4);                                                      \
+        else LOLA_STREAM(DPL, 8);                                                                  \
+    } while (0)
+        if (dm.d == 32) LOLA_STREAM_G(1);
+        else if (dm.d == 64) LOLA_STREAM_G(2);
+        else LOLA_STREAM_G(4);
+#undef LOLA_STREAM_G
+#undef LOLA_STREAM
+        return;
+    }
     dim3 grid(dm.nsplit, dm.ns);
     const size_t smem = dec_layout(dm).total;
     const int threads = 32 * dm.dec_nw;
@@ -734,15 +1319,9 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
         }                                                                                          \
         decode3_kernel<T, DPL><<<grid, threads, smem, stream>>>(dm, S, a, do_append);              \
     } while (0)
-    if (dm.dtype == 0) {
-        if (dm.d == 32) LOLA_DECODE3(float, 1);
-        else if (dm.d == 64) LOLA_DECODE3(float, 2);
-        else LOLA_DECODE3(float, 4);
-    } else {
-        if (dm.d == 32) LOLA_DECODE3(__nv_bfloat16, 1);
-        else if (dm.d == 64) LOLA_DECODE3(__nv_bfloat16, 2);
-        else LOLA_DECODE3(__nv_bfloat16, 4);
-    }
+    if (dm.d == 32) LOLA_DECODE3(float, 1);
+    else if (dm.d == 64) LOLA_DECODE3(float, 2);
+    else LOLA_DECODE3(float, 4);
 #undef LOLA_DECODE3
 }
 

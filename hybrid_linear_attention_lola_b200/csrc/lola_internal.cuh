@@ -23,7 +23,7 @@ enum : int { ERR_BOUNDS = 1, ERR_TIMEOUT = 2 };
 struct Dims {
     int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
     int Nmax, mmax;   // prefill scratch capacity: tokens per call, intervals per call
-    int nsplit;       // decode: CTAs per stream
+    int nsplit;       // decode: partial records per stream (CTAs, or warp ranges)
     int dec_nw;       // decode: warps per CTA
     int dec_nst;      // decode: staging buffers per warp
     int dec_sb;       // decode: bytes per staging buffer
@@ -45,7 +45,8 @@ struct DevState {
     int *err;          // [4]          device error words
     // decode scratch (phi buffers hold the input dtype)
     void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
-    float *part;       // [ns][nsplit][g][2d + 4] split partials
+    float *part;       // [ns][nsplit][g][2d + 4] partials of the warps / CTAs sharing a stream
+    float *phiQd;      // [B][Hq][D]   fp32 phi(q) of the decode step (bfloat16 path)
     int *dec_cnt;      // [ns] finished decode CTAs per stream (reset by the last one)
 };
 
@@ -124,10 +125,10 @@ __device__ __forceinline__ float warp_min(float x)
 
 // phi(x) = [softmax(x W), softmax(-x W)] of one row, computed by one warp. W (fp32, [d][Dh]) sits in shared memory; lane l owns
 // features l, l + 32, ... The row max / min shift is exact in real arithmetic.
-template <typename T>
+template <typename T, typename O>
 __device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const float *__restrict__ Ws,
                                              float *__restrict__ xs, int d, int Dh,
-                                             T *__restrict__ out)
+                                             O *__restrict__ out)
 {
     const int lane = threadIdx.x & 31;
     for (int a = lane; a < d; a += 32) xs[a] = to_f<T>(x[a]);
@@ -170,8 +171,8 @@ __device__ __forceinline__ void phi_row_warp(const T *__restrict__ x, const floa
     for (int u = 0; u < 4; ++u) {
         const int i = lane + 32 * u;
         if (i < Dh) {
-            out[i] = from_f<T>(ep[u] * rp);
-            out[Dh + i] = from_f<T>(en[u] * rn);
+            out[i] = from_f<O>(ep[u] * rp);
+            out[Dh + i] = from_f<O>(en[u] * rn);
         }
     }
     __syncwarp();

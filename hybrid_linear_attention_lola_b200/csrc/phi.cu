@@ -24,7 +24,7 @@ __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, cons
         const int st = (int)(r / per_stream);
         const int i = (int)(r % per_stream);
         const int vrow = i < nS ? i : dm.lam + (i - nS);
-        phi_row_warp<T>(src.krow(st, vrow), Ws, xs, dm.d, dm.Dh,
+        phi_row_warp<T, T>(src.krow(st, vrow), Ws, xs, dm.d, dm.Dh,
                         phi_out + ((size_t)st * nvrows + vrow) * dm.D);
     }
 }
@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) phi_q_kernel(int d, int Dh, const float *
     const int warps = blockDim.x >> 5;
     for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < rows;
          r += (long long)gridDim.x * warps)
-        phi_row_warp<T>(q + (size_t)r * d, Ws, xs, d, Dh, phi_out + (size_t)r * 2 * Dh);
+        phi_row_warp<T, T>(q + (size_t)r * d, Ws, xs, d, Dh, phi_out + (size_t)r * 2 * Dh);
 }
 
 static int grid_for(long long rows, int warps_per_block)

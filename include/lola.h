@@ -113,12 +113,14 @@ lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const
  * or code running while a CUDA graph is being captured, where cudaMalloc is
  * not allowed. The paper has no counterpart to this call; it only changes
  * where temporaries live. The per-step scratch of the decode attention (the
- * partial sums of the CTAs that share a stream) is taken from an 8 MiB array
- * inside the library (a static device array: every GPU that loads the library
- * holds it until the process exits) instead of the workspace. The call
- * allocates nothing. Configs whose decode scratch,
- * streams*splits*(n_q_heads/n_kv_heads)*(2*head_dim+4)*4 bytes (rounded up to
- * 256; splits = CTAs per stream, chosen by the library), exceed 8 MiB get
+ * partial sums of the warps or CTAs that share a stream, and for bfloat16 the
+ * fp32 query features) is taken from an 8 MiB array inside the library (a
+ * static device array: every GPU that loads the library holds it until the
+ * process exits) instead of the workspace. The call allocates nothing.
+ * Configs whose decode scratch,
+ * streams*parts*(n_q_heads/n_kv_heads)*(2*head_dim+4)*4 bytes (parts = partial
+ * records per stream, chosen by the library) plus, for bfloat16,
+ * batch*n_q_heads*feat_dim*4 bytes (each rounded up to 256), exceed 8 MiB get
  * LOLA_ERR_WORKSPACE.
  * The first call on a device looks up the array's device address (once per
  * device, with the device current); make that first call before any stream

@@ -30,6 +30,17 @@ def test_state_bytes_for_every_workload(lib):
         assert n > 0 and n % 256 == 0
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("head_dim,feat_dim,g", [(32, 32, 1), (64, 128, 4), (128, 256, 8), (128, 64, 3)])
+def test_state_bytes_across_shapes(lib, dtype, head_dim, feat_dim, g):
+    # every documented head_dim / feat_dim / group size keeps a launch shape that fits
+    cfg = L.make_config(batch=3, n_q_heads=2 * g, n_kv_heads=2, head_dim=head_dim, feat_dim=feat_dim,
+                        window=64, lambda_=512, chunk=64, decode_interval=64, max_prefill_tokens=128,
+                        eps=1e-6, dtype=dtype)
+    n = L.lola_state_bytes(cfg)
+    assert n > 0 and n % 256 == 0
+
+
 def test_stream_bytes_constant_in_sequence_length(lib):
     w = wl.WORKLOADS["long-context"]
     sizes = {L.lola_state_stream_bytes(L.config_from_workload(w, max_prefill_tokens=n))

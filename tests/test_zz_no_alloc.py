@@ -67,7 +67,7 @@ def test_static_decode_matches_decode_step_twice():
 
 def test_static_decode_rejects_scratch_beyond_limit():
     # 128 sequences x 64 query heads (8 per kv-head), head_dim 128, feat_dim 256:
-    # query features 4 MiB + split partials 8.5 MB exceed the 8 MiB array
+    # the fp32 query features alone (8 MiB) plus the partials exceed the 8 MiB array
     cfg = L.make_config(batch=128, n_q_heads=64, n_kv_heads=8, head_dim=128, feat_dim=256,
                         window=1, lambda_=0, chunk=1, decode_interval=1, max_prefill_tokens=1,
                         eps=1e-6, dtype="bf16")
