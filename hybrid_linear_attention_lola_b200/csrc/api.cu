@@ -37,6 +37,7 @@ struct lola_state {
     cudaStream_t chain_stream;
     cudaEvent_t ev_fork;
     cudaEvent_t ev_seg[kMaxSeg];
+    lola::DecMaps maps;              // TMA descriptors of the cache / ring arrays (bf16 decode)
     int32_t *sel_log;
     long long sel_cap;
     const int32_t *ovr;
@@ -302,7 +303,7 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
     Sx.phiQd = phiq;
     {
         PhaseScope ps(st, PH_DECODE, stream);
-        lola::launch_decode_attn(dm, Sx, da, do_append, stream);
+        lola::launch_decode_attn(dm, Sx, da, do_append, dm.dec_tma ? &st->maps : nullptr, stream);
         counted(1);
     }
     st->pos = pos + 1;
@@ -389,6 +390,13 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
             return LOLA_ERR_CUDA;
         }
         st->seg_len = len;
+    }
+    if (dm.dec_tma && !lola::make_decode_maps(dm, st->S, &st->maps)) {
+        fprintf(stderr, "lola: cuTensorMapEncodeTiled failed\n");
+        cudaGetLastError();
+        if (st->chain_stream != nullptr) cudaStreamDestroy(st->chain_stream);
+        delete st;
+        return LOLA_ERR_CUDA;
     }
     lola::launch_init_state(dm, st->S, W, (cudaStream_t)cuda_stream);
     counted(1);

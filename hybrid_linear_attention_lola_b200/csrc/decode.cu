@@ -24,6 +24,8 @@
 #include "lola_internal.cuh"
 #include "umma.cuh"
 
+#include <cudaTypedefs.h>
+
 namespace lola {
 
 namespace {
@@ -112,12 +114,17 @@ template <int VN> __device__ __forceinline__ int qidx(int x) { return qoff<VN>(x
 //   [nkc, nkc + nlc)    16 linear-band tokens of [jlo, lhi) (left the window this
 //                       interval; folded ones are linear, kept ones are skipped)
 //   [nkc + nlc, ni)     hrows feature rows of the state (H, s)
+// With tma, softmax keys come in aligned 32-row blocks instead: cache slots
+// [32c, 32c + 32) (c < ncc), then the blocks of 32 ring slots the window
+// [wlo, p] touches (nwc of them, from block wblk0 on, modulo R / 32); rows of a
+// block outside the key set are masked.
 struct Items {
     long long jlo, wlo, lhi;
     int nsoft, nkc, nlc, ni;
+    int ncc, nwc, wblk0;
 };
 
-__device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a, int hrows)
+__host__ __device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a, int hrows, int tma)
 {
     Items it;
     const long long p = a.pos;
@@ -125,8 +132,21 @@ __device__ __forceinline__ Items make_items(const Dims &dm, const DecodeArgs &a,
     it.wlo = p - dm.eta + 1 > it.jlo ? p - dm.eta + 1 : it.jlo;
     it.lhi = a.L_hi < it.wlo ? a.L_hi : it.wlo;
     if (it.lhi < it.jlo) it.lhi = it.jlo;
-    it.nsoft = a.nS + (int)(p - it.wlo + 1);
-    it.nkc = (it.nsoft + 31) / 32;
+    const int nwin = (int)(p - it.wlo + 1);
+    it.nsoft = a.nS + nwin;
+    it.ncc = (a.nS + 31) / 32;
+    it.nwc = 0;
+    it.wblk0 = 0;
+    if (tma) {
+        if (nwin > 0) {
+            const int f = (int)(it.wlo & (dm.R - 1)) >> 5, l = (int)(p & (dm.R - 1)) >> 5;
+            it.nwc = ((l - f) & ((dm.R >> 5) - 1)) + 1;
+            it.wblk0 = f;
+        }
+        it.nkc = it.ncc + it.nwc;
+    } else {
+        it.nkc = (it.nsoft + 31) / 32;
+    }
     it.nlc = (int)((it.lhi - it.jlo + 15) / 16);
     it.ni = it.nkc + it.nlc + dm.D / hrows;
     return it;
@@ -147,7 +167,7 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
     const int D = dm.D, Dh = dm.Dh, g = dm.g, lam = dm.lam, R = dm.R;
     const long long p = a.pos;
     const int nS = a.nS;
-    const Items IT = make_items(dm, a, 32);
+    const Items IT = make_items(dm, a, 32, 0);
     const int gw = split * nw + warp, wstride = dm.nsplit * nw;
     const int nmine = gw < IT.ni ? (IT.ni - gw + wstride - 1) / wstride : 0;
     const DecLayout L = dec_layout(dm);
@@ -727,7 +747,8 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, D
 // writes its partial (m, l, linear den, softmax num, linear num per head); the
 // warp that writes a stream's last partial merges them (a per-stream counter).
 template <int DPL, int G>
-__global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S, DecodeArgs a, int per, int wbytes)
+__global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S, DecodeArgs a, int per, int wbytes,
+                                                             const __grid_constant__ DecMaps maps)
 {
     using T = __nv_bfloat16;
     constexpr int d = 32 * DPL;
@@ -738,8 +759,10 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     constexpr int ND = d / 8;                          // n-tiles of P V (8 value dims each)
     constexpr int HR = 16;                             // state rows per item
     constexpr int NST = 3;                             // staging buffers per warp
-    constexpr int RS = d * E + 16;                     // padded row stride of key / value tiles
-    constexpr int KTB = 32 * RS;                       // bytes of a 32-row tile
+    constexpr int RS = d * E + 16;                     // padded row stride of key / value tiles (bulk path)
+    const bool tma = dm.dec_tma != 0;
+    // bytes of a 32-row key (or value) tile: swizzled 128-byte rows (TMA path) or padded rows
+    const int KTB = tma ? 32 * 128 * ((CPR + 7) / 8) : 32 * RS;
     const int SB = dm.dec_sb;
     const int nw = blockDim.x >> 5;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -747,7 +770,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     const int D = dm.D, g = dm.g, lam = dm.lam, R = dm.R;
     const long long p = a.pos;
     const int nS = a.nS;
-    const Items IT = make_items(dm, a, HR);
+    const Items IT = make_items(dm, a, HR, dm.dec_tma);
     const int ni = IT.ni;
     const long long total = (long long)dm.ns * ni;
     const long long gw = (long long)blockIdx.x * nw + warp;
@@ -759,7 +782,9 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     const int XMD = CPD >= 16 ? 7 : (CPD >> 1) - 1;
     const float scale = rsqrtf((float)d);
 
-    extern __shared__ __align__(128) uint8_t smd[];
+    extern __shared__ __align__(128) uint8_t smraw_d[];
+    // 1024-byte aligned base: the 128-byte swizzle of TMA boxes is address based
+    uint8_t *smd = smraw_d + (((umma::smem_u32(smraw_d) + 1023u) & ~1023u) - umma::smem_u32(smraw_d));
     uint8_t *wbase = smd + (size_t)warp * wbytes;
     uint8_t *ring = wbase;
     float *phq = (float *)(wbase + NST * SB);            // [G][PS]
@@ -777,7 +802,20 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         const int st = (int)(gi / ni), it = (int)(gi % ni);
         uint8_t *buf = ring + (size_t)s * SB;
         uint64_t *bar = &mb[s];
-        if (it < IT.nkc) {
+        if (it < IT.nkc && tma) {
+            if (lane == 0) {
+                const bool cache = it < IT.ncc;
+                const int y = cache ? it * 32 : ((IT.wblk0 + (it - IT.ncc)) & ((R >> 5) - 1)) * 32;
+                const CUtensorMap *mk = cache ? &maps.ks : &maps.kr;
+                const CUtensorMap *mv = cache ? &maps.vs : &maps.vr;
+                const int nbox = (d + 63) / 64;
+                umma::mbar_arrive_expect_tx(bar, (uint32_t)(nbox * 2 * 4096));
+                for (int bx = 0; bx < nbox; ++bx) {
+                    umma::tma_load_3d(buf + bx * 4096, mk, bx * 64, y, st, bar);
+                    umma::tma_load_3d(buf + KTB + bx * 4096, mv, bx * 64, y, st, bar);
+                }
+            }
+        } else if (it < IT.nkc) {
             const int k0 = it * 32;
             const int nv = min(32, IT.nsoft - k0);
             if (lane == 0) umma::mbar_arrive_expect_tx(bar, (uint32_t)nv * 2 * d * E);
@@ -960,13 +998,23 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         }
         const uint8_t *buf = ring + (size_t)s * SB;
         if (it < IT.nkc) {
-            const int k0 = it * 32;
-            const int key = k0 + lane;
-            bool soft = key < IT.nsoft;
-            if (soft && key >= nS) {
-                const long long j = IT.wlo + (key - nS);
-                if (j >= a.L_lo && j < a.L_hi && fate[(int)(j - a.L_lo)] == 0) soft = false;   // kept: a cache slot
+            bool soft;
+            long long j = -1;   // window token of this lane's row, if any
+            if (tma) {
+                if (it < IT.ncc) {
+                    soft = it * 32 + lane < nS;
+                } else {
+                    const int slot = ((IT.wblk0 + (it - IT.ncc)) & ((R >> 5) - 1)) * 32 + lane;
+                    j = IT.wlo + ((slot - (int)(IT.wlo & (R - 1))) & (R - 1));
+                    soft = j <= p;
+                }
+            } else {
+                const int key = it * 32 + lane;
+                soft = key < IT.nsoft;
+                if (soft && key >= nS) j = IT.wlo + (key - nS);
             }
+            if (soft && j >= 0 && j >= a.L_lo && j < a.L_hi && fate[(int)(j - a.L_lo)] == 0)
+                soft = false;   // kept leaving pair: attended as a cache slot
             const unsigned smask = __ballot_sync(0xffffffffu, soft);
             const uint32_t kb = umma::smem_u32(buf), vb = kb + KTB;
             float sc[4][4];
@@ -980,7 +1028,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                     const int krow = np * 16 + (mi >> 1) * 8 + rr;
                     const int kch = kp * 2 + (mi & 1);
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4(kb + (uint32_t)(krow * RS + kch * 16), b0, b1, b2, b3);
+                    ldsm_x4(kb + (tma ? swz<CPR>(krow, kch) : (uint32_t)(krow * RS + kch * 16)), b0, b1, b2, b3);
                     mma16816(sc[np * 2], qa0[kp], qa2[kp], b0, b1);
                     mma16816(sc[np * 2 + 1], qa0[kp], qa2[kp], b2, b3);
                 }
@@ -1019,7 +1067,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                     const int vrow = kk * 16 + (mi & 1) * 8 + rr;
                     const int vch = n + (mi >> 1);
                     uint32_t b0, b1, b2, b3;
-                    ldsm_x4_t(vb + (uint32_t)(vrow * RS + vch * 16), b0, b1, b2, b3);
+                    ldsm_x4_t(vb + (tma ? swz<CPR>(vrow, vch) : (uint32_t)(vrow * RS + vch * 16)), b0, b1, b2, b3);
                     mma16816(oc[n], pa[kk * 2], pa[kk * 2 + 1], b0, b1);
                     mma16816(oc[n + 1], pa[kk * 2], pa[kk * 2 + 1], b2, b3);
                 }
@@ -1112,7 +1160,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
 inline int stream_warp_bytes(const Dims &dm, int G)
 {
     const size_t b = (size_t)3 * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
-    return (int)((b + 127) / 128 * 128);
+    return (int)((b + 1023) / 1024 * 1024);   // every warp's buffers start 1024-byte aligned
 }
 
 // Appends the step's key/value to the window ring (one CTA per stream) and,
@@ -1156,12 +1204,14 @@ bool decode_plan(Dims *dm)
     if (dm->dtype != 0) {
         // streaming kernel: 3 buffers per warp of key chunks (2 swizzled 32-row tiles),
         // linear-band items (16 phi rows + 16 value rows) or state items (16 H rows + s)
-        const size_t sb_keys = (size_t)2 * 32 * (dm->d * 2 + 16);
+        dm->dec_tma = (dm->d == 64 || dm->d == 128) && dm->R >= 32 ? 1 : 0;
+        const size_t sb_keys = dm->dec_tma ? (size_t)2 * 32 * 128 * (dm->d / 64)
+                                           : (size_t)2 * 32 * (dm->d * 2 + 16);
         const size_t sb_lin = (size_t)16 * (dm->D + dm->d) * 2;
         const size_t sb_h = (size_t)16 * dm->d * 4 + 64;
         size_t sb = sb_keys > sb_h ? sb_keys : sb_h;
         if (sb_lin > sb) sb = sb_lin;
-        dm->dec_sb = (int)((sb + 127) / 128 * 128);
+        dm->dec_sb = (int)((sb + 1023) / 1024 * 1024);
         dm->dec_nst = 3;
         const int G = dm->g <= 1 ? 1 : dm->g <= 2 ? 2 : dm->g <= 4 ? 4 : 8;
         // warps per CTA: the most resident warps per SM (shared memory, ~160 registers per thread)
@@ -1169,8 +1219,8 @@ bool decode_plan(Dims *dm)
         int best = 0;
         dm->dec_nw = 0;
         for (int nw = 4; nw >= 1; --nw) {
-            if ((size_t)nw * wb > 227 * 1024) continue;
-            int res = (int)((228 * 1024) / (nw * wb + 1280));
+            if ((size_t)nw * wb + 1024 > 227 * 1024) continue;
+            int res = (int)((228 * 1024) / (nw * wb + 1024 + 1280));
             const int rlim = 65536 / (nw * 32 * 160);
             if (res > rlim) res = rlim;
             if (res * nw > best) {
@@ -1184,6 +1234,7 @@ bool decode_plan(Dims *dm)
         dm->nsplit = (int)((items + kMinPer - 1) / kMinPer + 1);
         return true;
     }
+    dm->dec_tma = 0;
     const int e = 4;
     const int hrows = 32;
     const size_t sb_keys = (size_t)32 * 2 * dm->d * e;
@@ -1238,21 +1289,8 @@ void launch_decode_append(const Dims &dm, const DevState &S, const void *k, cons
             dm, S, (const __nv_bfloat16 *)k, (const __nv_bfloat16 *)v, pos, with_phi);
 }
 
-// Items of one stream at this step (the host mirror of make_items).
-static long long host_items(const Dims &dm, const DecodeArgs &a, int hrows)
-{
-    const long long p = a.pos;
-    const long long jlo = a.t0 - dm.eta > 0 ? a.t0 - dm.eta : 0;
-    const long long wlo = p - dm.eta + 1 > jlo ? p - dm.eta + 1 : jlo;
-    long long lhi = a.L_hi < wlo ? a.L_hi : wlo;
-    if (lhi < jlo) lhi = jlo;
-    const long long nsoft = a.nS + (p - wlo + 1);
-    return (nsoft + 31) / 32 + (lhi - jlo + 15) / 16 + dm.D / hrows;
-}
-
-
 void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, int do_append,
-                        cudaStream_t stream)
+                        const DecMaps *maps, cudaStream_t stream)
 {
     if (dm.dtype != 0) {
         // bfloat16: preparation, then the persistent streaming kernel
@@ -1272,11 +1310,13 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
         const int G = dm.g <= 1 ? 1 : dm.g <= 2 ? 2 : dm.g <= 4 ? 4 : 8;
         const int wb = stream_warp_bytes(dm, G);
         const int nw = dm.dec_nw;
-        const size_t smem = (size_t)nw * wb;
-        int res = (int)((228 * 1024) / (smem + 1280));
+        const size_t smem = (size_t)nw * wb + 1024;   // + alignment slack
+        DecMaps mp{};
+        if (maps != nullptr) mp = *maps;
+        int res = (int)((228 * 1024) / (smem + 1280));   // smem includes the alignment slack
         if (res < 1) res = 1;
         if (res > 65536 / (nw * 32 * 160)) res = 65536 / (nw * 32 * 160);
-        const long long total = (long long)dm.ns * host_items(dm, a, 16);
+        const long long total = (long long)dm.ns * make_items(dm, a, 16, dm.dec_tma).ni;
         const long long warps_cap = (long long)kSMs * res * nw;
         long long per = (total + warps_cap - 1) / warps_cap;
         if (per < kMinPer) per = kMinPer;
@@ -1290,7 +1330,7 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);          \
             attr = smem;                                                                           \
         }                                                                                          \
-        decode_stream_kernel<DPL, GG><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb);    \
+        decode_stream_kernel<DPL, GG><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb, mp); \
     } while (0)
 #define LOLA_STREAM_G(DPL)                                                                         \
     do {                                                                                           \
@@ -1323,6 +1363,30 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
     else if (dm.d == 64) LOLA_DECODE3(float, 2);
     else LOLA_DECODE3(float, 4);
 #undef LOLA_DECODE3
+}
+
+bool make_decode_maps(const Dims &dm, const DevState &S, DecMaps *maps)
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+    if (encode == nullptr) {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+            return false;
+        encode = (PFN_cuTensorMapEncodeTiled_v12000)fn;
+    }
+    auto one = [&](CUtensorMap *m, void *base, int rows) {
+        const cuuint64_t dims[3] = {(cuuint64_t)dm.d, (cuuint64_t)(rows > 0 ? rows : 1), (cuuint64_t)dm.ns};
+        const cuuint64_t strides[2] = {(cuuint64_t)dm.d * 2, (cuuint64_t)dm.d * 2 * (rows > 0 ? rows : 1)};
+        const cuuint32_t box[3] = {64, 32, 1};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, base, dims, strides, box, estr,
+                      CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                      CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    };
+    return one(&maps->ks, S.KS, dm.lam) && one(&maps->vs, S.VS, dm.lam) && one(&maps->kr, S.KR, dm.R) &&
+           one(&maps->vr, S.VR, dm.R);
 }
 
 void launch_get_indices(const Dims &dm, const DevState &S, int nS, int32_t *idx, int32_t *cnt,

@@ -12,6 +12,7 @@
 // phi(k) scratch is laid out over the same rows.
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -27,6 +28,7 @@ struct Dims {
     int dec_nw;       // decode: warps per CTA
     int dec_nst;      // decode: staging buffers per warp
     int dec_sb;       // decode: bytes per staging buffer
+    int dec_tma;      // decode (bf16): key/value chunks arrive by tiled TMA loads (128 B swizzle)
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
     float eps;
@@ -243,6 +245,12 @@ void launch_finalize_prefill(const Dims &dm, const DevState &S, const PrefillScr
                              const void *kin, const void *vin, long long call_start, int n,
                              int nK, cudaStream_t stream);
 
+// Tiled TMA descriptors of the cache and ring key/value arrays, 3-D
+// [stream][row][head_dim] with 32-row x 64-element boxes and 128-byte swizzle.
+struct DecMaps {
+    CUtensorMap ks, vs, kr, vr;
+};
+
 struct DecodeArgs {
     long long pos;          // token index of this step
     long long t0;           // start of the open interval
@@ -262,7 +270,9 @@ void launch_decode_append(const Dims &dm, const DevState &S, const void *k, cons
                           long long pos, int with_phi, cudaStream_t stream);
 // do_append: the kernel also appends the step's k, v (and phi(k)) to the window ring.
 void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, int do_append,
-                        cudaStream_t stream);
+                        const DecMaps *maps, cudaStream_t stream);
+// Encodes the four maps for the state's buffers; false if the driver call fails.
+bool make_decode_maps(const Dims &dm, const DevState &S, DecMaps *maps);
 void launch_get_indices(const Dims &dm, const DevState &S, int nS, int32_t *idx, int32_t *cnt,
                         cudaStream_t stream);
 

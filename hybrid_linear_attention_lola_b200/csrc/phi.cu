@@ -107,6 +107,14 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
     for (long long e = tid; e < (long long)dm.ns * dm.D; e += stride) S.s[e] = 0.f;
     for (long long e = tid; e < (long long)dm.ns * dm.lam; e += stride) S.idxS[e] = -1;
     for (long long e = tid; e < (long long)dm.ns * dm.Lmax; e += stride) S.pend[e] = 0;
+    // cache slots start at zero: tiled loads of aligned 32-slot blocks read the
+    // not yet filled slots of a block too (with zero weight)
+    const long long nS_ = (long long)dm.ns * dm.lam * dm.d;
+    T *KS = (T *)S.KS, *VS = (T *)S.VS;
+    for (long long e = tid; e < nS_; e += stride) {
+        KS[e] = from_f<T>(0.f);
+        VS[e] = from_f<T>(0.f);
+    }
     const long long nR = (long long)dm.ns * dm.R * dm.d;
     T *KR = (T *)S.KR, *VR = (T *)S.VR;
     for (long long e = tid; e < nR; e += stride) {
