@@ -28,6 +28,7 @@ namespace {
 using bf16 = __nv_bfloat16;
 constexpr int kThreads = 256;
 constexpr int KT = 64;                // keys per tile
+constexpr float kLazy = 8.f;          // shift slack of the lazy rescaling (natural log units)
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
 
@@ -325,36 +326,44 @@ __global__ void __launch_bounds__(kThreads, 1)
     };
 
     float m = 0.f, lpart = 0.f;
+    // QK^T (and, for tiles with folded band keys, phi(Q) phi(K)^T) of tile t into TMEM
+    auto issue_scores = [&](int t) {
+        const TileMeta &M = meta[t & 1];
+        const uint32_t q0 = umma::smem_u32(sQ), k0 = umma::smem_u32(base + g.off_K[t & 1]);
+        for (int ks = 0; ks < d / 16; ++ks)
+            umma::mma_ss(tS, umma::kmajor_desc(q0, ks, 128), umma::kmajor_desc(k0, ks, KT), id_s, ks > 0 ? 1u : 0u);
+        if (M.lin[0] | M.lin[1]) {
+            const uint32_t pq0 = umma::smem_u32(sPhq), pk0 = umma::smem_u32(sPhk);
+            for (int ks = 0; ks < FP / 16; ++ks)
+                umma::mma_ss(tG, umma::kmajor_desc(pq0, ks, 128), umma::kmajor_desc(pk0, ks, KT), id_s,
+                             ks > 0 ? 1u : 0u);
+        }
+    };
     if (ntiles > 0 && ok) {
         if (tid < KT) fill_meta(0, meta[0]);
         __syncthreads();
         issue_copies(meta[0], 0);
-    }
-    const int nch = g.NB / 16, split = (nch + 1) / 2;   // O chunks rescaled by half 0 / half 1
-    for (int i = 0; i < ntiles && ok; ++i) {
-        const TileMeta &M = meta[i & 1];
+        if (ntiles > 1 && tid < KT) fill_meta(1, meta[1]);
         umma::cp_async_wait_all();
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
-        const bool lin = (M.lin[0] | M.lin[1]) != 0;
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t q0 = umma::smem_u32(sQ), k0 = umma::smem_u32(base + g.off_K[i & 1]);
-            for (int ks = 0; ks < d / 16; ++ks)
-                umma::mma_ss(tS, umma::kmajor_desc(q0, ks, 128), umma::kmajor_desc(k0, ks, KT), id_s, ks > 0 ? 1u : 0u);
-            if (lin) {
-                const uint32_t pq0 = umma::smem_u32(sPhq), pk0 = umma::smem_u32(sPhk);
-                for (int ks = 0; ks < FP / 16; ++ks)
-                    umma::mma_ss(tG, umma::kmajor_desc(pq0, ks, 128), umma::kmajor_desc(pk0, ks, KT), id_s,
-                                 ks > 0 ? 1u : 0u);
-            }
+            issue_scores(0);
             umma::mma_commit(&mbar);
         }
-        if (i + 1 < ntiles && tid < KT) fill_meta(i + 1, meta[(i + 1) & 1]);
+    }
+    const int nch = g.NB / 16, split = (nch + 1) / 2;   // O chunks rescaled by half 0 / half 1
+    // Per tile i, one completion wait: it covers QK^T(i) and PV(i-1), which were
+    // committed together. Then tile i+1's rows load while tile i's softmax runs, and
+    // PV(i) and QK^T(i+1) go to the tensor cores together.
+    for (int i = 0; i < ntiles && ok; ++i) {
+        const TileMeta &M = meta[i & 1];
         if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
-        // tile i+1 loads while tile i is finished (its phi(K) buffer is free: G is done)
+        // buffers (i+1)&1 held tile i-1, whose MMAs are complete
         if (i + 1 < ntiles) issue_copies(meta[(i + 1) & 1], (i + 1) & 1);
+        const bool lin = (M.lin[0] | M.lin[1]) != 0;
 
         // ---- softmax / linear weights; this half exponentiates keys [32*half, 32*half + 32)
         float sv[KT];
@@ -379,7 +388,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (soft) tmax = fmaxf(tmax, sv[j]);
             }
         }
-        const bool grow_m = tmax > m;
+        // lazy rescaling: the shift m only moves when the row's maximum exceeds it by
+        // more than kLazy (weights stay below e^kLazy; numerator and denominator share m)
+        const bool grow_m = tmax > m + kLazy;
         if (__any_sync(0xffffffffu, grow_m)) {
             // TMEM accesses are warp-collective: the whole warp rescales its chunk range
             const float f = grow_m ? __expf(m - tmax) : 1.f;
@@ -441,6 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             *(uint4 *)(sP + umma::kmajor_offset(r, half * 32 + j0, 128)) = pk;
         }
         lpart += rs;
+        // tile i+1's rows (issued above) have landed; P is written
+        umma::cp_async_wait_all();
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
@@ -449,10 +462,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t p0 = umma::smem_u32(sP), v0 = umma::smem_u32(base + g.off_V[i & 1]);
             for (int ks = 0; ks < KT / 16; ++ks)
                 umma::mma_ss(tO, umma::kmajor_desc(p0, ks, 128), umma::mnmajor_desc(v0, ks, d), id_pv, 1u);
+            if (i + 1 < ntiles) issue_scores(i + 1);
             umma::mma_commit(&mbar);
         }
-        if (!(ok = wait_mbar(&mbar, phase, &okflag, S.err))) break;
+        // meta[i & 1] is free (every thread is past tile i's softmax): tile i+2's metadata
+        if (i + 2 < ntiles && tid < KT) fill_meta(i + 2, meta[i & 1]);
     }
+    // the last PV
+    if (ok && ntiles > 0) ok = wait_mbar(&mbar, phase, &okflag, S.err);
     umma::cp_async_wait_all();
 
     if (ok) {
