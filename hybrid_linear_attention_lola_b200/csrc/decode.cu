@@ -34,6 +34,10 @@ constexpr int kMaxG = 8;
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per staging-buffer wait
 constexpr int kSMs = 148;
 constexpr int kMinPer = 8;   // items per warp of the streaming kernel, at least
+#ifndef LOLA_DECODE_BUFS
+#define LOLA_DECODE_BUFS 2
+#endif
+constexpr int kStreamBufs = LOLA_DECODE_BUFS;   // staging buffers per warp of the streaming kernel
 
 // ---------------------------------------------------------------- shared memory plan
 
@@ -758,7 +762,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     constexpr int KS_ = d / 16;                        // k-steps of Q K^T
     constexpr int ND = d / 8;                          // n-tiles of P V (8 value dims each)
     constexpr int HR = 16;                             // state rows per item
-    constexpr int NST = 3;                             // staging buffers per warp
+    constexpr int NST = kStreamBufs;                   // staging buffers per warp
     constexpr int RS = d * E + 16;                     // padded row stride of key / value tiles (bulk path)
     const bool tma = dm.dec_tma != 0;
     // bytes of a 32-row key (or value) tile: swizzled 128-byte rows (TMA path) or padded rows
@@ -1159,7 +1163,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
 // bytes of shared memory per warp of decode_stream_kernel
 inline int stream_warp_bytes(const Dims &dm, int G)
 {
-    const size_t b = (size_t)3 * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
+    const size_t b = (size_t)kStreamBufs * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
     return (int)((b + 1023) / 1024 * 1024);   // every warp's buffers start 1024-byte aligned
 }
 
@@ -1212,7 +1216,7 @@ bool decode_plan(Dims *dm)
         size_t sb = sb_keys > sb_h ? sb_keys : sb_h;
         if (sb_lin > sb) sb = sb_lin;
         dm->dec_sb = (int)((sb + 1023) / 1024 * 1024);
-        dm->dec_nst = 3;
+        dm->dec_nst = kStreamBufs;
         const int G = dm->g <= 1 ? 1 : dm->g <= 2 ? 2 : dm->g <= 4 ? 4 : 8;
         // warps per CTA: the most resident warps per SM (shared memory, ~160 registers per thread)
         const size_t wb = (size_t)stream_warp_bytes(*dm, G);
