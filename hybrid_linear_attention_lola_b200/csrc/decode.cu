@@ -33,7 +33,7 @@ namespace {
 constexpr int kMaxG = 8;
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per staging-buffer wait
 constexpr int kSMs = 148;
-constexpr int kMinPer = 8;   // items per warp of the streaming kernel, at least
+constexpr int kMinPer = 8;   // items per warp of the streaming kernel, at least (many streams)
 #ifndef LOLA_DECODE_BUFS
 #define LOLA_DECODE_BUFS 2
 #endif
@@ -894,13 +894,39 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             qa0[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + tig * 2) : 0u;
             qa2[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + 8 + tig * 2) : 0u;
         }
-        const float *pg = S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
-        for (int e = lane; e < g * D; e += 32) {
-            const int h = e / D, f = e - h * D;
-            phq[h * PS + qidx<VN>(f)] = pg[e];
+        // 16-byte loads, all issued before any is used (g * D is a multiple of 128)
+        const float4 *pg4 = (const float4 *)(S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D);
+        const int n4 = g * D / 4;
+        for (int e0 = 0; e0 < n4; e0 += 32 * 8) {
+            float4 v4[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int e = e0 + t * 32 + lane;
+                if (e < n4) v4[t] = __ldcg(pg4 + e);
+            }
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                const int e = e0 + t * 32 + lane;
+                if (e < n4) {
+                    const int h = (e * 4) / D, f = e * 4 - h * D;   // 4 features, one 16-byte piece
+                    float *dst = phq + h * PS + qidx<VN>(f);
+                    dst[0] = v4[t].x;
+                    dst[1] = v4[t].y;
+                    dst[2] = v4[t].z;
+                    dst[3] = v4[t].w;
+                }
+            }
         }
         const int nL = (int)(a.L_hi - a.L_lo);
-        for (int i = lane; i < nL; i += 32) fate[i] = S.pend[(size_t)st * dm.Lmax + i];
+        {
+            const uint8_t *pe = S.pend + (size_t)st * dm.Lmax;
+            uint8_t fv[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) fv[t] = t * 32 + lane < nL ? pe[t * 32 + lane] : 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+                if (t * 32 + lane < nL) fate[t * 32 + lane] = fv[t];
+        }
         mrow = 0.f;
         lrow = 0.f;
 #pragma unroll
@@ -953,20 +979,45 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         __threadfence();
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
         for (int h = 0; h < g; ++h) {
+            // lane q holds partials q, q + 32, ...: maximum shift and the scalar sums in parallel
             float M = 0.f;
-            for (int q2 = 0; q2 < nparts; ++q2) M = fmaxf(M, __ldcg(base + ((size_t)q2 * g + h) * rec));
-            float Ls = 0.f, LD = 0.f, O[DPL], LO[DPL];
+            for (int q2 = lane; q2 < nparts; q2 += 32) M = fmaxf(M, __ldcg(base + ((size_t)q2 * g + h) * rec));
+            M = warp_max(M);
+            float Ls = 0.f, LD = 0.f;
+            for (int q2 = lane; q2 < nparts; q2 += 32) {
+                const float *pr = base + ((size_t)q2 * g + h) * rec;
+                Ls = fmaf(__expf(__ldcg(pr) - M), __ldcg(pr + 1), Ls);
+                LD += __ldcg(pr + 2);
+            }
+            Ls = warp_sum(Ls);
+            LD = warp_sum(LD);
+            // value columns: lane owns dims [lane*DPL, lane*DPL + DPL); loads of 4 partials in flight
+            float O[DPL], LO[DPL];
 #pragma unroll
             for (int u = 0; u < DPL; ++u) O[u] = LO[u] = 0.f;
-            for (int q2 = 0; q2 < nparts; ++q2) {
-                const float *pr = base + ((size_t)q2 * g + h) * rec;
-                const float f = __expf(__ldcg(pr) - M);
-                Ls = fmaf(f, __ldcg(pr + 1), Ls);
-                LD += __ldcg(pr + 2);
+            for (int q0 = 0; q0 < nparts; q0 += 4) {
+                float mv[4], ov[4][DPL], lv[4][DPL];
 #pragma unroll
-                for (int u = 0; u < DPL; ++u) {
-                    O[u] = fmaf(f, __ldcg(pr + 4 + lane * DPL + u), O[u]);
-                    LO[u] += __ldcg(pr + 4 + d + lane * DPL + u);
+                for (int t = 0; t < 4; ++t) {
+                    const int q2 = q0 + t < nparts ? q0 + t : q0;
+                    const float *pr = base + ((size_t)q2 * g + h) * rec;
+                    mv[t] = __ldcg(pr);
+#pragma unroll
+                    for (int u = 0; u < DPL; ++u) {
+                        ov[t][u] = __ldcg(pr + 4 + lane * DPL + u);
+                        lv[t][u] = __ldcg(pr + 4 + d + lane * DPL + u);
+                    }
+                }
+#pragma unroll
+                for (int t = 0; t < 4; ++t) {
+                    if (q0 + t < nparts) {
+                        const float f = __expf(mv[t] - M);
+#pragma unroll
+                        for (int u = 0; u < DPL; ++u) {
+                            O[u] = fmaf(f, ov[t][u], O[u]);
+                            LO[u] += lv[t][u];
+                        }
+                    }
                 }
             }
             const float em = __expf(-M);
@@ -1233,9 +1284,15 @@ bool decode_plan(Dims *dm)
             }
         }
         if (dm->dec_nw == 0) return false;
-        const long long nkeys = (long long)dm->lam + dm->eta + 1;
-        const long long items = (nkeys + 31) / 32 + (dm->Cdec + 15) / 16 + dm->D / 16;
-        dm->nsplit = (int)((items + kMinPer - 1) / kMinPer + 1);
+        // aligned 32-row blocks: the cache and up to two more blocks for the window
+        const long long items = ((long long)dm->lam + 31) / 32 + (dm->eta + 31) / 32 + 2 +
+                                (dm->Cdec + 15) / 16 + dm->D / 16;
+        // with few streams every warp takes fewer items, so that the whole GPU streams
+        long long mp = (long long)dm->ns * items / ((long long)kSMs * 8);
+        if (mp < 1) mp = 1;
+        if (mp > kMinPer) mp = kMinPer;
+        dm->dec_minper = (int)mp;
+        dm->nsplit = (int)((items + mp - 1) / mp + 1);
         return true;
     }
     dm->dec_tma = 0;
@@ -1323,7 +1380,7 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
         const long long total = (long long)dm.ns * make_items(dm, a, 16, dm.dec_tma).ni;
         const long long warps_cap = (long long)kSMs * res * nw;
         long long per = (total + warps_cap - 1) / warps_cap;
-        if (per < kMinPer) per = kMinPer;
+        if (per < dm.dec_minper) per = dm.dec_minper;
         const long long nwarps = (total + per - 1) / per;
         const int grid = (int)((nwarps + nw - 1) / nw);
 #define LOLA_STREAM(DPL, GG)                                                                       \

@@ -29,6 +29,7 @@ struct Dims {
     int dec_nst;      // decode: staging buffers per warp
     int dec_sb;       // decode: bytes per staging buffer
     int dec_tma;      // decode (bf16): key/value chunks arrive by tiled TMA loads (128 B swizzle)
+    int dec_minper;   // decode (bf16): fewest work items per warp (fewer for few streams)
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
     float eps;

@@ -74,6 +74,15 @@ WORKLOADS = {
                              head_dim=128, feat_dim=256, window=64, lambda_=2048,
                              chunk=128, decode_interval=64, seq_len=65536,
                              decode_steps=512, dtype="bf16", needles=256),
+    # the pages' own cache setting for the 4K single-needle evaluation (window 256,
+    # sparse cache 256) on the 8B-shaped heads, with planted needles as in prefill-1b
+    "pages-4k": Workload("pages-4k", 6, batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128,
+                         feat_dim=256, window=256, lambda_=256, chunk=64, decode_interval=64,
+                         seq_len=4096, decode_steps=64, dtype="bf16", needles=64),
+    # token-by-token update intervals (C = C_dec = 1)
+    "token-by-token": Workload("token-by-token", 7, batch=2, n_q_heads=4, n_kv_heads=2,
+                               head_dim=64, feat_dim=64, window=16, lambda_=24, chunk=1,
+                               decode_interval=1, seq_len=96, decode_steps=32, dtype="f32"),
 }
 
 

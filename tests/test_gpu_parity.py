@@ -188,3 +188,24 @@ def test_long_context_sampled():
               np.concatenate([vp, vd], 1), None)
     plan = [("prefill", 16384)] * (T // 16384) + [("decode", w.decode_steps)]
     _case(w, plan, forced=True, subset=([0], [3]), qmask_every=251, seed_inputs=inputs)
+
+
+# ---------------------------------------------------------------- next rows: the pages' setting, C = 1
+
+def test_pages_cache_setting_prefill_then_decode():
+    # window 256, sparse cache 256, 4K context with needles, then decode steps
+    w = wl.WORKLOADS["pages-4k"]
+    qp, kp, vp, _ = wl.make_inputs(w, part="prefill")
+    qd, kd, vd, _ = wl.make_inputs(w, part="decode")
+    inputs = (np.concatenate([qp, qd], 1), np.concatenate([kp, kd], 1),
+              np.concatenate([vp, vd], 1), None)
+    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], forced=True, unforced=True,
+                seed_inputs=inputs)
+    assert res["forced"]["exact"] + res["forced"]["under"] == res["forced"]["checked"]
+
+
+def test_token_by_token_intervals():
+    # every token is its own update interval, in prefill (C = 1) and in decode (C_dec = 1)
+    w = wl.WORKLOADS["token-by-token"]
+    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], forced=True, unforced=True)
+    assert res["unforced"]["exact"] == res["unforced"]["checked"]
