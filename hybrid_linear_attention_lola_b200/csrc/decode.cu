@@ -894,39 +894,13 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             qa0[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + tig * 2) : 0u;
             qa2[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + 8 + tig * 2) : 0u;
         }
-        // 16-byte loads, all issued before any is used (g * D is a multiple of 128)
-        const float4 *pg4 = (const float4 *)(S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D);
-        const int n4 = g * D / 4;
-        for (int e0 = 0; e0 < n4; e0 += 32 * 8) {
-            float4 v4[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const int e = e0 + t * 32 + lane;
-                if (e < n4) v4[t] = __ldcg(pg4 + e);
-            }
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                const int e = e0 + t * 32 + lane;
-                if (e < n4) {
-                    const int h = (e * 4) / D, f = e * 4 - h * D;   // 4 features, one 16-byte piece
-                    float *dst = phq + h * PS + qidx<VN>(f);
-                    dst[0] = v4[t].x;
-                    dst[1] = v4[t].y;
-                    dst[2] = v4[t].z;
-                    dst[3] = v4[t].w;
-                }
-            }
+        const float *pg = S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
+        for (int e = lane; e < g * D; e += 32) {
+            const int h = e / D, f = e - h * D;
+            phq[h * PS + qidx<VN>(f)] = pg[e];
         }
         const int nL = (int)(a.L_hi - a.L_lo);
-        {
-            const uint8_t *pe = S.pend + (size_t)st * dm.Lmax;
-            uint8_t fv[8];
-#pragma unroll
-            for (int t = 0; t < 8; ++t) fv[t] = t * 32 + lane < nL ? pe[t * 32 + lane] : 0;
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-                if (t * 32 + lane < nL) fate[t * 32 + lane] = fv[t];
-        }
+        for (int i = lane; i < nL; i += 32) fate[i] = S.pend[(size_t)st * dm.Lmax + i];
         mrow = 0.f;
         lrow = 0.f;
 #pragma unroll
