@@ -31,7 +31,7 @@ constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion w
 struct Geo {
     int D, d, NB, NBa, FP, nblk, lam, Lmax, QC, nbuf;
     uint32_t ncols;
-    size_t off_Bs, off_ones, off_X, off_X1, off_B1, off_part, off_keys, off_rank, off_lst, off_slotTok,
+    size_t off_Bs, off_ones, off_X, off_X1, off_B1, off_part, off_keys, off_keys1, off_rank, off_lst, off_slotTok,
         off_slotVrow, off_free, off_keep, off_flag, off_lf, off_hist, off_scal, total;
 };
 
@@ -70,6 +70,8 @@ __host__ __device__ inline Geo make_geo_n(const Dims &dm, int nbuf)
     o = g.off_part + 128 * 4;
     g.off_keys = al(o, 16);
     o = g.off_keys + (size_t)g.QC * 4;
+    g.off_keys1 = o;                                           // second key buffer (odd intervals)
+    o += (size_t)g.QC * 4;
     g.off_rank = o;
     o += (size_t)g.QC * 4;
     g.off_lst = o;
@@ -327,15 +329,21 @@ __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict_
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    chain_tc_kernel(Dims dm, DevState S, PrefillScratch P, ChainArgs a, KVSrc<bf16> src)
+    chain_tc_kernel(Dims dm, DevState S, PrefillScratch P, ChainArgs a, KVSrc<bf16> src, int nc)
 {
-    const int st = blockIdx.x;
+    // nc > 1: a cluster of nc CTAs per stream; every CTA holds the state and applies the
+    // same folds, the SRE tiles are dealt round-robin, the keys are exchanged through
+    // distributed shared memory, and rank 0 alone writes to global memory
+    const int st = blockIdx.x / nc;
+    const int crank = nc > 1 ? (int)umma::cluster_ctarank() : 0;
+    const bool lead = crank == 0;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const Geo g = make_geo(dm);
     const int D = g.D, d = g.d, lam = g.lam, eta = dm.eta, Lmax = g.Lmax;
 
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar;
+    __shared__ uint64_t kready[2];   // peers' keys of an even / odd interval have arrived
     __shared__ uint32_t tslot;
     __shared__ int okflag;
     const uint32_t raw = umma::smem_u32(smraw);
@@ -346,7 +354,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     c.Bs = base + g.off_Bs;
     c.ones = base + g.off_ones;
     c.X = base + g.off_X;
-    unsigned *keys = (unsigned *)(base + g.off_keys);      // high 32 bits of each candidate's key
+    unsigned *keys0 = (unsigned *)(base + g.off_keys);     // high 32 bits of each candidate's key
+    unsigned *keys1 = (unsigned *)(base + g.off_keys1);    // (two buffers: even / odd intervals)
     int *rank = (int *)(base + g.off_rank);
     int *lst = (int *)(base + g.off_lst);
     int *slotTok = (int *)(base + g.off_slotTok);
@@ -371,11 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         *(bf16 *)(c.ones + umma::kmajor_offset(r, k, 16)) = __float2bfloat16_rn(r == 0 ? 1.f : 0.f);
     }
 
-    if (tid == 0) umma::mbar_init(&mbar, 1);
+    if (tid == 0) {
+        umma::mbar_init(&mbar, 1);
+        umma::mbar_init(&kready[0], nc > 1 ? nc - 1 : 1);
+        umma::mbar_init(&kready[1], nc > 1 ? nc - 1 : 1);
+    }
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
+    if (nc > 1) umma::cluster_sync();   // every peer's barriers exist before anyone arrives
     c.tm = tslot;
 
     float *Hg = S.H + (size_t)st * D * d;
@@ -439,6 +453,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
 
+        unsigned *keys = (ci & 1) ? keys1 : keys0;
         // 2. score the candidates (cache slots, then pairs leaving in [t0, t1))
         const long long Llo = t0 - eta > 0 ? t0 - eta : 0;
         const long long Lhi = t1 - eta > Llo ? t1 - eta : Llo;
@@ -451,10 +466,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         const int lgc = __ffs(g.FP >> 3) - 1;   // 16-byte chunks per phi row (power of two)
         const int ntile = (nQ + 127) / 128;
-        // phi rows of tile t (K-major A operand) into buffer t % nbuf; one cp.async group
-        auto load_tile = [&](int t) {
-            uint8_t *dstT = base + (t % g.nbuf ? g.off_X1 : g.off_X);
-            const int m0 = t * 128, nr = min(128, nQ - m0);
+        const int nmy = ntile > crank ? (ntile - crank + nc - 1) / nc : 0;   // this CTA's tiles
+        // phi rows of this CTA's tile lt (K-major A operand) into buffer lt % nbuf; one cp.async group
+        auto load_tile = [&](int lt) {
+            uint8_t *dstT = base + (lt % g.nbuf ? g.off_X1 : g.off_X);
+            const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
             for (int e = tid; e < (nr << lgc); e += kThreads) {
                 const int r = e >> lgc, kc = e & ((1 << lgc) - 1);
                 uint8_t *dst = dstT + umma::kmajor_offset(r, kc * 8, 128);
@@ -463,21 +479,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             umma::cp_async_commit();
         };
-        if (ntile > 0) load_tile(0);
-        if (g.nbuf == 2 && ntile > 1) load_tile(1);
+        if (nmy > 0) load_tile(0);
+        if (g.nbuf == 2 && nmy > 1) load_tile(1);
         const int q = warp & 3, half = warp >> 2;
         const int r = q * 32 + lane;                      // this thread's row of the tile
         const int hd = d >> 1;                            // value dims per thread
-        for (int t = 0; t < ntile && ok; ++t) {
-            const int m0 = t * 128, nr = min(128, nQ - m0);
-            if (g.nbuf == 2 && t + 1 < ntile) umma::cp_async_wait_1();
+        for (int lt = 0; lt < nmy && ok; ++lt) {
+            const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
+            if (g.nbuf == 2 && lt + 1 < nmy) umma::cp_async_wait_1();
             else umma::cp_async_wait_all();
             umma::fence_async_smem();
             umma::fence_before_sync();
             __syncthreads();
             if (tid == 0) {
                 umma::fence_after_sync();
-                const uint32_t a0 = umma::smem_u32(base + (t % g.nbuf ? g.off_X1 : g.off_X));
+                const uint32_t a0 = umma::smem_u32(base + (lt % g.nbuf ? g.off_X1 : g.off_X));
                 const uint32_t bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
                 for (int ks = 0; ks < g.FP / 16; ++ks) {
                     const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
@@ -495,8 +511,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (i * 8 < hd) vr4[i] = vsrc[i];
             }
             if (!(ok = wait_mma(c))) break;
-            if (g.nbuf == 1 && t + 1 < ntile) load_tile(t + 1);         // the tile buffer is free
-            if (g.nbuf == 2 && t + 2 < ntile) load_tile(t + 2);
+            if (g.nbuf == 1 && lt + 1 < nmy) load_tile(lt + 1);         // the tile buffer is free
+            if (g.nbuf == 2 && lt + 2 < nmy) load_tile(lt + 2);
             {
                 const uint32_t rowaddr = tS(c) + ((uint32_t)(q * 32) << 16);
                 float v[16];
@@ -531,6 +547,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
         if (!ok) break;
+        if (nc > 1) {
+            // push this CTA's keys into every peer's buffer, then signal it; wait for theirs
+            for (int pr = 1; pr < nc; ++pr) {
+                const uint32_t peer = (uint32_t)((crank + pr) % nc);
+                const uint32_t rk = umma::cluster_map(keys, peer);
+                for (int lt = 0; lt < nmy; ++lt) {
+                    const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
+                    for (int i = tid; i < nr; i += kThreads)
+                        umma::st_cluster_u32(rk + (uint32_t)(m0 + i) * 4u, keys[m0 + i]);
+                }
+            }
+            __syncthreads();
+            if (tid == 0) {
+                umma::fence_cluster();
+                for (int pr = 1; pr < nc; ++pr)
+                    umma::mbar_arrive_cluster(umma::cluster_map(&kready[ci & 1], (uint32_t)((crank + pr) % nc)));
+                const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
+                const bool got = !aborted && umma::mbar_wait_cluster(&kready[ci & 1], (uint32_t)((ci >> 1) & 1), kWaitNs);
+                if (!got) raise_error(S.err, ERR_TIMEOUT);
+                okflag = got ? 1 : 0;
+            }
+            __syncthreads();
+            if (!(ok = okflag != 0)) break;
+        }
 
         // 3. keep the nK smallest keys (highest SRE, lower token on ties)
         const int nK = nQ < lam ? nQ : lam;
@@ -545,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = tid; i < nQ; i += kThreads) keep[i] = 1;
         }
         __syncthreads();
-        if (a.sel_log != nullptr && iglob < a.sel_cap) {
+        if (a.sel_log != nullptr && iglob < a.sel_cap && lead) {
             int32_t *lg = a.sel_log + ((size_t)iglob * dm.ns + st) * (lam + 1);
             const int cnt = scan_excl(keep, rank, nQ, scal);
             for (int i = tid; i < nQ; i += kThreads)
@@ -586,12 +626,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!(ok = fold_tc(c, lst, nE, phi_st, src, st))) break;
             refresh_image(c);
         }
-        if (a.mode == 0 && P.snapImg != nullptr && tid == 0) {
+        if (a.mode == 0 && P.snapImg != nullptr && tid == 0 && lead) {
             // the image (written and proxy-fenced by refresh_image) goes out as one bulk store
             uint8_t *dst = (uint8_t *)P.snapImg + ((size_t)st * dm.mmax + a.ci0 + ci) * g.NB * g.FP * 2;
             umma::bulk_s2g(dst, c.Bimg, (uint32_t)(g.NB * g.FP * 2));
         }
-        if (a.mode == 0 && a.snap_f32) {
+        if (a.mode == 0 && a.snap_f32 && lead) {
             // fp32 (H', s') for the SIMT attention kernel
             const int q = warp & 3;
             float *sh = P.snapH + ((size_t)st * dm.mmax + a.ci0 + ci) * D * d;
@@ -644,7 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
         }
         __syncthreads();
-        if (a.mode == 0) {
+        if (a.mode == 0 && lead) {
             const size_t lb = (size_t)st * dm.mmax + a.ci0 + ci;
             for (int i = tid; i < nK; i += kThreads) {
                 P.logTok[lb * lam + i] = slotTok[i];
@@ -662,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
     }
 
-    if (ok) {
+    if (ok && lead) {
         // TMEM -> state
         const int q = warp & 3;
         for (int bk = warp >> 2; bk < g.nblk; bk += kThreads / 128) {
@@ -688,7 +728,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 P.slotVrow[(size_t)st * lam + i] = slotVrow[i];
             }
         }
-    } else {
+    } else if (!ok) {
         if (tid == 0) {
             raise_error(S.err, ERR_TIMEOUT);
             umma::mbar_wait(&mbar, c.phase ^ 1u, kWaitNs);  // let an MMA still in flight drain
@@ -698,6 +738,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma::fence_before_sync();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(c.tm, g.ncols);
+    // no CTA leaves while a peer may still write into its shared memory (every CTA gets
+    // here: all waits above are bounded)
+    if (nc > 1) umma::cluster_sync();
 }
 
 }  // namespace
@@ -720,7 +763,32 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     cudaFuncSetAttribute(chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     PrefillScratch Pv{};
     if (P) Pv = *P;
-    chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src);
+    // prefill with few streams: a cluster of up to 4 CTAs per stream shares the scoring
+    // (at most 32 CTAs, so that the attention keeps the other SMs)
+    int nc = 1;
+    if (a.mode == 0) {
+        nc = 32 / dm.ns;
+        if (nc > 4) nc = 4;
+        if (nc < 1) nc = 1;
+        if (nc == 3) nc = 2;
+    }
+    if (nc == 1) {
+        chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src, 1);
+        return;
+    }
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)(dm.ns * nc), 1, 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)nc;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, chain_tc_kernel, dm, S, Pv, a, src, nc);
 }
 
 }  // namespace lola
