@@ -374,9 +374,9 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->seg_len = 0;
     st->chain_stream = nullptr;
     if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
-        // segments of at least 4 intervals, at most kMaxSeg of them per call
+        // segments of at least 8 intervals, at most kMaxSeg of them per call
         int len = dm.mmax / 32;
-        if (len < 4) len = 4;
+        if (len < 8) len = 8;
         while ((dm.mmax + len - 1) / len > lola_state::kMaxSeg) ++len;
         int lo = 0, hi = 0;
         bool okc = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&

@@ -247,11 +247,16 @@ __device__ void refresh_image(Ctx &c)
     // the last snapshot store must have read the image before it is overwritten
     if (threadIdx.x == 0) umma::bulk_wait_read();
     __syncthreads();
-    for (int bk = warp >> 2; bk < c.g.nblk; bk += kThreads / 128) {
+    // units of (feature block, 16-column piece or the s column), dealt to the two
+    // groups of four warps; warp w reads TMEM lanes 32 * (w % 4) ..
+    const int npc = c.g.d / 16 + 1;
+    for (int u = warp >> 2; u < c.g.nblk * npc; u += kThreads / 128) {
+        const int bk = u / npc, cc = u - bk * npc;
         const int f = bk * 128 + q * 32 + lane;
         const uint32_t row = tH(c, bk) + ((uint32_t)(q * 32) << 16);
-        for (int c0 = 0; c0 < c.g.d; c0 += 16) {
-            float v[16];
+        float v[16];
+        if (cc * 16 < c.g.d) {
+            const int c0 = cc * 16;
             umma::tmem_ld16(row + (uint32_t)c0, v);
             umma::tmem_wait_ld();
             uint4 h0, h1;
@@ -265,11 +270,11 @@ __device__ void refresh_image(Ctx &c)
             h1.w = umma::pack_bf16x2(v[14], v[15]);
             *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0, c.g.d)) = h0;
             *(uint4 *)(c.Bimg + umma::mnmajor_offset(f, c0 + 8, c.g.d)) = h1;
+        } else {
+            umma::tmem_ld16(row + (uint32_t)c.g.d, v);
+            umma::tmem_wait_ld();
+            *(bf16 *)(c.Bs + umma::kmajor_offset(0, f, 16)) = __float2bfloat16_rn(v[0]);
         }
-        float v[16];
-        umma::tmem_ld16(row + (uint32_t)c.g.d, v);
-        umma::tmem_wait_ld();
-        *(bf16 *)(c.Bs + umma::kmajor_offset(0, f, 16)) = __float2bfloat16_rn(v[0]);
     }
     umma::fence_async_smem();
     umma::fence_before_sync();
@@ -763,14 +768,15 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     cudaFuncSetAttribute(chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     PrefillScratch Pv{};
     if (P) Pv = *P;
-    // prefill with few streams: a cluster of up to 4 CTAs per stream shares the scoring
-    // (at most 32 CTAs, so that the attention keeps the other SMs)
+    // prefill with few streams: a cluster of up to 8 CTAs per stream shares the scoring,
+    // one SRE tile each (at most about 40 CTAs, so that the attention keeps the other SMs)
     int nc = 1;
     if (a.mode == 0) {
-        nc = 32 / dm.ns;
-        if (nc > 4) nc = 4;
+        const int tiles = (dm.lam + dm.C + 127) / 128;   // SRE tiles of a full interval
+        nc = 40 / dm.ns;                                  // at most about 40 CTAs
+        if (nc > tiles) nc = tiles;
+        if (nc > 8) nc = 8;
         if (nc < 1) nc = 1;
-        if (nc == 3) nc = 2;
     }
     if (nc == 1) {
         chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src, 1);
