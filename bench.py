@@ -31,6 +31,9 @@ from hybrid_linear_attention_lola_b200 import workloads as wl  # noqa: E402
 METRIC = "LoLA prefill & decode tokens/sec on 1xB200; % of tensor/HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# DRAM bytes (read + write) per call of the dominant kernel, from one ncu capture of the
+# current kernel (profiles/chain_tc_prefill-1b.md); None where no capture matches.
+MEASURED_TRAFFIC = {("prefill-1b", "chain"): 27.35e6}
 
 
 # ---------------------------------------------------------------- helpers
@@ -295,7 +298,8 @@ def run_engine(args, ws, rank, local):
     achieved = fl[dom] / (cand[dom] / 1e3) / 1e12
     peak = float(peaks["bf16_tflops"])
     roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 3), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 5), "traffic": None,
+                "unit": "TFLOP/s", "frac": round(achieved / peak, 5),
+                "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
                 "peak_source": f"{peak_src} bf16 dense (burst)",
                 "phase_ms": {ph: round(v[0] / args.steps, 4) for ph, v in phase_ms.items()
                              if v[1]},
