@@ -781,7 +781,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     const long long i0 = gw * per;
     if (i0 >= total) return;                            // warp-uniform; no CTA-wide barriers below
     const int nmine = (int)min((long long)per, total - i0);
-    const int PS = D + D / 8;                           // padded phi(q) row (floats)
+    const int PS = D;                                   // phi(q) row stride (floats; plain rows)
     const int CPD = D / VN;
     const int XMD = CPD >= 16 ? 7 : (CPD >> 1) - 1;
     const float scale = rsqrtf((float)d);
@@ -791,10 +791,10 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     uint8_t *smd = smraw_d + (((umma::smem_u32(smraw_d) + 1023u) & ~1023u) - umma::smem_u32(smraw_d));
     uint8_t *wbase = smd + (size_t)warp * wbytes;
     uint8_t *ring = wbase;
-    float *phq = (float *)(wbase + NST * SB);            // [G][PS]
+    float *phq = (float *)(wbase + NST * SB);            // [G][D], filled by a bulk copy per stream
     float *pws = phq + G * PS;                           // [G][32]
     uint8_t *fate = (uint8_t *)(pws + G * 32);           // [Lmax]
-    uint64_t *mb = (uint64_t *)(fate + 256);             // [NST]
+    uint64_t *mb = (uint64_t *)(fate + 256);             // [NST] staging buffers, [NST] phi(q)
 
     // ---- copies of item k of this warp into buffer s: bulk (TMA) copies, completion
     //      counted on the buffer's mbarrier. Key chunks: one copy per key row and per
@@ -875,12 +875,14 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         }
     };
     if (lane == 0)
-        for (int i = 0; i < NST; ++i) umma::mbar_init(&mb[i], 1);
+        for (int i = 0; i <= NST; ++i) umma::mbar_init(&mb[i], 1);
     __syncwarp();
     for (int k = 0; k < NST; ++k) issue(k, k);
 
     // ---- per-stream state of this warp
     int cur = -1;
+    uint32_t nbeg = 0;      // streams begun (phase of the phi(q) barrier)
+    bool need_q = false;    // phi(q) of the current stream not yet waited for
     uint32_t qa0[KS_], qa2[KS_];
     float mrow = 0.f, lrow = 0.f;
     float oc[ND][4];
@@ -894,11 +896,18 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             qa0[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + tig * 2) : 0u;
             qa2[ks] = hv ? *(const uint32_t *)(qg + (size_t)gq * d + ks * 16 + 8 + tig * 2) : 0u;
         }
-        const float *pg = S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D;
-        for (int e = lane; e < g * D; e += 32) {
-            const int h = e / D, f = e - h * D;
-            phq[h * PS + qidx<VN>(f)] = pg[e];
+        // phi(q) of the group's heads: one bulk copy, waited for before the first
+        // linear-band or state item of the stream (key chunks come first)
+        fence_proxy_async();   // earlier reads of phq are done before the copy overwrites it
+        __syncwarp();
+        if (lane == 0) {
+            // a copy whose stream needed no phi(q) lands before the next one is issued
+            if (need_q) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
+            umma::mbar_arrive_expect_tx(&mb[NST], (uint32_t)(g * D * 4));
+            umma::bulk_g2s(phq, S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D, (uint32_t)(g * D * 4), &mb[NST]);
         }
+        ++nbeg;
+        need_q = true;
         const int nL = (int)(a.L_hi - a.L_lo);
         for (int i = lane; i < nL; i += 32) fate[i] = S.pend[(size_t)st * dm.Lmax + i];
         mrow = 0.f;
@@ -943,14 +952,15 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                 for (int u = 0; u < DPL; ++u) pr[4 + d + lane * DPL + u] = lo[h][u];
             }
         }
-        __threadfence();
+        // publish the partial (release) and count it; the last one acquires all the others
         __syncwarp();
         int prev = 0;
-        if (lane == 0) prev = atomicAdd(&S.dec_cnt[st], 1);
+        if (lane == 0)
+            asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(prev) : "l"(&S.dec_cnt[st]) : "memory");
         prev = __shfl_sync(0xffffffffu, prev, 0);
+        __syncwarp();
         if (prev != nparts - 1) return;
         // this warp wrote the stream's last partial: merge (online-softmax identity) and write out
-        __threadfence();
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
         for (int h = 0; h < g; ++h) {
             // lane q holds partials q, q + 32, ...: maximum shift and the scalar sums in parallel
@@ -1026,6 +1036,15 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             return;
         }
         const uint8_t *buf = ring + (size_t)s * SB;
+        if (it >= IT.nkc && need_q) {
+            bool okq = true;
+            if (lane == 0) {
+                okq = umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
+                if (!okq) raise_error(S.err, ERR_TIMEOUT);
+            }
+            if (__shfl_sync(0xffffffffu, okq ? 1 : 0, 0) == 0) return;
+            need_q = false;
+        }
         if (it < IT.nkc) {
             bool soft;
             long long j = -1;   // window token of this lane's row, if any
@@ -1119,7 +1138,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
 #pragma unroll
                     for (int h = 0; h < G; ++h) {
                         if (h < g) {
-                            const float *ph = phq + h * PS + qoff<VN>(c2, 0);
+                            const float *ph = phq + h * PS + c2 * VN;
 #pragma unroll
                             for (int u = 0; u < VN; u += 4) {
                                 const float4 q4 = *(const float4 *)(ph + u);
@@ -1166,7 +1185,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
 #pragma unroll
                 for (int u = 0; u < DPL; ++u) hv[u] = Hs[i * d + lane * DPL + u];
                 const float si = ss[i];
-                const int fi = qidx<VN>(r0 + i);
+                const int fi = r0 + i;
 #pragma unroll
                 for (int h = 0; h < G; ++h) {
                     if (h < g) {
@@ -1183,6 +1202,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         issue(k + NST, s);
     }
     flush(cur);
+    if (need_q && lane == 0) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);   // no copy outlives the warp
 }
 
 // bytes of shared memory per warp of decode_stream_kernel
