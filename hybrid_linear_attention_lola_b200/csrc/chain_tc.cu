@@ -27,6 +27,9 @@ using bf16 = __nv_bfloat16;
 constexpr int kThreads = 256;
 constexpr int kFoldTok = 64;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
+#ifndef LOLA_CHAIN_CTAS
+#define LOLA_CHAIN_CTAS 40   // CTAs a prefill chain may spread over (the attention keeps the rest)
+#endif
 
 struct Geo {
     int D, d, NB, NBa, FP, nblk, lam, Lmax, QC, nbuf;
@@ -228,8 +231,7 @@ __device__ __forceinline__ uint32_t tS(const Ctx &c) { return c.tm + (uint32_t)(
 __device__ bool wait_mma(Ctx &c)
 {
     if (threadIdx.x == 0) {
-        const bool aborted = (*(volatile int *)c.err & ERR_TIMEOUT) != 0;
-        const bool ok = !aborted && umma::mbar_wait(c.mbar, c.phase, kWaitNs);
+        const bool ok = umma::mbar_wait_abortable(c.mbar, c.phase, kWaitNs, c.err, ERR_TIMEOUT);
         if (!ok) raise_error(c.err, ERR_TIMEOUT);
         *c.okflag = ok ? 1 : 0;
     }
@@ -568,8 +570,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::fence_cluster();
                 for (int pr = 1; pr < nc; ++pr)
                     umma::mbar_arrive_cluster(umma::cluster_map(&kready[ci & 1], (uint32_t)((crank + pr) % nc)));
-                const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
-                const bool got = !aborted && umma::mbar_wait_cluster(&kready[ci & 1], (uint32_t)((ci >> 1) & 1), kWaitNs);
+                const bool got = umma::mbar_wait_cluster_abortable(&kready[ci & 1], (uint32_t)((ci >> 1) & 1), kWaitNs,
+                                                                   S.err, ERR_TIMEOUT);
                 if (!got) raise_error(S.err, ERR_TIMEOUT);
                 okflag = got ? 1 : 0;
             }
@@ -769,11 +771,11 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     PrefillScratch Pv{};
     if (P) Pv = *P;
     // prefill with few streams: a cluster of up to 8 CTAs per stream shares the scoring,
-    // one SRE tile each (at most about 40 CTAs, so that the attention keeps the other SMs)
+    // one SRE tile each (at most LOLA_CHAIN_CTAS CTAs, so that the attention keeps the other SMs)
     int nc = 1;
     if (a.mode == 0) {
         const int tiles = (dm.lam + dm.C + 127) / 128;   // SRE tiles of a full interval
-        nc = 40 / dm.ns;                                  // at most about 40 CTAs
+        nc = LOLA_CHAIN_CTAS / dm.ns;
         if (nc > tiles) nc = tiles;
         if (nc > 8) nc = 8;
         if (nc < 1) nc = 1;

@@ -374,8 +374,7 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
         const uint32_t par = (uint32_t)((k / nst) & 1);
         bool got = true;
         if (lane == 0) {
-            const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
-            got = !aborted && umma::mbar_wait(&mb[s], par, kWaitNs);
+            got = umma::mbar_wait_abortable(&mb[s], par, kWaitNs, S.err, ERR_TIMEOUT);
             if (!got) raise_error(S.err, ERR_TIMEOUT);
         }
         got = __shfl_sync(0xffffffffu, got ? 1 : 0, 0) != 0;
@@ -1024,15 +1023,17 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         }
         bool got = true;
         if (lane == 0) {
-            const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
-            got = !aborted && umma::mbar_wait(&mb[s], (uint32_t)((k / NST) & 1), kWaitNs);
+            got = umma::mbar_wait_abortable(&mb[s], (uint32_t)((k / NST) & 1), kWaitNs, S.err, ERR_TIMEOUT);
             if (!got) raise_error(S.err, ERR_TIMEOUT);
         }
         if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
-            // give up on the step (the error word is set): let copies in flight land
-            if (lane == 0)
-                for (int k2 = k + 1; k2 < k + NST && k2 < nmine; ++k2)
+            // give up on the step (the error word is set): let copies in flight land,
+            // this item's included (an abort does not wait for it)
+            if (lane == 0) {
+                for (int k2 = k; k2 < k + NST && k2 < nmine; ++k2)
                     umma::mbar_wait(&mb[k2 % NST], (uint32_t)((k2 / NST) & 1), kWaitNs);
+                if (need_q) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
+            }
             return;
         }
         const uint8_t *buf = ring + (size_t)s * SB;

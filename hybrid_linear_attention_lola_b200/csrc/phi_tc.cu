@@ -131,8 +131,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::mma_ss(tz, umma::kmajor_desc(x0, ks, 128), umma::kmajor_desc(w0, ks, Dh), idesc,
                              ks > 0 ? 1u : 0u);
             umma::mma_commit(&mbar);
-            const bool aborted = (*(volatile int *)S.err & ERR_TIMEOUT) != 0;
-            const bool fine = !aborted && umma::mbar_wait(&mbar, phase, kWaitNs);
+            const bool fine = umma::mbar_wait_abortable(&mbar, phase, kWaitNs, S.err, ERR_TIMEOUT);
             if (!fine) raise_error(S.err, ERR_TIMEOUT);
             okflag = fine ? 1 : 0;
         }

@@ -142,6 +142,23 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
 }
+// 32 lanes x 32 consecutive fp32 columns
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
+{
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+          "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+          "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
 __device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 lanes x 16 columns store (thread t writes lane lane_base + t).
@@ -193,6 +210,31 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint6
         if (done) return true;
         if (globaltimer_ns() - start > limit_ns) return false;
     }
+}
+
+// One non-blocking probe of an mbarrier phase (acquire, CTA scope).
+__device__ __forceinline__ bool mbar_test(uint64_t *mbar, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(mbar)), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// As mbar_wait, but gives up at once when *err already holds a bit of abort_mask
+// (another thread of the grid gave up). The error word, a global read, is only
+// consulted when the phase is not complete at the first probe.
+__device__ __forceinline__ bool mbar_wait_abortable(uint64_t *mbar, uint32_t parity, uint64_t limit_ns,
+                                                    const int *err, int abort_mask)
+{
+    if (mbar_test(mbar, parity)) return true;
+    if ((*(const volatile int *)err & abort_mask) != 0) return false;
+    return mbar_wait(mbar, parity, limit_ns);
 }
 
 // Expects `bytes` more transaction bytes on the mbarrier and arrives once.
@@ -280,6 +322,23 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *mbar, uint32_t parit
         if (globaltimer_ns() - start > limit_ns) return false;
     }
 }
+// mbar_wait_cluster that gives up at once when *err holds a bit of abort_mask; the
+// error word is only read when the phase is not complete at the first probe
+__device__ __forceinline__ bool mbar_wait_cluster_abortable(uint64_t *mbar, uint32_t parity, uint64_t limit_ns,
+                                                            const int *err, int abort_mask)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(smem_u32(mbar)), "r"(parity)
+        : "memory");
+    if (done) return true;
+    if ((*(const volatile int *)err & abort_mask) != 0) return false;
+    return mbar_wait_cluster(mbar, parity, limit_ns);
+}
 // full cluster barrier (every thread of every CTA of the cluster)
 __device__ __forceinline__ void cluster_sync()
 {
@@ -287,6 +346,14 @@ __device__ __forceinline__ void cluster_sync()
     asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
+
+// 2^x by the hardware approximation (ex2.approx, flush-to-zero)
+__device__ __forceinline__ float ex2_approx(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 // Two fp32 -> one register holding two bf16 (round to nearest even); lo in bits 0..15.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
