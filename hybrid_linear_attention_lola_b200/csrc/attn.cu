@@ -248,59 +248,69 @@ size_t attn_smem(const Dims &dm)
 
 // ---------------------------------------------------------------- finalize
 
+// One copy unit of a key/value row: 16 bytes when the row is a whole number of them.
+template <typename T> __device__ __forceinline__ int row_vec(int d)
+{
+    return (d * (int)sizeof(T)) % 16 == 0 ? 16 / (int)sizeof(T) : 1;
+}
+template <typename T> __device__ __forceinline__ void copy_unit(T *dst, const T *src, int vec)
+{
+    if (vec * sizeof(T) == 16) *(uint4 *)dst = *(const uint4 *)src;
+    else for (int k = 0; k < vec; ++k) dst[k] = src[k];
+}
+
+// Cache slot i <- its pair's key/value row (from the window ring or this call's input),
+// idxS <- its token; one thread per (stream, slot, copy unit) over the whole grid.
 template <typename T>
 __global__ void finalize_cache_kernel(Dims dm, DevState S, PrefillScratch P, KVSrc<T> src, int nK)
 {
-    const int st = blockIdx.x;
     const int lam = dm.lam, d = dm.d;
-    T *KS = (T *)S.KS + (size_t)st * lam * d;
-    T *VS = (T *)S.VS + (size_t)st * lam * d;
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-    for (int i = warp; i < lam; i += nw) {
+    const int vec = row_vec<T>(d), upr = d / vec;
+    const long long total = (long long)dm.ns * lam * upr;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int u = (int)(e % upr);
+        const long long rs = e / upr;
+        const int i = (int)(rs % lam), st = (int)(rs / lam);
+        const size_t slot = (size_t)st * lam + i;
         if (i >= nK) {
-            if (lane == 0) S.idxS[(size_t)st * lam + i] = -1;
+            if (u == 0) S.idxS[slot] = -1;
             continue;
         }
-        const int vr = P.slotVrow[(size_t)st * lam + i];
+        const int vr = P.slotVrow[slot];
         if (vr >= lam) {
-            const T *kr = src.krow(st, vr);
-            const T *vv = src.vrow(st, vr);
-            for (int c = lane; c < d; c += 32) {
-                KS[(size_t)i * d + c] = kr[c];
-                VS[(size_t)i * d + c] = vv[c];
-            }
-        } else if (vr != i && lane == 0) {
+            copy_unit((T *)S.KS + slot * d + u * vec, src.krow(st, vr) + u * vec, vec);
+            copy_unit((T *)S.VS + slot * d + u * vec, src.vrow(st, vr) + u * vec, vec);
+        } else if (vr != i && u == 0) {
             raise_error(S.err, ERR_BOUNDS);
         }
-        if (lane == 0) S.idxS[(size_t)st * lam + i] = P.slotTok[(size_t)st * lam + i];
+        if (u == 0) S.idxS[slot] = P.slotTok[slot];
     }
 }
 
-// Ring slot (token mod R) <- the call's last min(n, R) tokens.
+// Ring slot (token mod R) <- the call's last min(n, R) tokens; one thread per copy unit.
 template <typename T>
 __global__ void ring_update_kernel(Dims dm, DevState S, const T *__restrict__ kin,
                                    const T *__restrict__ vin, long long call_start, int n)
 {
     const int first = n > dm.R ? n - dm.R : 0;
     const int cnt = n - first;
-    const long long total = (long long)cnt * dm.ns;
-    const int warps = blockDim.x >> 5, lane = threadIdx.x & 31;
+    const int vec = row_vec<T>(dm.d), upr = dm.d / vec;
+    const long long total = (long long)cnt * dm.ns * upr;
     T *KR = (T *)S.KR, *VR = (T *)S.VR;
-    for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < total;
-         r += (long long)gridDim.x * warps) {
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (long long)gridDim.x * blockDim.x) {
+        const int u = (int)(e % upr);
+        const long long r = e / upr;
         const int st = (int)(r % dm.ns);
         const int t = first + (int)(r / dm.ns);
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
         const long long tok = call_start + t;
         const int slot = (int)(tok & (dm.R - 1));
-        const T *ks = kin + (((size_t)b * n + t) * dm.Hkv + hk) * dm.d;
-        const T *vs = vin + (((size_t)b * n + t) * dm.Hkv + hk) * dm.d;
-        T *kd = KR + ((size_t)st * dm.R + slot) * dm.d;
-        T *vd = VR + ((size_t)st * dm.R + slot) * dm.d;
-        for (int c = lane; c < dm.d; c += 32) {
-            kd[c] = ks[c];
-            vd[c] = vs[c];
-        }
+        const size_t so = (((size_t)b * n + t) * dm.Hkv + hk) * dm.d + (size_t)u * vec;
+        const size_t dof = ((size_t)st * dm.R + slot) * dm.d + (size_t)u * vec;
+        copy_unit(KR + dof, kin + so, vec);
+        copy_unit(VR + dof, vin + so, vec);
     }
 }
 
@@ -337,19 +347,24 @@ void launch_finalize_prefill(const Dims &dm, const DevState &S, const PrefillScr
                              const void *kin, const void *vin, long long call_start, int n,
                              int nK, cudaStream_t stream)
 {
-    const long long rows = (long long)(n > dm.R ? dm.R : n) * dm.ns;
-    long long g = (rows + 7) / 8;
-    if (g > 148 * 8) g = 148 * 8;
-    if (g < 1) g = 1;
+    auto blocks = [](long long units) {
+        long long g = (units + 255) / 256;
+        if (g > 148 * 8) g = 148 * 8;
+        return (int)(g < 1 ? 1 : g);
+    };
+    // upper bounds of the copy units (one per element when rows are not whole 16-byte units)
+    const long long ring_units = (long long)(n > dm.R ? dm.R : n) * dm.ns * dm.d;
+    const long long cache_units = (long long)dm.ns * dm.lam * dm.d;
+    const int g = blocks(ring_units / 4 + 1), gc = blocks(cache_units / 4 + 1);
     if (dm.dtype == 0) {
-        finalize_cache_kernel<float><<<dm.ns, 256, 0, stream>>>(
+        finalize_cache_kernel<float><<<gc, 256, 0, stream>>>(
             dm, S, P, make_src<float>(dm, S, kin, vin, call_start, n), nK);
-        ring_update_kernel<float><<<(int)g, 256, 0, stream>>>(dm, S, (const float *)kin,
+        ring_update_kernel<float><<<g, 256, 0, stream>>>(dm, S, (const float *)kin,
                                                               (const float *)vin, call_start, n);
     } else {
-        finalize_cache_kernel<__nv_bfloat16><<<dm.ns, 256, 0, stream>>>(
+        finalize_cache_kernel<__nv_bfloat16><<<gc, 256, 0, stream>>>(
             dm, S, P, make_src<__nv_bfloat16>(dm, S, kin, vin, call_start, n), nK);
-        ring_update_kernel<__nv_bfloat16><<<(int)g, 256, 0, stream>>>(
+        ring_update_kernel<__nv_bfloat16><<<g, 256, 0, stream>>>(
             dm, S, (const __nv_bfloat16 *)kin, (const __nv_bfloat16 *)vin, call_start, n);
     }
 }

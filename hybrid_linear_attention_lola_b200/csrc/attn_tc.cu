@@ -43,7 +43,15 @@ enum : int { INFO_SOFT = 0, INFO_FOLDED = 1, INFO_SKIP = 2 };
 struct TileMeta {
     int tok[KT], vrow[KT];
     unsigned char info[KT];
+    unsigned skip32[2], fold32[2];   // per 32 keys: never a softmax key here / a folded leaving pair
+    int maxtok32[2];                 // per 32 keys: largest token of a key that is not skipped
 };
+
+// bits 0..x set (none for x < 0, all for x >= 63)
+__device__ __forceinline__ unsigned long long prefix_mask(long long x)
+{
+    return x < 0 ? 0ull : x >= 63 ? ~0ull : (2ull << x) - 1ull;
+}
 
 // Shared memory: [Q][ones][P region][ring region][tile metadata][row sums]
 //   P region: two 128 x 64 weight tiles (P0, P1); during setup W^T, then phi(K_L)
@@ -181,7 +189,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int grow = mt * 128 + r;
     const bool row_ok = grow < rows_total;
     const long long p = t0 + grow / gq;              // query position of the row
-    const long long pmin = t0 + (mt * 128) / gq;     // smallest position in the CTA
     const float scale = rsqrtf((float)d);
     const int lgd = __ffs(d >> 3) - 1, lgf = __ffs(FP >> 3) - 1;   // 16-byte chunks per row
 
@@ -478,11 +485,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     };
     auto meta_store = [&](int t, int tok, int vr, int info) {
-        if (tid < KT) {
+        if (tid < KT) {   // warps 0 and 1, one key per thread
             TileMeta &M = meta[t % MS];
             M.tok[tid] = tok;
             M.vrow[tid] = vr;
             M.info[tid] = (unsigned char)info;
+            const unsigned sk = __ballot_sync(0xffffffffu, info == INFO_SKIP);
+            const unsigned fo = __ballot_sync(0xffffffffu, info == INFO_FOLDED);
+            const int mx = __reduce_max_sync(0xffffffffu, info == INFO_SKIP ? (int)0x80000000 : tok);
+            if (lane == 0) {
+                M.skip32[warp] = sk;
+                M.fold32[warp] = fo;
+                M.maxtok32[warp] = mx;
+            }
         }
     };
     // key rows of tile t into its K buffer (no commit); its metadata is in shared memory
@@ -582,21 +597,41 @@ __global__ void __launch_bounds__(kThreads, 1)
                 sv[32 + j] = v1[j];
             }
         }
-        // every key of the tile a causal softmax key for every row of the CTA
-        const bool fast = __all_sync(0xffffffffu, M.info[lane] == INFO_SOFT && (long long)M.tok[lane] <= pmin &&
-                                                      M.info[lane + 32] == INFO_SOFT &&
-                                                      (long long)M.tok[lane + 32] <= pmin);
-        float tmax = -INFINITY;
-        if (fast) {
-#pragma unroll
-            for (int j = 0; j < KT; ++j) tmax = fmaxf(tmax, sv[j]);
+        // live keys of this row (softmax keys it may see), one bit per key
+        const unsigned long long skipm = (unsigned long long)M.skip32[0] | ((unsigned long long)M.skip32[1] << 32);
+        unsigned long long live;
+        if (i < ntb) {
+            // window tile: token = kb + j; a folded pair is a softmax key only inside the window
+            const long long kb = jL0 + (long long)i * KT;
+            const unsigned long long foldm =
+                (unsigned long long)M.fold32[0] | ((unsigned long long)M.fold32[1] << 32);
+            live = ~skipm & prefix_mask(p - kb) & ~(foldm & prefix_mask(p - eta - kb));
+        } else if ((long long)max(M.maxtok32[0], M.maxtok32[1]) <= p) {
+            live = ~skipm;   // cached keys, all causal for this row
         } else {
+            live = 0;
+            for (int j = 0; j < KT; ++j)
+                if (!((skipm >> j) & 1ull) && (long long)M.tok[j] <= p) live |= 1ull << j;
+        }
+        if (!row_ok) live = 0;
+        const bool all_live = __all_sync(0xffffffffu, live == ~0ull);
+        float tmax;
+        {
+            float t[32];
+            if (all_live) {
 #pragma unroll
-            for (int j = 0; j < KT; ++j) {
-                const int info = M.info[j], tok = M.tok[j];
-                const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
-                if (soft) tmax = fmaxf(tmax, sv[j]);
+                for (int j = 0; j < 32; ++j) t[j] = fmaxf(sv[j], sv[j + 32]);
+            } else {
+                const uint32_t lo = (uint32_t)live, hi = (uint32_t)(live >> 32);
+#pragma unroll
+                for (int j = 0; j < 32; ++j)
+                    t[j] = fmaxf((lo >> j) & 1u ? sv[j] : -INFINITY, (hi >> j) & 1u ? sv[j + 32] : -INFINITY);
             }
+#pragma unroll
+            for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+                for (int j = 0; j < w; ++j) t[j] = fmaxf(t[j], t[j + w]);
+            tmax = t[0];
         }
         tmax *= scale;
         // lazy rescaling: the shift m only moves when the row's maximum exceeds it by
@@ -629,23 +664,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (grow_m) m = tmax;
         }
         const float mc = m * 1.4426950408889634f;
+        const uint32_t w32 = (uint32_t)(live >> (half * 32));   // this half's keys
         uint8_t *sP = pbuf(i);
 #pragma unroll
         for (int j0 = 0; j0 < 32; j0 += 8) {
             float pf[8];
 #pragma unroll
             for (int jj = 0; jj < 8; ++jj) {
-                const int k = j0 + jj, j = half * 32 + k;
+                const int k = j0 + jj;
                 const float s = half ? sv[32 + k] : sv[k];   // static indices keep sv in registers
-                float pw;
-                if (fast) {
-                    pw = umma::ex2_approx(fmaf(s, c1, -mc));
-                } else {
-                    const int info = M.info[j], tok = M.tok[j];
-                    const bool soft = info != INFO_SKIP && tok <= p && !(info == INFO_FOLDED && tok <= p - eta);
-                    pw = soft ? umma::ex2_approx(fmaf(s, c1, -mc)) : 0.f;
-                }
-                pf[jj] = row_ok ? pw : 0.f;
+                const float e = umma::ex2_approx(fmaf(s, c1, -mc));
+                pf[jj] = all_live ? e : ((w32 >> k) & 1u ? e : 0.f);
             }
             uint4 pk;
             pk.x = umma::pack_bf16x2(pf[0], pf[1]);
