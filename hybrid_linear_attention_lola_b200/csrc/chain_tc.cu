@@ -28,7 +28,7 @@ constexpr int kThreads = 256;
 constexpr int kFoldTok = 64;
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s per tensor-core completion wait
 #ifndef LOLA_CHAIN_CTAS
-#define LOLA_CHAIN_CTAS 40   // CTAs a prefill chain may spread over (the attention keeps the rest)
+#define LOLA_CHAIN_CTAS 64   // CTAs a prefill chain may spread over (the attention keeps the rest)
 #endif
 
 struct Geo {
@@ -770,14 +770,15 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     cudaFuncSetAttribute(chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     PrefillScratch Pv{};
     if (P) Pv = *P;
-    // prefill with few streams: a cluster of up to 8 CTAs per stream shares the scoring,
-    // one SRE tile each (at most LOLA_CHAIN_CTAS CTAs, so that the attention keeps the other SMs)
+    // prefill with few streams: a cluster of up to 5 CTAs per stream shares the scoring,
+    // one SRE tile each or more (at most LOLA_CHAIN_CTAS CTAs, so that the attention keeps the
+    // other SMs; wider clusters measured slower: the key exchange grows with the width)
     int nc = 1;
     if (a.mode == 0) {
         const int tiles = (dm.lam + dm.C + 127) / 128;   // SRE tiles of a full interval
         nc = LOLA_CHAIN_CTAS / dm.ns;
         if (nc > tiles) nc = tiles;
-        if (nc > 8) nc = 8;
+        if (nc > 5) nc = 5;
         if (nc < 1) nc = 1;
     }
     if (nc == 1) {
