@@ -19,6 +19,7 @@ import json
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -104,10 +105,12 @@ class ClockSampler:
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
+    # raw samples go to LOLA_CLOCKS_DIR (default: the system temp directory)
     def __init__(self, bus_id=None):
         self.bus_id = (bus_id or "").lower()
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+        out_dir = os.environ.get("LOLA_CLOCKS_DIR") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"lola_clocks_{os.getpid()}.csv")
 
     def start(self):
         try:
@@ -350,7 +353,7 @@ def run_engine(args, ws, rank, local):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": f"{w.name} prefill (configs[{w.wid - 1}])", "batch": w.batch,
+            "config": {"workload": f"{w.name} prefill", "batch": w.batch,
                        "seq_len": T, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
                        "head_dim": w.head_dim, "feat_dim": w.feat_dim, "window": w.window,
                        "lambda": w.lambda_, "chunk": w.chunk,
@@ -428,7 +431,7 @@ def run_decode(args, ws, rank, dev, flush, peaks, peak_src):
     achieved = bytes_step / (ms_step / 1e3) / 1e9
     peak = float(peaks["hbm_gbs"])
     S.close()
-    return {"workload": f"{w.name} (configs[{w.wid - 1}]): prefix {Tp} prefilled, "
+    return {"workload": f"{w.name}: prefix {Tp} prefilled, "
                         f"{n_dec} timed decode steps, interval {w.decode_interval}",
             "prefix_prefill_calls_of": piece,
             "value": round(whole_job_rate(w.batch, ws, ms_step / 1e3), 1), "unit": UNIT,
@@ -465,7 +468,7 @@ def run_reference(args, ws, rank):
             "n_gpus": ws, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(wall / args.steps * 1e3, 2), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": f"{w.name} prefill (configs[{w.wid - 1}])", "batch": w.batch,
+            "config": {"workload": f"{w.name} prefill", "batch": w.batch,
                        "seq_len": w.seq_len, "parallelism": "host threads"},
             "cpu_baseline": {"value": round(value, 2), "unit": UNIT, "cores": last["cores"],
                              "kind": "oracle", "sample": last["sample"]},
