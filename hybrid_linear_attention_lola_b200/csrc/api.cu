@@ -136,7 +136,8 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
     if (!lola::decode_plan(dm)) return LOLA_ERR_INVALID_ARG;
-    dm->tc_chain = (c->dtype == LOLA_BF16 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
+    // the tensor-core chain selects into a cache: lambda = 0 runs on the SIMT chain
+    dm->tc_chain = (c->dtype == LOLA_BF16 && dm->lam > 0 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;

@@ -156,6 +156,37 @@ def test_gqa_group_of_eight_and_eps_zero():
     _case(w, [("prefill", 160)], forced=True, unforced=True)
 
 
+# ---------------------------------------------------------------- edge cases (bfloat16)
+# head_dim 64 keeps these on the tensor-core chain and attention and the streaming decode
+
+def _small_bf16(**kw):
+    base = dict(head_dim=64, feat_dim=64, dtype="bf16")
+    base.update(kw)
+    return _small(**base)
+
+
+def test_bf16_no_window_no_cache_is_linear_attention():
+    w = _small_bf16(window=0, lambda_=0, decode_interval=1)
+    _case(w, [("prefill", 64), ("decode", 16)], forced=False, unforced=True)
+
+
+def test_bf16_chunk_longer_than_window_ragged_tiles():
+    # partial cache and window tiles, query rows past the interval, and kept leaving
+    # pairs that are later than some queries of their interval (chunk > window)
+    w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6)
+    _case(w, [("prefill", 240), ("decode", 13)], forced=True, unforced=True)
+
+
+def test_bf16_zero_window_with_cache():
+    w = _small_bf16(window=0, lambda_=9, chunk=8, decode_interval=1)
+    _case(w, [("prefill", 80), ("decode", 5)], forced=True, unforced=True)
+
+
+def test_bf16_gqa_group_of_eight():
+    w = _small_bf16(n_q_heads=16, n_kv_heads=2, head_dim=128, feat_dim=128, lambda_=20, chunk=32, window=16)
+    _case(w, [("prefill", 160)], forced=True, unforced=True)
+
+
 # ---------------------------------------------------------------- bf16 workloads
 
 def test_prefill_1b_full():
