@@ -741,14 +741,17 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, D
 
 // Streaming decode (bfloat16 path). A persistent grid; the work items of all
 // streams form one list (stream-major, see make_items) and every warp takes a
-// contiguous range of it, flowing its items through its own ring of three
-// shared-memory buffers (16-byte cp.async, 128-byte XOR-swizzled key/value
-// rows). For a chunk of 32 keys, S = Q K^T and O += P V run as mma.sync
-// m16n8k16 (bf16 in, fp32 accumulate) with the group's heads as the M rows
-// (padded to 16); the score fragments become the P operand directly. Linear
-// band and state items run on the SIMT units. When a warp leaves a stream it
-// writes its partial (m, l, linear den, softmax num, linear num per head); the
-// warp that writes a stream's last partial merges them (a per-stream counter).
+// contiguous range of it, flowing its items through its own ring of
+// shared-memory buffers (two by default): 32-key chunks of cache and window as
+// tiled TMA loads with 128-byte swizzle (d = 64 or 128; other d as bulk copies of
+// padded rows), linear-band rows and state rows as bulk copies, each completing on
+// the buffer's mbarrier. For a chunk of 32 keys,
+// S = Q K^T and O += P V run as mma.sync m16n8k16 (bf16 in, fp32 accumulate)
+// with the group's heads as the M rows (padded to 16); the score fragments become
+// the P operand directly. Linear band and state items run on the SIMT units. When
+// a warp leaves a stream it writes its partial (m, l, linear den, softmax num,
+// linear num per head); the warp that writes a stream's last partial merges them
+// (a per-stream counter).
 template <int DPL, int G>
 __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S, DecodeArgs a, int per, int wbytes,
                                                              const __grid_constant__ DecMaps maps)
