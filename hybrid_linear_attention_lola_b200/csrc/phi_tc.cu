@@ -58,7 +58,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int d = dm.d, D = dm.D;
     const PGeo g = make_pgeo(d, D);
     const int Dh = g.Dh;
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int tid = threadIdx.x, warp = tid >> 5;
     const int lgd = __ffs(d >> 3) - 1;   // 16-byte chunks per input row (power of two)
 
     extern __shared__ uint8_t smraw[];
