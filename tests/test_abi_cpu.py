@@ -80,3 +80,29 @@ def test_status_strings(lib):
     for code in range(9):
         assert lib.lola_status_string(code)
     assert b"unknown" in lib.lola_status_string(99)
+
+
+def test_workspace_checked_before_any_device_work(lib):
+    # a misaligned or short workspace is refused before the library touches the device
+    # (the pointers below are never dereferenced)
+    cfg = L.config_from_workload(wl.WORKLOADS["prefill-1b"])
+    need = ctypes.c_size_t(0)
+    assert lib.lola_state_bytes(ctypes.byref(cfg), ctypes.byref(need)) == 0
+    W = (ctypes.c_float * 4)()
+    h = ctypes.c_void_p(0)
+    misaligned = ctypes.c_void_p(0x100000 + 8)
+    assert lib.lola_init_state(ctypes.byref(cfg), W, misaligned, need.value, None, ctypes.byref(h)) == 5
+    aligned = ctypes.c_void_p(0x100000)
+    assert lib.lola_init_state(ctypes.byref(cfg), W, aligned, need.value - 1, None, ctypes.byref(h)) == 5
+    assert h.value is None
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_no_cache_config_is_sized(lib, dtype):
+    # lambda = 0 (window + linear state only) is a valid configuration for both dtypes
+    cfg = L.config_from_workload(wl.WORKLOADS["prefill-1b"])
+    cfg.lambda_ = 0
+    cfg.dtype = 0 if dtype == "f32" else 1
+    n = ctypes.c_size_t(0)
+    assert lib.lola_state_bytes(ctypes.byref(cfg), ctypes.byref(n)) == 0
+    assert n.value > 0
