@@ -580,7 +580,12 @@ lola_status lola_sync(lola_state *st, void *cuda_stream)
     if (cudaMemcpy(err, st->S.err, sizeof(err), cudaMemcpyDeviceToHost) != cudaSuccess)
         return check_launch();
     if (err[0] != 0) {
+        // A kernel that gave up left its work unfinished, including the per-stream
+        // counters by which the decode kernels find the last partial of a stream:
+        // they restart from zero, and the caller resets the state (lola_reset_state)
+        // before using it again.
         cudaMemset(st->S.err, 0, sizeof(err));
+        cudaMemset(st->S.dec_cnt, 0, (size_t)st->dm.ns * sizeof(int));
         return (err[0] & lola::ERR_TIMEOUT) ? LOLA_ERR_TIMEOUT : LOLA_ERR_DEVICE;
     }
     return LOLA_OK;

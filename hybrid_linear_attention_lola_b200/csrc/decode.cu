@@ -881,7 +881,8 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     float mrow = 0.f, lrow = 0.f;
     float oc[ND][4];
     float ld[G], lo[G][DPL];
-    auto begin = [&](int st) {
+    // false: the wait for the previous stream's phi(q) copy gave up (error word set)
+    auto begin = [&](int st) -> bool {
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
         const T *qg = (const T *)a.q + ((size_t)b * dm.Hq + (size_t)hk * g) * d;
         const bool hv = gq < g;
@@ -894,12 +895,20 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         // linear-band or state item of the stream (key chunks come first)
         fence_proxy_async();   // earlier reads of phq are done before the copy overwrites it
         __syncwarp();
+        bool okq = true;
         if (lane == 0) {
             // a copy whose stream needed no phi(q) lands before the next one is issued
-            if (need_q) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
-            umma::mbar_arrive_expect_tx(&mb[NST], (uint32_t)(g * D * 4));
-            umma::bulk_g2s(phq, S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D, (uint32_t)(g * D * 4), &mb[NST]);
+            if (need_q) {
+                okq = umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
+                if (!okq) raise_error(S.err, ERR_TIMEOUT);
+            }
+            if (okq) {
+                umma::mbar_arrive_expect_tx(&mb[NST], (uint32_t)(g * D * 4));
+                umma::bulk_g2s(phq, S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D, (uint32_t)(g * D * 4),
+                               &mb[NST]);
+            }
         }
+        if (__shfl_sync(0xffffffffu, okq ? 1 : 0, 0) == 0) return false;
         ++nbeg;
         need_q = true;
         const int nL = (int)(a.L_hi - a.L_lo);
@@ -913,6 +922,17 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             ld[h] = 0.f;
 #pragma unroll
             for (int u = 0; u < DPL; ++u) lo[h][u] = 0.f;
+        }
+        __syncwarp();
+        return true;
+    };
+    // Leaves the step after a wait gave up (the error word is set): lets the copies
+    // in flight land, item k's included (an abort does not wait for it).
+    auto drain = [&](int k) {
+        if (lane == 0) {
+            for (int k2 = k; k2 < k + NST && k2 < nmine; ++k2)
+                umma::mbar_wait(&mb[k2 % NST], (uint32_t)((k2 / NST) & 1), kWaitNs);
+            if (need_q) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
         }
         __syncwarp();
     };
@@ -1013,7 +1033,10 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         const int st = (int)(gi / ni), it = (int)(gi % ni);
         if (st != cur) {
             if (cur >= 0) flush(cur);
-            begin(st);
+            if (!begin(st)) {
+                drain(k);
+                return;
+            }
             cur = st;
         }
         bool got = true;
@@ -1022,13 +1045,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             if (!got) raise_error(S.err, ERR_TIMEOUT);
         }
         if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
-            // give up on the step (the error word is set): let copies in flight land,
-            // this item's included (an abort does not wait for it)
-            if (lane == 0) {
-                for (int k2 = k; k2 < k + NST && k2 < nmine; ++k2)
-                    umma::mbar_wait(&mb[k2 % NST], (uint32_t)((k2 / NST) & 1), kWaitNs);
-                if (need_q) umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
-            }
+            drain(k);
             return;
         }
         const uint8_t *buf = ring + (size_t)s * SB;
@@ -1038,7 +1055,11 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                 okq = umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
                 if (!okq) raise_error(S.err, ERR_TIMEOUT);
             }
-            if (__shfl_sync(0xffffffffu, okq ? 1 : 0, 0) == 0) return;
+            if (__shfl_sync(0xffffffffu, okq ? 1 : 0, 0) == 0) {
+                need_q = false;   // that copy was waited for (and given up on) just now
+                drain(k);
+                return;
+            }
             need_q = false;
         }
         if (it < IT.nkc) {
