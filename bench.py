@@ -6,9 +6,13 @@ one chunkwise prefill call over the workload's sequence (feature map, SRE
 scoring, top-lambda selection, fold, attention output, cache/window update).
 `value` is whole-job prefill tokens/s with inputs resident in HBM; `e2e` is the
 same through the C ABI with host buffers (H2D of q,k,v and D2H of the output
-inside the timed region). A batched-decode measurement is attached under
-"decode". Every timed number comes from CUDA events on the launching stream,
-with L2 flushed (a 256 MiB write) between timed iterations.
+inside the timed region). Decode measurements (batched decode, and single-
+sequence decode after the long-context prefill) are attached under "decode".
+Every timed number comes from CUDA events on the launching stream, with L2
+flushed (a 256 MiB write) between timed iterations.
+
+The default workload is the 8B-shaped prefill (B 4, 32/8 heads, head dim 128,
+16384 tokens), the configuration the tensor-peak target is stated on.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
 """
@@ -32,9 +36,12 @@ from hybrid_linear_attention_lola_b200 import workloads as wl  # noqa: E402
 METRIC = "LoLA prefill & decode tokens/sec on 1xB200; % of tensor/HBM roofline"
 UNIT = "tokens/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# DRAM bytes (read + write) per call of the dominant kernel, from one ncu capture of the
-# current kernel (profiles/chain_tc_prefill-1b.md); None where no capture matches.
-MEASURED_TRAFFIC = {("prefill-1b", "chain"): 27.35e6}
+# DRAM bytes per launch of a kernel, copied from ncu captures (profiles/dram_traffic.json);
+# an entry counts only while the kernel's source file is unchanged since its capture
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
+KERNEL_SOURCES = {"attn": "hybrid_linear_attention_lola_b200/csrc/attn_tc.cu",
+                  "chain": "hybrid_linear_attention_lola_b200/csrc/chain_tc.cu",
+                  "decode": "hybrid_linear_attention_lola_b200/csrc/decode.cu"}
 
 
 # ---------------------------------------------------------------- helpers
@@ -50,6 +57,30 @@ def load_peaks():
 
 def host_cores() -> int:
     return len(os.sched_getaffinity(0))
+
+
+def source_sha(rel: str) -> str:
+    import hashlib
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def captured_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
+    committed ncu summary, or (None, reason) when there is none for the current
+    source of the kernel."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            entries = json.load(f)
+    except (OSError, ValueError):
+        return None, "no ncu capture committed"
+    for e in entries:
+        if e.get("kernel") == kernel and e.get("workload") == workload:
+            src = KERNEL_SOURCES.get(kernel)
+            if src is None or e.get("source_sha") != source_sha(src):
+                return None, "kernel changed since its ncu capture"
+            return e.get("dram_bytes_per_launch"), "ncu capture (profiles/dram_traffic.json)"
+    return None, "no ncu capture for this kernel and workload"
 
 
 def interval_sizes(w, T, lam=None):
@@ -191,7 +222,7 @@ def whole_job_rate(units_per_rank: float, ws: int, seconds_max: float) -> float:
 
 # ---------------------------------------------------------------- oracle baseline
 
-def cpu_baseline(w, budget_s=15.0, threads=None):
+def cpu_baseline(w, budget_s=15.0, threads=None, single_thread=True):
     """Times the oracle, as it stands, on a bounded sample of the workload:
     a subset of (batch, kv-head) streams over a prefix of the sequence."""
     import numpy as np
@@ -213,16 +244,71 @@ def cpu_baseline(w, budget_s=15.0, threads=None):
     hsel = list(range(min(n_streams, w.n_kv_heads)))
     qsel = [h * g + r for h in hsel for r in range(g)]
     qs, ks, vs = q[:, :, qsel], k[:, :, hsel], v[:, :, hsel]
+    ints = [w.chunk] * (Ts // w.chunk)
     t = time.perf_counter()
-    oracle.run(qs, ks, vs, W, window=w.window, lambda_=w.lambda_,
-               intervals=[w.chunk] * (Ts // w.chunk), eps=w.eps, threads=cores)
+    oracle.run(qs, ks, vs, W, window=w.window, lambda_=w.lambda_, intervals=ints, eps=w.eps, threads=cores)
     dt = time.perf_counter() - t
     frac = len(hsel) / w.n_kv_heads
     tokens = Ts * frac            # prefill tokens of one sequence, all heads equivalent
-    return {"value": tokens / dt, "unit": UNIT, "cores": min(cores, len(hsel)), "kind": "oracle",
-            "sample": f"{w.name}: batch 1 of {w.batch}, kv-heads {len(hsel)} of {w.n_kv_heads} "
-                      f"(with their {g} query heads each), first {Ts} of {T} tokens; "
-                      f"{dt:.2f} s wall, fp64 C oracle"}
+    out = {"value": tokens / dt, "unit": UNIT, "cores": min(cores, len(hsel)), "kind": "oracle",
+           "sample": f"{w.name}: batch 1 of {w.batch}, kv-heads {len(hsel)} of {w.n_kv_heads} "
+                     f"(with their {g} query heads each), first {Ts} of {T} tokens; "
+                     f"{dt:.2f} s wall, fp64 C oracle"}
+    if single_thread and len(hsel) > 1:
+        # the same prefix of one stream on one thread
+        t = time.perf_counter()
+        oracle.run(qs[:, :, :g], ks[:, :, :1], vs[:, :, :1], W, window=w.window, lambda_=w.lambda_,
+                   intervals=ints, eps=w.eps, threads=1)
+        dt1 = time.perf_counter() - t
+        out["single_thread"] = {"value": (Ts / w.n_kv_heads) / dt1, "unit": UNIT, "cores": 1,
+                                "sample": f"kv-head 0 of batch 0, first {Ts} tokens; {dt1:.2f} s wall"}
+    return out
+
+
+# ---------------------------------------------------------------- roofline
+
+def prefill_roofline(w, T, ms_step, phase_ms, steps, peaks, peak_src):
+    """Headline: the whole prefill step's algorithmic FLOPs over its time, against the
+    measured bf16 tensor peak (burst; the sustained figure beside it). Per phase: the
+    attention (tensor-bound contractions) and the chain (sequential per stream: its
+    FLOPs over its time are a latency figure, not a tensor-pipe one)."""
+    fl = prefill_flops(w, T)
+    total = sum(fl.values())
+    burst = float(peaks["bf16_tflops"])
+    sust = float(peaks.get("bf16_tflops_sustained", burst))
+    ach = total / (ms_step / 1e3) / 1e12
+    per_call = {ph: v[0] / steps for ph, v in phase_ms.items() if v[1]}
+    phases = {}
+    for ph, bound in (("attn", "tensor"), ("chain", "latency (sequential intervals per stream)"),
+                      ("phi", "hbm")):
+        if ph not in per_call:
+            continue
+        a = fl[ph] / (per_call[ph] / 1e3) / 1e12
+        phases[ph] = {"ms_per_call": round(per_call[ph], 4), "tflop_per_call": round(fl[ph] / 1e12, 5),
+                      "achieved_tflops": round(a, 3), "frac_of_burst": round(a / burst, 5),
+                      "frac_of_sustained": round(a / sust, 5), "bound": bound}
+    # traffic of the dominant kernel (the phase with the most device time)
+    dom = max((p for p in ("attn", "chain") if p in per_call), key=per_call.get, default="attn")
+    traffic, tsrc = captured_traffic(dom, w.name)
+    return {"bound": "tensor", "kernel": f"whole prefill step (dominant kernel: {dom})",
+            "achieved": round(ach, 3), "peak": burst, "unit": "TFLOP/s", "frac": round(ach / burst, 5),
+            "frac_of_sustained": round(ach / sust, 5), "peak_sustained": sust,
+            "traffic": traffic, "traffic_kernel": dom, "traffic_source": tsrc,
+            "peak_source": f"{peak_src} bf16 dense (burst; sustained beside it)",
+            "algorithmic_tflop_per_step": round(total / 1e12, 5), "phases": phases,
+            "phase_ms": {ph: round(v, 4) for ph, v in per_call.items()}}
+
+
+def memory_report(w, cfg_bytes_per_stream):
+    """State + cache bytes (constant in T) against a full key/value cache of the
+    same heads at the workload's length."""
+    e = 2 if w.dtype == "bf16" else 4
+    per_seq = cfg_bytes_per_stream * w.n_kv_heads
+    full = w.seq_len * w.n_kv_heads * w.head_dim * 2 * e
+    return {"state_cache_bytes_per_stream": cfg_bytes_per_stream,
+            "state_cache_bytes_per_sequence": per_seq,
+            "full_kv_bytes_per_sequence": full, "seq_len": w.seq_len,
+            "full_kv_over_state_cache": round(full / per_seq, 3)}
 
 
 # ---------------------------------------------------------------- engine arm
@@ -291,22 +377,7 @@ def run_engine(args, ws, rank, local):
     ms_step = max_over_ranks(sum(times) / len(times), ws, dev)
     value = whole_job_rate(w.batch * T, ws, ms_step / 1e3)
 
-    # roofline of the dominant kernel (tensor-bound contractions)
-    fl = prefill_flops(w, T)
-    # per-call device time of each phase (a phase may run as several launches, and the
-    # chain of one segment overlaps the attention of the previous one)
-    cand = {ph: phase_ms[ph][0] / args.steps for ph in ("attn", "chain", "phi")
-            if ph in phase_ms and phase_ms[ph][1] > 0}
-    dom = max(cand, key=cand.get)
-    achieved = fl[dom] / (cand[dom] / 1e3) / 1e12
-    peak = float(peaks["bf16_tflops"])
-    roofline = {"bound": "tensor", "kernel": dom, "achieved": round(achieved, 3), "peak": peak,
-                "unit": "TFLOP/s", "frac": round(achieved / peak, 5),
-                "traffic": MEASURED_TRAFFIC.get((w.name, dom)),
-                "peak_source": f"{peak_src} bf16 dense (burst)",
-                "phase_ms": {ph: round(v[0] / args.steps, 4) for ph, v in phase_ms.items()
-                             if v[1]},
-                "algorithmic_tflop_per_call": {ph: round(x / 1e12, 5) for ph, x in fl.items()}}
+    roofline = prefill_roofline(w, T, ms_step, phase_ms, args.steps, peaks, peak_src)
 
     # end to end through the C ABI from pinned host memory
     qh = torch.from_numpy(q).to(dt).pin_memory()
@@ -344,10 +415,12 @@ def run_engine(args, ws, rank, local):
     S.close()
     del qd, kd, vd, out
 
-    decode = None
-    if args.decode_workload != "none":
-        decode = run_decode(args, ws, rank, dev, flush, peaks, peak_src)
-        launches += decode.pop("_launches")
+    decode = []
+    for dname in [x for x in args.decode_workload.split(",") if x and x != "none"]:
+        dres = run_decode(args, dname, ws, rank, dev, flush, peaks, peak_src)
+        launches += dres.pop("_launches")
+        decode.append(dres)
+    sb = L.lola_state_stream_bytes(cfg)
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -360,19 +433,19 @@ def run_engine(args, ws, rank, local):
                        "parallelism": f"replicas x{ws} (independent streams, no collective)",
                        "l2": "flushed (256 MiB write) before every timed step"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
-            "decode": decode}
+            "decode": decode, "memory": memory_report(w, sb)}
     if rank == 0 and ws == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     if rank == 0:
         print(json.dumps(line), flush=True)
 
 
-def run_decode(args, ws, rank, dev, flush, peaks, peak_src):
-    """Batched decode: prefill the prefix (untimed), then time every decode step
-    (L2 flushed before each). Tokens/s = batch / step time."""
+def run_decode(args, name, ws, rank, dev, flush, peaks, peak_src):
+    """Decode on workload `name`: prefill the prefix (untimed), then time every decode
+    step (L2 flushed before each). Tokens/s = batch / step time."""
     import torch
     from hybrid_linear_attention_lola_b200 import lola as L
-    w = wl.WORKLOADS[args.decode_workload]
+    w = wl.WORKLOADS[name]
     Tp, n_dec = w.seq_len, w.decode_steps
     q, k, v, _ = wl.make_inputs(w, T=Tp)
     qn, kn, vn, _ = wl.make_inputs(w, part="decode")
@@ -425,6 +498,7 @@ def run_decode(args, ws, rank, dev, flush, peaks, peak_src):
     barrier(ws)
     L.lola_set_timing(S.handle, False)
     ms_step = max_over_ranks(sum(times) / len(times), ws, dev)
+    sb = L.lola_state_stream_bytes(cfg)
     bytes_step = decode_bytes_per_step(w)
     dec_ms = ph["decode"][0] / ph["decode"][1]
     upd = ph.get("update", [0.0, 0])
@@ -438,11 +512,14 @@ def run_decode(args, ws, rank, dev, flush, peaks, peak_src):
             "ms_per_step": round(ms_step, 5), "batch": w.batch,
             "roofline": {"bound": "hbm", "kernel": "whole decode step", "achieved": round(achieved, 1),
                          "peak": peak, "unit": "GB/s", "frac": round(achieved / peak, 4),
-                         "traffic": None, "peak_source": f"{peak_src} HBM copy",
+                         "traffic": captured_traffic("decode", w.name)[0],
+                         "traffic_source": captured_traffic("decode", w.name)[1],
+                         "peak_source": f"{peak_src} HBM copy",
                          "algorithmic_bytes_per_step": bytes_step,
                          "phase_ms": {"decode_attn": round(dec_ms, 5),
                                       "interval_update_per_interval": round(upd[0] / max(upd[1], 1), 5),
                                       "append": round(ph["append"][0] / ph["append"][1], 5)}},
+            "memory": memory_report(w, sb),
             "l2": "flushed before every timed step", "_launches": launches}
 
 
@@ -455,12 +532,12 @@ def run_reference(args, ws, rank):
         return
     w = wl.WORKLOADS[args.workload]
     for _ in range(args.warmup):
-        cpu_baseline(w, budget_s=4.0)
+        cpu_baseline(w, budget_s=4.0, single_thread=False)
     vals = []
     t0 = time.perf_counter()
     last = None
     for _ in range(args.steps):
-        last = cpu_baseline(w, budget_s=4.0)
+        last = cpu_baseline(w, budget_s=4.0, single_thread=False)
         vals.append(last["value"])
     wall = time.perf_counter() - t0
     value = statistics.mean(vals)
@@ -483,9 +560,9 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="engine", choices=["engine", "reference"])
-    ap.add_argument("--workload", default="prefill-1b", choices=sorted(wl.WORKLOADS))
-    ap.add_argument("--decode-workload", default="decode-batched",
-                    choices=sorted(wl.WORKLOADS) + ["none"])
+    ap.add_argument("--workload", default="prefill-8b", choices=sorted(wl.WORKLOADS))
+    ap.add_argument("--decode-workload", default="decode-batched,long-context",
+                    help="comma-separated decode workloads (or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     ws, rank, local = dist_setup()

@@ -38,10 +38,17 @@ struct lola_state {
     cudaEvent_t ev_fork;
     cudaEvent_t ev_seg[kMaxSeg];
     lola::DecMaps maps;              // TMA descriptors of the cache / ring arrays (bf16 decode)
+    CUtensorMap phik_map, phik_box;  // row maps (1-row and 128-row boxes) of the prefill and the
+    CUtensorMap phiv_map, phiv_box;  // decode phi rows (tensor-core chain)
     int32_t *sel_log;
     long long sel_cap;
     const int32_t *ovr;
     long long ovr_n;
+    float *score_sre;
+    int32_t *score_tok;
+    long long score_cap;
+    int inject_where;                // fault-injection hook (one shot): 1 chain, 2 decode streaming kernel
+    unsigned long long inject_ns;
     // timing hook
     bool timing;
     struct Mark { int phase; cudaEvent_t a, b; };
@@ -136,8 +143,10 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
     if (!lola::decode_plan(dm)) return LOLA_ERR_INVALID_ARG;
-    // the tensor-core chain selects into a cache: lambda = 0 runs on the SIMT chain
-    dm->tc_chain = (c->dtype == LOLA_BF16 && dm->lam > 0 && lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
+    // the tensor-core chain selects into a cache (lambda = 0 runs on the SIMT chain) and
+    // holds the state image as an N-contiguous operand of whole 64-column atoms
+    dm->tc_chain = (c->dtype == LOLA_BF16 && dm->lam > 0 && dm->d % 64 == 0 &&
+                    lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
@@ -216,6 +225,14 @@ void reset_host(lola_state *st)
     st->phiV_valid = false;
 }
 
+// The armed fault-injection wait limit if it targets `where` (then disarmed), else 0.
+unsigned long long take_injection(lola_state *st, int where)
+{
+    if (st->inject_where != where) return 0;
+    st->inject_where = 0;
+    return st->inject_ns;
+}
+
 // Host mirror of one interval's bookkeeping (identical for every stream).
 void advance_interval(lola_state *st, long long t0, int len)
 {
@@ -280,7 +297,11 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;
         ca.ovr_n = st->ovr_n;
-        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, stream);
+        ca.score_sre = st->score_sre;
+        ca.score_tok = st->score_tok;
+        ca.score_cap = st->score_cap;
+        ca.inject_ns = take_injection(st, 1);
+        if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, nullptr, ca, st->phiv_map, st->phiv_box, stream);
         else lola::launch_chain(dm, st->S, nullptr, ca, stream);
         counted(1);
         if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
@@ -299,6 +320,7 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
     da.k = k;
     da.v = v;
     da.out = out;
+    da.inject_ns = dm.dtype == LOLA_BF16 ? take_injection(st, 2) : 0;
     lola::DevState Sx = st->S;
     Sx.part = part;
     Sx.phiQd = phiq;
@@ -391,6 +413,18 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
             return LOLA_ERR_CUDA;
         }
         st->seg_len = len;
+    }
+    const unsigned long long rk = (unsigned long long)dm.ns * (dm.lam + dm.R + dm.Nmax);
+    const unsigned long long rv = (unsigned long long)dm.ns * (dm.lam + dm.R);
+    if (dm.tc_chain && (!lola::make_row_map(&st->phik_map, st->P.phiK, rk, dm.D, 1) ||
+                        !lola::make_row_map(&st->phik_box, st->P.phiK, rk, dm.D, 128) ||
+                        !lola::make_row_map(&st->phiv_map, st->S.phiV, rv, dm.D, 1) ||
+                        !lola::make_row_map(&st->phiv_box, st->S.phiV, rv, dm.D, 128))) {
+        fprintf(stderr, "lola: cuTensorMapEncodeTiled failed (phi row maps)\n");
+        cudaGetLastError();
+        if (st->chain_stream != nullptr) cudaStreamDestroy(st->chain_stream);
+        delete st;
+        return LOLA_ERR_CUDA;
     }
     if (dm.dec_tma && !lola::make_decode_maps(dm, st->S, &st->maps)) {
         fprintf(stderr, "lola: cuTensorMapEncodeTiled failed\n");
@@ -494,12 +528,16 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;
         ca.ovr_n = st->ovr_n;
+        ca.score_sre = st->score_sre;
+        ca.score_tok = st->score_tok;
+        ca.score_cap = st->score_cap;
+        ca.inject_ns = take_injection(st, 1);
         ca.ci0 = ci0;
         ca.cont = sg > 0 ? 1 : 0;
         {
             PhaseScope ps(st, PH_CHAIN, cs);
             ca.snap_f32 = dm.tc_attn ? 0 : 1;
-            if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, cs);
+            if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, st->phik_map, st->phik_box, cs);
             else lola::launch_chain(dm, st->S, &st->P, ca, cs);
             counted(1);
         }
@@ -568,6 +606,26 @@ lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept,
     if (!st || n_intervals < 0) return LOLA_ERR_INVALID_ARG;
     st->ovr = dev_kept;
     st->ovr_n = dev_kept ? n_intervals : 0;
+    return LOLA_OK;
+}
+
+lola_status lola_set_fault_injection(lola_state *st, int32_t where, int64_t wait_limit_ns)
+{
+    if (!st || where < 0 || where > 2 || (where != 0 && (wait_limit_ns <= 0 || wait_limit_ns > 2000000000LL)))
+        return LOLA_ERR_INVALID_ARG;
+    if (where == 1 && !st->dm.tc_chain) return LOLA_ERR_INVALID_ARG;   // the hook sits in the tensor-core chain
+    if (where == 2 && st->dm.dtype != LOLA_BF16) return LOLA_ERR_INVALID_ARG;
+    st->inject_where = where;
+    st->inject_ns = where ? (unsigned long long)wait_limit_ns : 0;
+    return LOLA_OK;
+}
+
+lola_status lola_set_score_log(lola_state *st, float *dev_sre, int32_t *dev_tok, int64_t capacity)
+{
+    if (!st || capacity < 0 || ((dev_sre == nullptr) != (dev_tok == nullptr))) return LOLA_ERR_INVALID_ARG;
+    st->score_sre = dev_sre;
+    st->score_tok = dev_tok;
+    st->score_cap = dev_sre ? capacity : 0;
     return LOLA_OK;
 }
 

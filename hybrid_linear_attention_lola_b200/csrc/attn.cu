@@ -35,8 +35,9 @@ struct RowAcc {
 
 template <typename T>
 __global__ void __launch_bounds__(NW * 32)
-    attn_prefill_kernel(Dims dm, PrefillScratch P, AttnArgs a, KVSrc<T> src)
+    attn_prefill_kernel(Dims dm, PrefillScratch P, AttnArgs a, KVSrc<T> src, const int *err)
 {
+    if (cta_error_pending(err)) return;   // the chain of this call gave up: its logs are incomplete
     const int d = dm.d, D = dm.D, eta = dm.eta, lam = dm.lam;
     const int qsplit = (dm.C + QR - 1) / QR;
     const int ci = a.ci0 + blockIdx.x / qsplit, qp = blockIdx.x % qsplit;
@@ -264,6 +265,7 @@ template <typename T> __device__ __forceinline__ void copy_unit(T *dst, const T 
 template <typename T>
 __global__ void finalize_cache_kernel(Dims dm, DevState S, PrefillScratch P, KVSrc<T> src, int nK)
 {
+    if (*(const volatile int *)S.err != 0) return;   // the chain gave up: slot rows may be incomplete
     const int lam = dm.lam, d = dm.d;
     const int vec = row_vec<T>(d), upr = d / vec;
     const long long total = (long long)dm.ns * lam * upr;
@@ -334,12 +336,12 @@ void launch_attn_prefill(const Dims &dm, const DevState &S, const PrefillScratch
         cudaFuncSetAttribute(attn_prefill_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         attn_prefill_kernel<float><<<grid, NW * 32, smem, stream>>>(
-            dm, P, a, make_src<float>(dm, S, a.kin, a.vin, a.pos0, a.n_call));
+            dm, P, a, make_src<float>(dm, S, a.kin, a.vin, a.pos0, a.n_call), S.err);
     } else {
         cudaFuncSetAttribute(attn_prefill_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         attn_prefill_kernel<__nv_bfloat16><<<grid, NW * 32, smem, stream>>>(
-            dm, P, a, make_src<__nv_bfloat16>(dm, S, a.kin, a.vin, a.pos0, a.n_call));
+            dm, P, a, make_src<__nv_bfloat16>(dm, S, a.kin, a.vin, a.pos0, a.n_call), S.err);
     }
 }
 

@@ -174,6 +174,7 @@ __device__ __forceinline__ void mma_kn(uint32_t dt, uint32_t a0, int ra, uint32_
 __global__ void __launch_bounds__(kThreads, 1)
     attn_tc_kernel(Dims dm, DevState S, PrefillScratch P, AttnArgs a, KVSrc<bf16> src)
 {
+    if (cta_error_pending(S.err)) return;   // the chain of this call gave up: its logs are incomplete
     const AGeo g = make_ageo(dm);
     const int d = g.d, D = g.D, FP = g.FP, Dh = g.Dh, eta = dm.eta, lam = dm.lam, gq = dm.g;
     const int NK = g.NK, NV = g.NV, MS = g.MS;

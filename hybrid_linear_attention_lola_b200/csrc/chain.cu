@@ -212,7 +212,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             e = warp_sum(e);
-            if (lane == 0) keys[c] = make_key(e, ctok[c]);
+            if (lane == 0) {
+                keys[c] = make_key(e, ctok[c]);
+                if (a.score_sre != nullptr && iglob < a.score_cap) {
+                    const size_t o = ((size_t)iglob * dm.ns + st) * QC + c;
+                    a.score_sre[o] = e;
+                    a.score_tok[o] = ctok[c];
+                }
+            }
         }
         __syncthreads();
 

@@ -13,7 +13,14 @@
 // operand. The SRE of 128 candidates at a time is then one MMA chain
 // Phi_Q [H | s] into TMEM, and one thread per candidate finishes
 // || num / (den + eps) - v ||^2 with the candidate's value row staged in shared
-// memory. The kept set is the nK smallest order-preserving keys (SRE bits
+// memory. Scoring tiles arrive by TMA: a tile of 128 cached candidates is one
+// contiguous block of slot-ordered phi rows (the phi array's rows [0, lam)
+// mirror the cache slots; the kernel rewrites a slot's row when a new pair
+// takes it), loaded as one 128-row box per 64 features; a tile of leaving
+// pairs is contiguous too when they all come from this call (prefill) or from
+// one unwrapped run of the ring (decode); other tiles gather four rows per
+// instruction (tile::gather4). The fold operands are gathered by 16-byte copies. The kept set is the nK
+// smallest order-preserving keys (SRE bits
 // inverted, token index), found by an 8-pass radix select. Prefill mode stores
 // the image after the eviction fold as the interval's snapshot for attention.
 #include "lola_internal.cuh"
@@ -220,6 +227,9 @@ struct Ctx {
     uint8_t *Bs, *ones, *X;
     uint32_t tm;           // TMEM base
     uint64_t *mbar;
+    const CUtensorMap *phimap;   // phi rows of this launch, [ns * nvrows][D]
+    long long row0;        // map row of this stream's virtual row 0
+    int oob_row;           // a map row past the extent (reads as zeros)
     int *okflag;
     int *err;              // device error word (timeouts stop every CTA's waits)
     uint32_t phase;
@@ -300,6 +310,8 @@ __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict_
     for (int base = 0; base < cnt; base += kFoldTok) {
         const int nt = min(kFoldTok, cnt - base);
         const int ntp = (nt + 15) & ~15;
+        // A = Phi_F^T, MN-major per 128-feature block (16-byte copies; tokens past nt
+        // and features past D are zeros)
         for (int e = tid; e < (ntp << lgf); e += kThreads) {
             const int t = e >> lgf, f = (e & ((1 << lgf) - 1)) * 8;
             uint8_t *dst = Af + (size_t)(f >> 7) * 64 * 128 * 2 + umma::mnmajor_offset(t, f & 127, 128);
@@ -336,7 +348,8 @@ __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict_
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
-    chain_tc_kernel(Dims dm, DevState S, PrefillScratch P, ChainArgs a, KVSrc<bf16> src, int nc)
+    chain_tc_kernel(Dims dm, DevState S, PrefillScratch P, ChainArgs a, KVSrc<bf16> src, int nc,
+                    const __grid_constant__ CUtensorMap phimap, const __grid_constant__ CUtensorMap boxmap)
 {
     // nc > 1: a cluster of nc CTAs per stream; every CTA holds the state and applies the
     // same folds, the SRE tiles are dealt round-robin, the keys are exchanged through
@@ -350,6 +363,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t mbar;
+    __shared__ uint64_t tbar[2];     // SRE tile buffer 0 / 1 has landed
+    __shared__ uint64_t never;       // nothing arrives here (fault-injection hook)
     __shared__ uint64_t kready[2];   // peers' keys of an even / odd interval have arrived
     __shared__ uint32_t tslot;
     __shared__ int okflag;
@@ -374,9 +389,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     int *hist = (int *)(base + g.off_hist);
     int *scal = (int *)(base + g.off_scal);
     c.mbar = &mbar;
+    c.phimap = &phimap;
+    c.row0 = (long long)st * a.nvrows;
+    c.oob_row = dm.ns * a.nvrows;
     c.okflag = &okflag;
     c.err = S.err;
     c.phase = 0;
+    // thread 0 (lane 0 of the issuing warp): tile loads issued into / waited for per buffer
+    uint32_t tiss[2] = {0u, 0u}, twait[2] = {0u, 0u};
     // constant operands: s image rows 1..15 and the ones column (row 0 of a 16 x 64 tile)
     for (int e = tid; e < g.FP * 16; e += kThreads) {
         const int r = e / g.FP, f = e - r * g.FP;
@@ -389,6 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) {
         umma::mbar_init(&mbar, 1);
+        umma::mbar_init(&tbar[0], 1);
+        umma::mbar_init(&tbar[1], 1);
+        umma::mbar_init(&never, 1);
         umma::mbar_init(&kready[0], nc > 1 ? nc - 1 : 1);
         umma::mbar_init(&kready[1], nc > 1 ? nc - 1 : 1);
     }
@@ -429,7 +452,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int i = tid; i < lam; i += kThreads) {
         if (a.mode == 0 && a.cont) {
             slotTok[i] = P.slotTok[(size_t)st * lam + i];
-            slotVrow[i] = P.slotVrow[(size_t)st * lam + i];
+            // written by the previous launch of this call; clamped so that a launch after
+            // one that gave up (error word set, scratch not written) stays in bounds
+            slotVrow[i] = min(max(P.slotVrow[(size_t)st * lam + i], 0), a.nvrows - 1);
         } else {
             slotTok[i] = i < nS ? S.idxS[(size_t)st * lam + i] : -1;
             slotVrow[i] = i;
@@ -448,6 +473,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const long long t1 = t0 + a.ilen;
         const long long iglob = a.iglob0 + ci;
 
+        if (a.inject_ns != 0 && ci == 0) {
+            // test hook: a bounded wait that runs out, handled like any other timeout
+            if (tid == 0) {
+                const bool got = umma::mbar_wait(&never, 0, a.inject_ns);
+                if (!got) raise_error(S.err, ERR_TIMEOUT);
+                okflag = got ? 1 : 0;
+            }
+            __syncthreads();
+            if (!(ok = okflag != 0)) break;
+        }
         // 1. fold the previous interval's leaving pairs that were not kept
         if (pend_n > 0) {
             const int nf = scan_excl(lf, rank, pend_n, scal);
@@ -471,20 +506,48 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cnd = tid; cnd < nQ; cnd += kThreads)
             cvrow[cnd] = cnd < nS ? slotVrow[cnd] : src.tok2vrow(Llo + (cnd - nS));
         __syncthreads();
-        const int lgc = __ffs(g.FP >> 3) - 1;   // 16-byte chunks per phi row (power of two)
         const int ntile = (nQ + 127) / 128;
         const int nmy = ntile > crank ? (ntile - crank + nc - 1) / nc : 0;   // this CTA's tiles
-        // phi rows of this CTA's tile lt (K-major A operand) into buffer lt % nbuf; one cp.async group
+        // phi rows of this CTA's tile lt (K-major A operand) into buffer lt % nbuf by TMA
+        // row gathers from warp 0 (rows r..r+3 of one 64-feature block per instruction;
+        // rows past the candidates read as zeros); completion on tbar[buffer]
         auto load_tile = [&](int lt) {
-            uint8_t *dstT = base + (lt % g.nbuf ? g.off_X1 : g.off_X);
+            if (warp != 0) return;
+            const int bsel = lt % g.nbuf;
+            uint8_t *dstT = base + (bsel ? g.off_X1 : g.off_X);
             const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
-            for (int e = tid; e < (nr << lgc); e += kThreads) {
-                const int r = e >> lgc, kc = e & ((1 << lgc) - 1);
-                uint8_t *dst = dstT + umma::kmajor_offset(r, kc * 8, 128);
-                if (kc * 8 < D) umma::cp_async16(dst, phi_st + (size_t)cvrow[m0 + r] * D + kc * 8);
-                else *(uint4 *)dst = make_uint4(0, 0, 0, 0);
+            const int natom = g.FP >> 6;
+            if (lane == 0) {
+                umma::mbar_arrive_expect_tx(&tbar[bsel], (uint32_t)(128 * g.FP * 2));
+                ++tiss[bsel];
             }
-            umma::cp_async_commit();
+            __syncwarp();
+            // one contiguous run of phi rows: 128-row boxes (rows past the tile's
+            // candidates are other rows of the array or zeros; their scores are unused)
+            long long brow = -1;
+            if (m0 + 128 <= nS) {
+                brow = m0;                                  // cached candidates = slots m0..
+            } else if (m0 >= nS) {
+                const long long t0L = Llo + (m0 - nS);      // first leaving pair of the tile
+                if (a.mode == 0 ? t0L >= a.call_start
+                                : ((int)(t0L & (dm.R - 1)) + nr <= dm.R))
+                    brow = src.tok2vrow(t0L);
+            }
+            if (brow >= 0) {
+                if (lane < natom)
+                    umma::tma_load_2d(dstT + umma::kmajor_row(0, lane, 128), &boxmap, lane * 64,
+                                      (int)(c.row0 + brow), &tbar[bsel]);
+                return;
+            }
+            for (int e = lane; e < 32 * natom; e += 32) {
+                const int grp = e / natom, at = e - grp * natom;
+                const int r = grp * 4;
+                int rr[4];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) rr[i] = r + i < nr ? (int)(c.row0 + cvrow[m0 + r + i]) : c.oob_row;
+                umma::gather4(dstT + umma::kmajor_row(r, at, 128), c.phimap, at * 64, rr[0], rr[1], rr[2], rr[3],
+                              &tbar[bsel]);
+            }
         };
         if (nmy > 0) load_tile(0);
         if (g.nbuf == 2 && nmy > 1) load_tile(1);
@@ -493,14 +556,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hd = d >> 1;                            // value dims per thread
         for (int lt = 0; lt < nmy && ok; ++lt) {
             const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
-            if (g.nbuf == 2 && lt + 1 < nmy) umma::cp_async_wait_1();
-            else umma::cp_async_wait_all();
-            umma::fence_async_smem();
-            umma::fence_before_sync();
-            __syncthreads();
             if (tid == 0) {
+                // the tile's rows have landed (a timeout stops the MMA wait below at once)
+                const int bsel = lt % g.nbuf;
+                const bool got = umma::mbar_wait_abortable(&tbar[bsel], twait[bsel] & 1u, kWaitNs, S.err, ERR_TIMEOUT);
+                if (got) ++twait[bsel];
+                else raise_error(S.err, ERR_TIMEOUT);   // the MMA wait below gives up at once
                 umma::fence_after_sync();
-                const uint32_t a0 = umma::smem_u32(base + (lt % g.nbuf ? g.off_X1 : g.off_X));
+                const uint32_t a0 = umma::smem_u32(base + (bsel ? g.off_X1 : g.off_X));
                 const uint32_t bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
                 for (int ks = 0; ks < g.FP / 16; ++ks) {
                     const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
@@ -548,6 +611,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (half == 0 && r < nr) {
                     err += part[r];
                     keys[m0 + r] = 0xFFFFFFFFu - __float_as_uint(fmaxf(err, 0.f));
+                    if (a.score_sre != nullptr && iglob < a.score_cap) {
+                        const int cand = m0 + r;
+                        const size_t o = ((size_t)iglob * dm.ns + st) * g.QC + cand;
+                        a.score_sre[o] = err;
+                        a.score_tok[o] = cand < nS ? slotTok[cand] : (int)(Llo + (cand - nS));
+                    }
                 }
             }
             umma::fence_before_sync();
@@ -672,6 +741,22 @@ __global__ void __launch_bounds__(kThreads, 1)
                 slotVrow[slot] = a.mode == 0 ? src.tok2vrow(tok) : slot;
             }
         }
+        if (a.mode == 0) {
+            // the slot's phi row follows its new pair (only the CTA that scores the
+            // slot's tile reads that row back, by TMA: fence for the async proxy)
+            bf16 *phw = (bf16 *)a.phi + (size_t)st * a.nvrows * D;
+            bool wrote = false;
+            for (int i = warp; i < nL; i += kThreads / 32) {
+                if (!keep[nS + i] || rank[i] >= nE + (lam - nS)) continue;
+                const int slot = freeSlot[rank[i]];
+                if ((slot >> 7) % nc != crank) continue;
+                const uint4 *from = (const uint4 *)(phw + (size_t)src.tok2vrow(Llo + i) * D);
+                uint4 *to = (uint4 *)(phw + (size_t)slot * D);
+                for (int e = lane; e < D / 8; e += 32) to[e] = from[e];
+                wrote = true;
+            }
+            if (wrote) umma::fence_async_global();
+        }
         if (a.mode == 1) {
             bf16 *KS = (bf16 *)S.KS + (size_t)st * lam * d;
             bf16 *VS = (bf16 *)S.VS + (size_t)st * lam * d;
@@ -739,6 +824,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (tid == 0) {
             raise_error(S.err, ERR_TIMEOUT);
             umma::mbar_wait(&mbar, c.phase ^ 1u, kWaitNs);  // let an MMA still in flight drain
+            for (int b = 0; b < 2; ++b)                      // and tile gathers still in flight
+                if (tiss[b] != twait[b]) umma::mbar_wait(&tbar[b], twait[b] & 1u, kWaitNs);
         }
     }
     if (tid == 0) umma::bulk_wait_all();
@@ -761,7 +848,7 @@ size_t snap_image_bytes(const Dims &dm)
 }
 
 void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
-                     cudaStream_t stream)
+                     const CUtensorMap &phimap, const CUtensorMap &boxmap, cudaStream_t stream)
 {
     KVSrc<bf16> src{(const bf16 *)S.KS, (const bf16 *)S.VS, (const bf16 *)S.KR, (const bf16 *)S.VR,
                     (const bf16 *)a.kin, (const bf16 *)a.vin, dm.lam, dm.R, a.n_call, dm.Hkv, dm.d,
@@ -782,7 +869,7 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
         if (nc < 1) nc = 1;
     }
     if (nc == 1) {
-        chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src, 1);
+        chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src, 1, phimap, boxmap);
         return;
     }
     cudaLaunchConfig_t cfg{};
@@ -797,7 +884,7 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, chain_tc_kernel, dm, S, Pv, a, src, nc);
+    cudaLaunchKernelEx(&cfg, chain_tc_kernel, dm, S, Pv, a, src, nc, phimap, boxmap);
 }
 
 }  // namespace lola

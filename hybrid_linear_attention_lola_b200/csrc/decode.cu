@@ -869,7 +869,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         }
     };
     if (lane == 0)
-        for (int i = 0; i <= NST; ++i) umma::mbar_init(&mb[i], 1);
+        for (int i = 0; i <= NST + 1; ++i) umma::mbar_init(&mb[i], 1);   // mb[NST + 1]: nothing arrives
     __syncwarp();
     for (int k = 0; k < NST; ++k) issue(k, k);
 
@@ -1027,6 +1027,19 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         if (lane == 0) S.dec_cnt[st] = 0;
     };
 
+    if (a.inject_ns != 0 && gw == 0) {
+        // test hook: a bounded wait that runs out, handled like any other timeout (the
+        // warp leaves before counting its partial)
+        bool got = true;
+        if (lane == 0) {
+            got = umma::mbar_wait(&mb[NST + 1], 0, a.inject_ns);
+            if (!got) raise_error(S.err, ERR_TIMEOUT);
+        }
+        if (__shfl_sync(0xffffffffu, got ? 1 : 0, 0) == 0) {
+            drain(0);
+            return;
+        }
+    }
     for (int k = 0; k < nmine; ++k) {
         const int s = k % NST;
         const long long gi = i0 + k;

@@ -9,7 +9,10 @@
 // stream:  [0, lam)            cache slot i
 //          [lam, lam + R)      ring slot (token mod R; R is a power of two)
 //          [lam + R, lam+R+n)  token call_start + (row - lam - R) of the call
-// phi(k) scratch is laid out over the same rows.
+// phi(k) scratch is laid out over the same rows. Its rows [0, lam) always hold
+// phi of the pair currently in each cache slot (the tensor-core chain rewrites
+// a slot's row when a new pair takes the slot), so the chain loads the cached
+// candidates as contiguous 128-row blocks.
 #pragma once
 
 #include <cuda.h>
@@ -186,6 +189,18 @@ __device__ __forceinline__ void raise_error(int *err, int code)
     if (err) atomicOr(err, code);
 }
 
+// CTA-uniform check at kernel entry: an earlier kernel of this state recorded an
+// error. Kernels that read the per-interval logs of the chain skip their work then
+// (after a chain gave up, those logs may be incomplete); lola_sync reports the
+// error and clears the word.
+__device__ __forceinline__ bool cta_error_pending(const int *err)
+{
+    __shared__ int flag;
+    if (threadIdx.x == 0) flag = *(const volatile int *)err;
+    __syncthreads();
+    return flag != 0;
+}
+
 // ---- host launch wrappers (defined in the .cu files) ----
 void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream);
 void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long call_start,
@@ -217,13 +232,19 @@ struct ChainArgs {
     long long sel_cap;
     const int32_t *ovr;     // test hook, may be null
     long long ovr_n;
+    unsigned long long inject_ns;   // test hook: > 0 makes the first interval wait this long on an
+                                    // mbarrier nothing arrives at (the wait runs out: timeout)
+    float *score_sre;       // test hook, may be null: SRE of every candidate
+    int32_t *score_tok;     //   and its token, [interval][ns][lam + Lmax] (candidate order)
+    long long score_cap;
     int snap_f32;           // prefill: also write fp32 (H', s') snapshots
     int ci0;                // prefill: index of the first interval within the call
     int cont;               // prefill: the call's earlier intervals ran in an earlier launch
                             // (slot contents come from the scratch, not the state)
 };
+// phimap / boxmap: row maps of a.phi as [ns * a.nvrows][D] with 1-row / 128-row boxes
 void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
-                     cudaStream_t stream);
+                     const CUtensorMap &phimap, const CUtensorMap &boxmap, cudaStream_t stream);
 size_t chain_tc_smem_bytes(const Dims &dm);
 size_t attn_tc_smem_bytes(const Dims &dm);
 size_t snap_image_bytes(const Dims &dm);
@@ -252,6 +273,11 @@ struct DecMaps {
     CUtensorMap ks, vs, kr, vr;
 };
 
+// Row map of a bfloat16 array [rows][cols]: boxes of box_rows x 64 columns,
+// 128-byte swizzle, zero fill past the extent (box_rows 1: tile::gather4 loads);
+// false if encoding fails.
+bool make_row_map(CUtensorMap *m, const void *base, unsigned long long rows, int cols, int box_rows);
+
 struct DecodeArgs {
     long long pos;          // token index of this step
     long long t0;           // start of the open interval
@@ -260,6 +286,8 @@ struct DecodeArgs {
     long long L_hi;
     const void *q, *k, *v;
     void *out;
+    unsigned long long inject_ns;   // test hook: > 0 makes the streaming kernel's first warp wait
+                                    // this long on an mbarrier nothing arrives at (timeout)
 };
 // Decode launch shape: splits per stream, warps per CTA, staging buffers and
 // their size (fills dm.nsplit, dec_nw, dec_nst, dec_sb); returns false if no

@@ -43,6 +43,19 @@ __device__ __forceinline__ uint32_t mnmajor_offset(int k, int n, int N)
                       ((((nn >> 3) ^ (k & 7))) << 4) + ((nn & 7) << 1));
 }
 
+// Start of the 128-byte row that holds row r of 64-column block kb of a K-major
+// tile (the row's 16-byte chunks are swizzled within it by the address).
+__device__ __forceinline__ uint32_t kmajor_row(int r, int kb, int R)
+{
+    return (uint32_t)(kb * R * 128 + (r >> 3) * 1024 + (r & 7) * 128);
+}
+// Start of the 128-byte row that holds k-row k of 64-column block nb of an
+// MN-major tile with N columns.
+__device__ __forceinline__ uint32_t mnmajor_row(int k, int nb, int N)
+{
+    return (uint32_t)((k >> 3) * (N >> 6) * 1024 + nb * 1024 + (k & 7) * 128);
+}
+
 __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
 {
     uint64_t d = 0;
@@ -278,6 +291,33 @@ __device__ __forceinline__ void tma_load_3d(void *smem_dst, const void *tmap, in
         "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];"
         :
         : "r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(smem_u32(mbar))
+        : "memory");
+}
+
+// Tiled 2-D TMA load of one box (no multicast); completion counted on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(void *smem_dst, const void *tmap, int x, int y, uint64_t *mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :
+        : "r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(y), "r"(smem_u32(mbar))
+        : "memory");
+}
+// Orders this thread's generic-proxy global writes before later async-proxy (TMA) reads.
+__device__ __forceinline__ void fence_async_global() { asm volatile("fence.proxy.async.global;" ::: "memory"); }
+
+// Row gather (TMA tile::gather4, no multicast): rows r0..r3 of a 2-D row map,
+// 64 columns from column x (x % 64 == 0), into four consecutive 128-byte rows
+// at smem_dst (128-byte aligned; the 128-byte swizzle follows the address).
+// Rows past the map's extent read as zero. Completion is counted on the mbarrier.
+__device__ __forceinline__ void gather4(void *smem_dst, const void *tmap, int x, int r0, int r1, int r2, int r3,
+                                        uint64_t *mbar)
+{
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
+        :
+        : "r"(smem_u32(smem_dst)), "l"(tmap), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3), "r"(smem_u32(mbar))
         : "memory");
 }
 

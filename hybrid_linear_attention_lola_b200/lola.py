@@ -62,6 +62,8 @@ def load_library() -> ctypes.CDLL:
         "lola_get_cache_indices": (I32, [P, P, P, P]),
         "lola_set_selection_log": (I32, [P, P, I64]),
         "lola_set_selection_override": (I32, [P, P, I64]),
+        "lola_set_score_log": (I32, [P, P, P, I64]),
+        "lola_set_fault_injection": (I32, [P, I32, I64]),
         "lola_sync": (I32, [P, P]),
         "lola_free_state": (I32, [P]),
         "lola_status_string": (ctypes.c_char_p, [I32]),
@@ -165,6 +167,14 @@ def lola_set_selection_log(h: int, buf: int, capacity: int):
     _check(load_library().lola_set_selection_log(h, buf, capacity), "lola_set_selection_log")
 
 
+def lola_set_fault_injection(handle, where: int, wait_limit_ns: int) -> None:
+    _check(load_library().lola_set_fault_injection(handle, where, wait_limit_ns), "lola_set_fault_injection")
+
+
+def lola_set_score_log(handle, sre_ptr: int, tok_ptr: int, capacity: int) -> None:
+    _check(load_library().lola_set_score_log(handle, sre_ptr, tok_ptr, capacity), "lola_set_score_log")
+
+
 def lola_set_selection_override(h: int, buf: int, n_intervals: int):
     _check(load_library().lola_set_selection_override(h, buf, n_intervals),
            "lola_set_selection_override")
@@ -266,6 +276,16 @@ class LolaState:
         lola_set_selection_log(self.handle, buf.data_ptr(), capacity)
         self._keep.append(buf)
         return buf
+
+    def enable_score_log(self, capacity: int):
+        """Per-candidate SRE log: returns (sre float32, tok int32) device tensors of
+        shape [capacity, streams, lambda + max(chunk, decode_interval)] (tok -1 unused)."""
+        qc = self.cfg.lambda_ + max(self.cfg.chunk, self.cfg.decode_interval)
+        sre = self.torch.zeros((capacity, self.streams, qc), dtype=self.torch.float32, device=self.device)
+        tok = self.torch.full((capacity, self.streams, qc), -1, dtype=self.torch.int32, device=self.device)
+        lola_set_score_log(self.handle, sre.data_ptr(), tok.data_ptr(), capacity)
+        self._keep += [sre, tok]
+        return sre, tok
 
     def set_selection_override(self, kept):
         """kept: int32 [n_int, streams, lambda+1] (count, ascending ids, -1 pad)."""

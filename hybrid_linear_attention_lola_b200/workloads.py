@@ -74,6 +74,16 @@ WORKLOADS = {
                              head_dim=128, feat_dim=256, window=64, lambda_=2048,
                              chunk=128, decode_interval=64, seq_len=65536,
                              decode_steps=512, dtype="bf16", needles=256),
+    # the same long-context stream at 128K and 256K tokens (same seed and feature map;
+    # the state and cache bytes do not grow with the sequence)
+    "long-context-128k": Workload("long-context-128k", 5, batch=1, n_q_heads=32, n_kv_heads=8,
+                                  head_dim=128, feat_dim=256, window=64, lambda_=2048,
+                                  chunk=128, decode_interval=64, seq_len=131072,
+                                  decode_steps=512, dtype="bf16", needles=256),
+    "long-context-256k": Workload("long-context-256k", 5, batch=1, n_q_heads=32, n_kv_heads=8,
+                                  head_dim=128, feat_dim=256, window=64, lambda_=2048,
+                                  chunk=128, decode_interval=64, seq_len=262144,
+                                  decode_steps=512, dtype="bf16", needles=256),
     # the pages' own cache setting for the 4K single-needle evaluation (window 256,
     # sparse cache 256) on the 8B-shaped heads, with planted needles as in prefill-1b
     "pages-4k": Workload("pages-4k", 6, batch=1, n_q_heads=32, n_kv_heads=8, head_dim=128,

@@ -162,6 +162,32 @@ lola_status lola_set_selection_log(lola_state *st, int32_t *dev_buf, int64_t cap
 lola_status lola_set_selection_override(lola_state *st, const int32_t *dev_kept,
                                         int64_t n_intervals);
 
+/* Test hook: log the Self-Recall Error the engine computed for every candidate
+ * of every update interval (in the precision of the state's tensor-core or SIMT
+ * path) and the candidate's token. dev_sre (float) and dev_tok (int32) are
+ * device buffers of capacity * B * n_kv_heads * (lambda_ + max(chunk,
+ * decode_interval)) entries; candidate c of interval i (counted from the last
+ * init/reset) of stream s goes to ((i * streams) + s) * (lambda_ + max(chunk,
+ * decode_interval)) + c, cache slots first, then the pairs leaving the window;
+ * entries past the interval's candidates are not written. Intervals >= capacity
+ * are not logged. NULL pointers (both) disable the log. Used to compare the
+ * engine's scores with the reference scores candidate by candidate. */
+lola_status lola_set_score_log(lola_state *st, float *dev_sre, int32_t *dev_tok, int64_t capacity);
+
+/* Test hook for failure detection. Arms one bounded device wait that nothing
+ * satisfies: where = 1, the tensor-core chain of the next prefill call (or decode
+ * interval) waits at its first interval; where = 2 (bfloat16), one warp of the
+ * next decode step's streaming kernel waits before its first work item. The wait
+ * gives up after wait_limit_ns (1 .. 2e9) nanoseconds, exactly like a real wait
+ * that runs out: the kernel records LOLA_ERR_TIMEOUT in the error word, lets its
+ * copies and tensor-core work in flight finish, and leaves its work; later kernels
+ * of the state that read the chain's per-interval logs skip theirs, and
+ * lola_sync() returns LOLA_ERR_TIMEOUT and clears the word. The state's contents
+ * are then undefined (reset it). One shot: the hook disarms itself when used;
+ * where = 0 disarms it. LOLA_ERR_INVALID_ARG for a target the config does not run
+ * (no tensor-core chain, or not bfloat16). */
+lola_status lola_set_fault_injection(lola_state *st, int32_t where, int64_t wait_limit_ns);
+
 /* Timing hook: when enabled (enable != 0), every entry point brackets each of
  * its kernel phases with CUDA events recorded on the caller's stream. Phases:
  * 0 feature map, 1 chain (score/select/fold), 2 attention (prefill), 3 call
@@ -190,7 +216,10 @@ int64_t lola_launch_count(void);
 
 /* Waits for the stream work of this state to finish and reports device-side
  * errors recorded since the last lola_sync (LOLA_ERR_DEVICE / LOLA_ERR_TIMEOUT),
- * clearing them. */
+ * clearing them. Once an error is recorded, the kernels that read the chain's
+ * per-interval logs (prefill attention, cache finalisation) skip their work until
+ * this call clears it; the state must then be reset (lola_reset_state) before its
+ * results mean anything again. */
 lola_status lola_sync(lola_state *st, void *cuda_stream);
 
 /* Frees the host handle only; the workspace stays the caller's. */

@@ -52,7 +52,7 @@ def _load():
         P = ctypes.c_void_p
         lib.oracle_run.restype = ctypes.c_int
         lib.oracle_run.argtypes = [ctypes.POINTER(OracleCfg), ctypes.c_int, P, P, P, P,
-                                   ctypes.c_int, P, P, P, P, P, P, P, P, P,
+                                   ctypes.c_int, P, P, P, ctypes.c_int, P, P, P, P, P, P, P,
                                    ctypes.c_int, P, P, ctypes.c_int]
         lib.oracle_phi.restype = None
         lib.oracle_phi.argtypes = [P, P, ctypes.c_int, ctypes.c_int, P]
@@ -88,7 +88,8 @@ def sre(phik: np.ndarray, v: np.ndarray, H: np.ndarray, s: np.ndarray, eps: floa
 class OracleResult:
     """Outputs and per-interval logs of one oracle run.
 
-    out      [B, T, Hq, d] fp64 (rows outside qmask are zero)
+    out      [B, T, Hq, d] fp64 (rows outside qmask are zero); with compact=True
+             [B, n_sel, Hq, d] holding only the qmask positions, in order (rows)
     kept     [n_int, B*Hkv, lam] int32: kept token ids after each interval, ascending, -1 pad
     nkept    [n_int, B*Hkv]
     nq       [n_int, B*Hkv] number of candidates |Q|
@@ -101,8 +102,10 @@ class OracleResult:
 def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: int,
         lambda_: int, intervals: Sequence[int], eps: float = 1e-6,
         qmask: Optional[np.ndarray] = None, want_cands: bool = False,
-        want_state: bool = False, threads: Optional[int] = None) -> OracleResult:
-    """Runs the recurrence from an empty state over tokens split into `intervals`."""
+        want_state: bool = False, threads: Optional[int] = None,
+        compact: bool = False) -> OracleResult:
+    """Runs the recurrence from an empty state over tokens split into `intervals`.
+    compact=True (with qmask) stores only the outputs of the masked positions."""
     lib = _load()
     q = np.ascontiguousarray(q, np.float32)
     k = np.ascontiguousarray(k, np.float32)
@@ -116,7 +119,15 @@ def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: i
     ns = B * Hkv
     cfg = OracleCfg(B, Hq, Hkv, d, D, window, lambda_, eps)
     r = OracleResult()
-    r.out = np.zeros((B, T, Hq, d), np.float64)
+    out_row = None
+    n_out = T
+    if compact and qmask is not None:
+        sel = np.flatnonzero(np.asarray(qmask) != 0)
+        out_row = np.full(T, -1, np.int32)
+        out_row[sel] = np.arange(len(sel), dtype=np.int32)
+        n_out = len(sel)
+        r.rows = sel
+    r.out = np.zeros((B, n_out, Hq, d), np.float64)
     lam_alloc = max(lambda_, 1)
     r.kept = np.full((n_int, ns, lam_alloc), -1, np.int32)
     r.nkept = np.zeros((n_int, ns), np.int32)
@@ -130,7 +141,7 @@ def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: i
     qm = None if qmask is None else np.ascontiguousarray(qmask, np.uint8)
     nt = threads if threads else max(1, len(os.sched_getaffinity(0)))
     rc = lib.oracle_run(ctypes.byref(cfg), T, _ptr(q), _ptr(k), _ptr(v), _ptr(W), n_int,
-                        _ptr(ints), _ptr(qm), _ptr(r.out),
+                        _ptr(ints), _ptr(qm), _ptr(out_row), n_out, _ptr(r.out),
                         _ptr(r.kept) if lambda_ > 0 else None, _ptr(r.nkept), _ptr(r.nq),
                         _ptr(r.margin), _ptr(r.cand_tok), _ptr(r.cand_sre), cap,
                         _ptr(r.H), _ptr(r.s), nt)

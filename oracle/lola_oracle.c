@@ -129,7 +129,9 @@ typedef struct {
     int n_int;
     const int32_t *int_len;
     const uint8_t *qmask; /* [T] or NULL: which query positions get outputs */
-    double *out;          /* [B][T][Hq][d] */
+    const int32_t *out_row; /* [T] or NULL: output row of each position (NULL: row = position) */
+    int n_out;            /* output rows per batch */
+    double *out;          /* [B][n_out][Hq][d] */
     int32_t *kept;        /* [n_int][nstreams][lam] or NULL (sorted ascending, -1 pad) */
     int32_t *nkept;       /* [n_int][nstreams] or NULL */
     int32_t *nq;          /* [n_int][nstreams] or NULL */
@@ -296,7 +298,8 @@ static void run_stream(job_t *J, int st)
                 }
                 double em = exp(-mx);
                 den += em * lden;
-                double *o = J->out + (((size_t)b * T + p) * Hq + hq) * d;
+                const int orow = J->out_row ? J->out_row[p] : p;
+                double *o = J->out + (((size_t)b * J->n_out + orow) * Hq + hq) * d;
                 for (int c = 0; c < d; ++c) o[c] = (num[c] + em * lin[c]) / den;
             }
         }
@@ -356,10 +359,12 @@ static void *worker(void *arg)
  * Tokens [0, T) are split into n_int consecutive intervals of the given lengths;
  * they must cover [0, T), and the last may extend past T when the pairs it
  * scores (those leaving the window before its end) all exist. Every output
- * pointer except `out` may be NULL.
+ * pointer except `out` may be NULL. With out_row, the output of position p goes
+ * to row out_row[p] of an [B][n_out][Hq][d] array (for sampled long runs).
  */
 int oracle_run(const oracle_cfg *cfg, int T, const float *q, const float *k, const float *v,
                const float *Wf, int n_int, const int32_t *int_len, const uint8_t *qmask,
+               const int32_t *out_row, int n_out,
                double *out, int32_t *kept, int32_t *nkept, int32_t *nq, double *margin,
                int32_t *cand_tok, double *cand_sre, int cand_cap, double *H_final,
                double *s_final, int nthreads)
@@ -384,6 +389,15 @@ int oracle_run(const oracle_cfg *cfg, int T, const float *q, const float *k, con
     memset(&J, 0, sizeof(J));
     J.cfg = cfg; J.T = T; J.q = q; J.k = k; J.v = v; J.W = W;
     J.n_int = n_int; J.int_len = int_len; J.qmask = qmask; J.out = out;
+    J.out_row = out_row; J.n_out = out_row ? n_out : T;
+    if (out_row) {
+        /* every position that gets an output needs a row inside [0, n_out) */
+        for (int p = 0; p < T; ++p)
+            if ((!qmask || qmask[p]) && (out_row[p] < 0 || out_row[p] >= n_out)) {
+                free(W);
+                return -5;
+            }
+    }
     J.kept = kept; J.nkept = nkept; J.nq = nq; J.margin = margin;
     J.cand_tok = cand_tok; J.cand_sre = cand_sre; J.cand_cap = cand_cap;
     J.H_final = H_final; J.s_final = s_final;

@@ -32,10 +32,14 @@ def _cuda():
     build.build()
 
 
-def _case(w, plan, *, forced=True, unforced=False, subset=None, qmask_every=None,
-          T=None, seed_inputs=None):
-    """Runs plan on the GPU and the oracle; returns a dict of metrics and asserts
-    the parity bar. subset=(batches, kv_heads) restricts the oracle's streams."""
+ROW_TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+def _case(w, plan, *, modes=("forced", "own"), subset=None, qmask_every=None,
+          T=None, seed_inputs=None, scores=False, name=None):
+    """Runs plan on the GPU (once per mode, see tests/parity.py) and the oracle once;
+    asserts the parity bar, records the counts, and returns a dict of metrics per
+    mode. subset=(batches, kv_heads) restricts the oracle's streams."""
     T = sum(n for _, n in plan) if T is None else T
     q, k, v, _ = seed_inputs if seed_inputs is not None else wl.make_inputs(w, T=T)
     W = wl.make_W(w)
@@ -47,45 +51,54 @@ def _case(w, plan, *, forced=True, unforced=False, subset=None, qmask_every=None
     hsel = list(range(w.n_kv_heads)) if subset is None else subset[1]
     g = w.group
     qsel = [hk * g + r for hk in hsel for r in range(g)]
-    qo = q[bsel][:, :, qsel]
-    ko = k[bsel][:, :, hsel]
-    vo = v[bsel][:, :, hsel]
-    qmask = None
+    qo = np.ascontiguousarray(q[bsel][:, :, qsel])
+    ko = np.ascontiguousarray(k[bsel][:, :, hsel])
+    vo = np.ascontiguousarray(v[bsel][:, :, hsel])
+    qmask = rows = None
     if qmask_every:
         qmask = np.zeros(T, np.uint8)
         qmask[::qmask_every] = 1
         qmask[-1] = 1
+        rows = np.flatnonzero(qmask)
     r = oracle.run(qo, ko, vo, W, window=w.window, lambda_=w.lambda_, intervals=ints,
-                   eps=w.eps, qmask=qmask, want_cands=True)
+                   eps=w.eps, qmask=qmask, want_cands=True, compact=qmask is not None)
     smap = [b * w.n_kv_heads + h for b in bsel for h in hsel]
+    ns = w.batch * w.n_kv_heads
     res = {}
-    runs = []
-    if forced:
-        runs.append(("forced", P.override_from(r, w.lambda_, w.batch * w.n_kv_heads, smap)))
-    if unforced:
-        runs.append(("unforced", None))
-    for name, ovr in runs:
-        out, log = P.run_gpu(cfg, W, q, k, v, plan, override=ovr, log_cap=len(ints))
+    for mode in modes:
+        ovr = None
+        if mode == "forced":
+            ovr = P.override_from(r, w.lambda_, ns, smap)
+        elif mode == "own":
+            ovr = P.override_from(r, w.lambda_, ns, smap, only_under_margin=True)
+        out, log, sc = P.run_gpu(cfg, W, q, k, v, plan, override=ovr, log_cap=len(ints), rows=rows,
+                                 score_cap=len(ints) if (scores and mode == "forced") else None)
         go = out[bsel][:, :, qsel]
-        if qmask is not None:
-            go = go[:, qmask == 1]
-            oo = r.out[:, qmask == 1]
-        else:
-            oo = r.out
         assert np.all(np.isfinite(go))
-        err = P.rel_l2(go, oo)
+        err = P.rel_l2(go, r.out)
+        rmax = P.row_rel_l2_max(go, r.out)
         checked, exact, under, hard = P.compare_selections(log, r, w.lambda_, smap)
-        res[name] = dict(rel_l2=err, checked=checked, exact=exact, under=under, hard=hard)
-        print(f"{w.name} {name}: rel_l2={err:.3e} intervals={checked} exact={exact} "
-              f"under-margin={under} hard={len(hard)}")
-        if name == "forced":
+        u = dict(rel_l2=err, row_rel_l2_max=rmax, intervals_checked=checked, exact=exact,
+                 under_margin_differ=under, hard=len(hard),
+                 forced_intervals=int(np.sum(ovr[:, smap, 0] >= 0)) if ovr is not None else 0)
+        if sc is not None:
+            u["sre_vs_oracle"] = P.score_errors(sc, r, smap)
+        res[mode] = u
+        print(f"{w.name} {mode}: {u}")
+        if mode in ("forced", "own"):
             assert not hard, hard[:4]
-            assert err <= TOL[w.dtype], err
-    if unforced:
-        u = res["unforced"]
-        # the product path without forcing: identical unless an ambiguous choice moved it
-        if u["exact"] == u["checked"]:
-            assert u["rel_l2"] <= TOL[w.dtype], u
+            assert err <= TOL[w.dtype], u
+            assert rmax <= ROW_TOL[w.dtype], u
+        elif exact == checked:
+            # the product path without any forcing: identical unless an ambiguous choice moved it
+            assert err <= TOL[w.dtype] and rmax <= ROW_TOL[w.dtype], u
+    P.record(name or w.name, {"workload": w.name, "dtype": w.dtype, "plan": [list(x) for x in plan],
+                              "streams_compared": len(smap), "streams_total": ns,
+                              "outputs_compared": "every position" if rows is None
+                              else f"every {qmask_every}th position and the last ({len(rows)})",
+                              "tolerance": {"rel_l2": TOL[w.dtype], "row_rel_l2": ROW_TOL[w.dtype],
+                                            "selection_margin": P.MARGIN},
+                              "oracle_margins": P.margin_summary(r), "runs": res})
     return res
 
 
@@ -99,61 +112,64 @@ def _small(**kw):
 
 # ---------------------------------------------------------------- tiny (fp32)
 
+ALL = ("forced", "own", "free")
+
+
 def test_tiny_prefill_parity():
     w = wl.WORKLOADS["tiny"]
-    res = _case(w, [("prefill", 512)], forced=True, unforced=True)
-    assert res["unforced"]["exact"] == res["unforced"]["checked"]
-    assert res["unforced"]["rel_l2"] <= 1e-4
+    res = _case(w, [("prefill", 512)], modes=ALL)
+    assert res["free"]["exact"] == res["free"]["intervals_checked"]
+    assert res["free"]["rel_l2"] <= 1e-4
 
 
 def test_tiny_prefill_then_decode_parity():
     w = wl.WORKLOADS["tiny"]
-    _case(w, [("prefill", 256), ("decode", 256)], forced=True, unforced=True)
+    _case(w, [("prefill", 256), ("decode", 256)], modes=ALL, name="tiny prefill+decode")
 
 
 def test_tiny_split_calls_equal_single_call():
     w = wl.WORKLOADS["tiny"]
-    _case(w, [("prefill", 128), ("prefill", 64), ("prefill", 320)], forced=True, unforced=True)
+    _case(w, [("prefill", 128), ("prefill", 64), ("prefill", 320)], modes=ALL, name="tiny split calls")
 
 
 def test_decode_then_prefill_then_decode():
     w = _small(decode_interval=8)
-    _case(w, [("prefill", 32), ("decode", 24), ("prefill", 48), ("decode", 20)],
-          forced=True, unforced=True)
+    _case(w, [("prefill", 32), ("decode", 24), ("prefill", 48), ("decode", 20)], modes=ALL,
+          name="f32 decode/prefill interleaved")
 
 
 # ---------------------------------------------------------------- edge cases (fp32)
 
 def test_no_window_no_cache_is_linear_attention():
     w = _small(window=0, lambda_=0, decode_interval=1)
-    _case(w, [("prefill", 64), ("decode", 16)], forced=False, unforced=True)
+    _case(w, [("prefill", 64), ("decode", 16)], modes=("free",), name="f32 linear only")
 
 
 def test_window_covering_everything_is_softmax():
     w = _small(window=200, lambda_=0, decode_interval=16)
-    _case(w, [("prefill", 128), ("decode", 32)], forced=False, unforced=True)
+    _case(w, [("prefill", 128), ("decode", 32)], modes=("free",), name="f32 softmax only")
 
 
 def test_cache_holding_everything():
     w = _small(window=4, lambda_=256, decode_interval=4)
-    _case(w, [("prefill", 96), ("decode", 32)], forced=False, unforced=True)
+    _case(w, [("prefill", 96), ("decode", 32)], modes=("free",), name="f32 cache holds all")
 
 
 def test_chunk_longer_than_window_ragged_tiles():
     # leaving pairs come from the current chunk; lambda and C off the 32/64 tile grid
     w = _small(window=5, lambda_=37, chunk=48, decode_interval=6, head_dim=64, feat_dim=64)
-    _case(w, [("prefill", 240), ("decode", 13)], forced=True, unforced=True)
+    _case(w, [("prefill", 240), ("decode", 13)], modes=ALL, name="f32 chunk > window, ragged")
 
 
 def test_zero_window_with_cache():
     w = _small(window=0, lambda_=9, chunk=8, decode_interval=1)
-    _case(w, [("prefill", 80), ("decode", 5)], forced=True, unforced=True)
+    _case(w, [("prefill", 80), ("decode", 5)], modes=ALL, name="f32 zero window")
 
 
 def test_gqa_group_of_eight_and_eps_zero():
     w = _small(n_q_heads=16, n_kv_heads=2, eps=0.0, head_dim=128, feat_dim=128, lambda_=20,
                chunk=32, window=16)
-    _case(w, [("prefill", 160)], forced=True, unforced=True)
+    _case(w, [("prefill", 160)], modes=ALL, name="f32 GQA 8, eps 0")
 
 
 # ---------------------------------------------------------------- edge cases (bfloat16)
@@ -167,58 +183,85 @@ def _small_bf16(**kw):
 
 def test_bf16_no_window_no_cache_is_linear_attention():
     w = _small_bf16(window=0, lambda_=0, decode_interval=1)
-    _case(w, [("prefill", 64), ("decode", 16)], forced=False, unforced=True)
+    _case(w, [("prefill", 64), ("decode", 16)], modes=("free",), name="bf16 linear only")
 
 
 def test_bf16_chunk_longer_than_window_ragged_tiles():
     # partial cache and window tiles, query rows past the interval, and kept leaving
     # pairs that are later than some queries of their interval (chunk > window)
     w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6)
-    _case(w, [("prefill", 240), ("decode", 13)], forced=True, unforced=True)
+    _case(w, [("prefill", 240), ("decode", 13)], modes=ALL, name="bf16 chunk > window, ragged")
 
 
 def test_bf16_zero_window_with_cache():
     w = _small_bf16(window=0, lambda_=9, chunk=8, decode_interval=1)
-    _case(w, [("prefill", 80), ("decode", 5)], forced=True, unforced=True)
+    _case(w, [("prefill", 80), ("decode", 5)], modes=ALL, name="bf16 zero window")
 
 
 def test_bf16_gqa_group_of_eight():
     w = _small_bf16(n_q_heads=16, n_kv_heads=2, head_dim=128, feat_dim=128, lambda_=20, chunk=32, window=16)
-    _case(w, [("prefill", 160)], forced=True, unforced=True)
+    _case(w, [("prefill", 160)], modes=ALL, name="bf16 GQA 8")
+
+
+def test_bf16_token_by_token():
+    # C = C_dec = 1 on the tensor-core chain and attention and the streaming decode
+    w = _small_bf16(window=16, lambda_=24, chunk=1, decode_interval=1, n_q_heads=4, n_kv_heads=2)
+    _case(w, [("prefill", 96), ("decode", 32)], modes=ALL, name="bf16 token-by-token")
+
+
+def test_bf16_head_dim_32():
+    # head_dim 32 runs the SIMT attention beside the tensor-core chain
+    w = _small_bf16(head_dim=32, feat_dim=64, window=8, lambda_=40, chunk=16, decode_interval=8)
+    _case(w, [("prefill", 192), ("decode", 24)], modes=ALL, name="bf16 head_dim 32")
 
 
 # ---------------------------------------------------------------- bf16 workloads
 
+def _with_decode(w, T=None):
+    qp, kp, vp, _ = wl.make_inputs(w, part="prefill", T=T)
+    qd, kd, vd, _ = wl.make_inputs(w, part="decode")
+    return (np.concatenate([qp, qd], 1), np.concatenate([kp, kd], 1), np.concatenate([vp, vd], 1), None)
+
+
 def test_prefill_1b_full():
     w = wl.WORKLOADS["prefill-1b"]
-    res = _case(w, [("prefill", w.seq_len)], forced=True, unforced=True)
-    assert res["forced"]["exact"] + res["forced"]["under"] == res["forced"]["checked"]
+    res = _case(w, [("prefill", w.seq_len)], modes=ALL, scores=True)
+    f = res["forced"]
+    assert f["exact"] + f["under_margin_differ"] == f["intervals_checked"]
 
 
 def test_decode_batched_subset():
+    # 64 of the 512 streams: batches 0, 9, ..., 63 with all eight kv-heads
     w = wl.WORKLOADS["decode-batched"]
-    qp, kp, vp, _ = wl.make_inputs(w, part="prefill")
-    qd, kd, vd, _ = wl.make_inputs(w, part="decode")
-    inputs = (np.concatenate([qp, qd], 1), np.concatenate([kp, kd], 1),
-              np.concatenate([vp, vd], 1), None)
-    _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], forced=True,
-          subset=([0, 37], [0, 5]), seed_inputs=inputs)
+    _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], modes=("forced", "own"),
+          subset=(list(range(0, 64, 9)), list(range(8))), seed_inputs=_with_decode(w))
 
 
 def test_prefill_8b_sampled():
+    # 8 of the 32 streams (every batch, kv-heads 0 and 5), every 97th position
     w = wl.WORKLOADS["prefill-8b"]
-    _case(w, [("prefill", w.seq_len)], forced=True, subset=([1], [0, 6]), qmask_every=97)
+    _case(w, [("prefill", w.seq_len)], modes=("forced", "own"), subset=([0, 1, 2, 3], [0, 5]),
+          qmask_every=97, scores=True)
 
 
-def test_long_context_sampled():
-    w = wl.WORKLOADS["long-context"]
+def _long_context(name, every):
+    w = wl.WORKLOADS[name]
     T = w.seq_len
-    qp, kp, vp, _ = wl.make_inputs(w, part="prefill")
-    qd, kd, vd, _ = wl.make_inputs(w, part="decode")
-    inputs = (np.concatenate([qp, qd], 1), np.concatenate([kp, kd], 1),
-              np.concatenate([vp, vd], 1), None)
     plan = [("prefill", 16384)] * (T // 16384) + [("decode", w.decode_steps)]
-    _case(w, plan, forced=True, subset=([0], [3]), qmask_every=251, seed_inputs=inputs)
+    _case(w, plan, modes=("forced", "own"), qmask_every=every, seed_inputs=_with_decode(w),
+          scores=True)
+
+
+def test_long_context_64k():
+    _long_context("long-context", 251)
+
+
+def test_long_context_128k():
+    _long_context("long-context-128k", 503)
+
+
+def test_long_context_256k():
+    _long_context("long-context-256k", 1009)
 
 
 # ---------------------------------------------------------------- next rows: the pages' setting, C = 1
@@ -226,17 +269,14 @@ def test_long_context_sampled():
 def test_pages_cache_setting_prefill_then_decode():
     # window 256, sparse cache 256, 4K context with needles, then decode steps
     w = wl.WORKLOADS["pages-4k"]
-    qp, kp, vp, _ = wl.make_inputs(w, part="prefill")
-    qd, kd, vd, _ = wl.make_inputs(w, part="decode")
-    inputs = (np.concatenate([qp, qd], 1), np.concatenate([kp, kd], 1),
-              np.concatenate([vp, vd], 1), None)
-    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], forced=True, unforced=True,
-                seed_inputs=inputs)
-    assert res["forced"]["exact"] + res["forced"]["under"] == res["forced"]["checked"]
+    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], modes=ALL,
+                seed_inputs=_with_decode(w))
+    f = res["forced"]
+    assert f["exact"] + f["under_margin_differ"] == f["intervals_checked"]
 
 
 def test_token_by_token_intervals():
     # every token is its own update interval, in prefill (C = 1) and in decode (C_dec = 1)
     w = wl.WORKLOADS["token-by-token"]
-    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], forced=True, unforced=True)
-    assert res["unforced"]["exact"] == res["unforced"]["checked"]
+    res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], modes=ALL)
+    assert res["free"]["exact"] == res["free"]["intervals_checked"]

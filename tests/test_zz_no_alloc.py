@@ -4,8 +4,8 @@ or code running during CUDA graph capture). Its per-step temporaries live in a
 fixed array inside the library instead of the workspace.
 
 Checked through the C ABI against lola_decode_step on two calls in a row (one
-that opens an update interval, one inside it), with the fp32 output tolerance
-the parity tests use, and for the size limit. Collected last on purpose: if it
+that opens an update interval, one inside it), in float32 and bfloat16, with the
+output tolerances the parity tests use, and for the size limit. Collected last on purpose: if it
 fails, a run that stops at the first failure has already run everything else.
 """
 import numpy as np
@@ -32,17 +32,24 @@ def _rel(a, b):
     return np.linalg.norm(a - b) / np.linalg.norm(b)
 
 
-def test_static_decode_matches_decode_step_twice():
+TOL = {"f32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_static_decode_matches_decode_step_twice(dtype):
+    # bfloat16 runs the streaming decode kernel, whose fp32 query features also
+    # live in the library's array (after the partial sums)
     w = wl.Workload("noalloc", 12, batch=2, n_q_heads=4, n_kv_heads=2, head_dim=64, feat_dim=64,
                     window=16, lambda_=24, chunk=32, decode_interval=16, seq_len=64,
-                    decode_steps=2, dtype="f32")
+                    decode_steps=2, dtype=dtype)
     q, k, v, _ = wl.make_inputs(w, T=w.seq_len + 2)
     W = torch.from_numpy(wl.make_W(w))
     dev = torch.device("cuda")
     cfg = L.config_from_workload(w, max_prefill_tokens=w.seq_len)
     A = L.LolaState(cfg, W, dev)
     Bst = L.LolaState(cfg, W, dev)
-    qd, kd, vd = (torch.from_numpy(x).to(dev) for x in (q, k, v))
+    dt = torch.float32 if dtype == "f32" else torch.bfloat16
+    qd, kd, vd = (torch.from_numpy(x).to(dev, dt) for x in (q, k, v))
     T = w.seq_len
     for S in (A, Bst):
         S.prefill(qd[:, :T].contiguous(), kd[:, :T].contiguous(), vd[:, :T].contiguous())
@@ -57,7 +64,7 @@ def test_static_decode_matches_decode_step_twice():
                                   out_static.data_ptr(), stream)
         torch.cuda.synchronize()
         assert torch.isfinite(out_static).all()
-        assert _rel(out_static, out_ref) <= 1e-4
+        assert _rel(out_static, out_ref) <= TOL[dtype]
         assert L.lola_position(Bst.handle) == L.lola_position(A.handle) == t + 1
     A.sync()
     Bst.sync()
