@@ -290,6 +290,8 @@ def prefill_roofline(w, T, ms_step, phase_ms, steps, peaks, peak_src):
     # traffic of the dominant kernel (the phase with the most device time)
     dom = max((p for p in ("attn", "chain") if p in per_call), key=per_call.get, default="attn")
     traffic, tsrc = captured_traffic(dom, w.name)
+    if w != wl.WORKLOADS.get(w.name):
+        traffic, tsrc = None, "workload overridden on the command line (no capture for it)"
     return {"bound": "tensor", "kernel": f"whole prefill step (dominant kernel: {dom})",
             "achieved": round(ach, 3), "peak": burst, "unit": "TFLOP/s", "frac": round(ach / burst, 5),
             "frac_of_sustained": round(ach / sust, 5), "peak_sustained": sust,
@@ -324,6 +326,8 @@ def run_engine(args, ws, rank, local):
     torch.cuda.set_device(dev)
     peaks, peak_src = load_peaks()
     w = wl.WORKLOADS[args.workload]
+    if args.batch:
+        w = w.replace(batch=args.batch)
     T = w.seq_len
     q, k, v, _ = wl.make_inputs(w, T=T)
     W = wl.make_W(w)
@@ -446,6 +450,10 @@ def run_decode(args, name, ws, rank, dev, flush, peaks, peak_src):
     import torch
     from hybrid_linear_attention_lola_b200 import lola as L
     w = wl.WORKLOADS[name]
+    if args.decode_prefix:
+        w = w.replace(seq_len=args.decode_prefix)
+    if args.decode_steps:
+        w = w.replace(decode_steps=min(args.decode_steps, w.decode_steps))
     Tp, n_dec = w.seq_len, w.decode_steps
     q, k, v, _ = wl.make_inputs(w, T=Tp)
     qn, kn, vn, _ = wl.make_inputs(w, part="decode")
@@ -564,6 +572,12 @@ def main(argv=None):
     ap.add_argument("--decode-workload", default="decode-batched,long-context",
                     help="comma-separated decode workloads (or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batch", type=int, default=None,
+                    help="override the prefill workload's batch (smaller cases for profiling)")
+    ap.add_argument("--decode-prefix", type=int, default=None,
+                    help="override the decode workloads' prefilled prefix length")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="override the number of timed decode steps")
     args = ap.parse_args(argv)
     ws, rank, local = dist_setup()
     try:

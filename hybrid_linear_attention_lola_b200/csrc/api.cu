@@ -145,10 +145,14 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     if (!lola::decode_plan(dm)) return LOLA_ERR_INVALID_ARG;
     // the tensor-core chain selects into a cache (lambda = 0 runs on the SIMT chain) and
     // holds the state image as an N-contiguous operand of whole 64-column atoms
+    // It folds every unkept pair of an interval at once, so the prefill attention that
+    // reads its snapshots is the tensor-core one (it takes the state at the interval's
+    // end): the two run together or not at all.
     dm->tc_chain = (c->dtype == LOLA_BF16 && dm->lam > 0 && dm->d % 64 == 0 &&
-                    lola::chain_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
+                    lola::chain_tc_smem_bytes(*dm) <= 227 * 1024 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024)
+                       ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
-    dm->tc_attn = (dm->tc_chain && dm->d % 64 == 0 && lola::attn_tc_smem_bytes(*dm) <= 227 * 1024) ? 1 : 0;
+    dm->tc_attn = dm->tc_chain;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     if (c->dtype == LOLA_BF16 && lola::phi_tc_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     return LOLA_OK;
@@ -321,6 +325,7 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
     da.v = v;
     da.out = out;
     da.inject_ns = dm.dtype == LOLA_BF16 ? take_injection(st, 2) : 0;
+    da.state_ahead = dm.tc_chain;
     lola::DevState Sx = st->S;
     Sx.part = part;
     Sx.phiQd = phiq;

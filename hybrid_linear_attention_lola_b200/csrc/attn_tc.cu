@@ -9,11 +9,14 @@
 //
 // Setup, all at shift m = 0:
 //   phi(Q) = [softmax(QW), softmax(-QW)]  (Z = QW on the tensor cores);
-//   O = phi(Q) H'                         (readout of the interval's snapshot);
-//   l = phi(Q).s'                         (linear denominator, CUDA cores);
-//   O += G V_L, l += sum G                (folded pairs that left the window of the
-//                                          query inside this interval:
-//                                          G = phi(Q) phi(K_L)^T, masked per row).
+//   O = phi(Q) H1                         (readout of the interval's snapshot: the
+//                                          state at the interval's end, with every
+//                                          pair the interval folds);
+//   l = phi(Q).s1                         (linear denominator, CUDA cores);
+//   O -= G V_L, l -= sum G                (folded leaving pairs still inside the
+//                                          window of the query, which the softmax
+//                                          attends: G = phi(Q) phi(K_L)^T, masked
+//                                          per row).
 // Main loop, per 64-key tile of softmax keys (window keys, then cached keys):
 //   S = Q K^T on the tensor cores into one of two TMEM score buffers;
 //   P = e^{s - m} with the running shift m = max(0, max score), O rescaled in
@@ -387,8 +390,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = wait_mbar(&bar_x, xph & 1u, &okflag, S.err);
         ++xph;
     }
-    // ---- linear chunks: weights G where the pair left the window of the row's query and
-    //      was folded; O += W V_L and l += sum W (the rounded weights), still at m = 0
+    // ---- linear chunks: weights -G where the pair was folded but is still inside the
+    //      window of the row's query; O += W V_L and l += sum W (the rounded weights),
+    //      still at m = 0
     for (int c = 0; c < nlch && ok; ++c) {
         if (c > 0) {
             // the previous chunk's PV reads the P region and buffer 0
@@ -420,8 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 16; ++jj) {
                 const long long j = j0 + half * 32 + c0 + jj;
-                const bool lin = row_ok && j < jL1 && j <= p - eta && llf[(int)(j - (t0 - eta))] != 0;
-                w[jj] = lin ? gv[jj] : 0.f;
+                // folded, and still inside the window of the row's query: the snapshot holds
+                // its linear term, the softmax attends it, so the linear term comes off
+                const bool sub = row_ok && j < jL1 && j > p - eta && llf[(int)(j - (t0 - eta))] != 0;
+                w[jj] = sub ? -gv[jj] : 0.f;
             }
 #pragma unroll
             for (int h8 = 0; h8 < 16; h8 += 8) {

@@ -5,24 +5,30 @@
 //
 // The fp32 state lives in TMEM for the whole call: feature f of block
 // bk = f / 128 is TMEM lane f % 128, columns [bk*NBa, bk*NBa + d) hold H[f][:],
-// column bk*NBa + d holds s[f]. Both folds are tcgen05 MMAs that accumulate into
-// it, H_blk += Phi_F^T V_F and s_blk += Phi_F^T 1, with the tokens' phi rows and
-// value rows used as N-contiguous operands exactly as they are stored. After
+// column bk*NBa + d holds s[f]. A fold is a tcgen05 MMA chain that accumulates
+// into it, H_blk += Phi_F^T V_F and s_blk += Phi_F^T 1, with the tokens' phi rows
+// and value rows used as N-contiguous operands exactly as they are stored. After
 // each fold a bf16 image of the state is written to shared memory: H as an
 // N-contiguous [feature][value dim] operand and s as row 0 of a 16-row K-major
 // operand. The SRE of 128 candidates at a time is then one MMA chain
 // Phi_Q [H | s] into TMEM, and one thread per candidate finishes
-// || num / (den + eps) - v ||^2 with the candidate's value row staged in shared
-// memory. Scoring tiles arrive by TMA: a tile of 128 cached candidates is one
-// contiguous block of slot-ordered phi rows (the phi array's rows [0, lam)
-// mirror the cache slots; the kernel rewrites a slot's row when a new pair
-// takes it), loaded as one 128-row box per 64 features; a tile of leaving
-// pairs is contiguous too when they all come from this call (prefill) or from
-// one unwrapped run of the ring (decode); other tiles gather four rows per
-// instruction (tile::gather4). The fold operands are gathered by 16-byte copies. The kept set is the nK
-// smallest order-preserving keys (SRE bits
-// inverted, token index), found by an 8-pass radix select. Prefill mode stores
-// the image after the eviction fold as the interval's snapshot for attention.
+// || num / (den + eps) - v ||^2 with the candidate's value row.
+//
+// Scoring tiles arrive by TMA: a tile of 128 cached candidates is one contiguous
+// block of slot-ordered phi rows (the phi array's rows [0, lam) mirror the cache
+// slots; the kernel rewrites a slot's row when a new pair takes it), loaded as
+// one 128-row box per 64 features; a tile of leaving pairs is contiguous too when
+// they all come from this call (prefill) or from one unwrapped run of the ring
+// (decode); other tiles gather four rows per instruction (tile::gather4). The
+// fold operands are gathered by 16-byte copies.
+//
+// The kept set is the nK smallest order-preserving keys (SRE bits inverted,
+// token index), found by an 8-pass radix select. Every pair that is not kept --
+// evicted cached pairs and leaving pairs alike -- folds right after the
+// selection, in one pass, so the state becomes the state at the interval's end.
+// Prefill mode stores its image as the interval's snapshot for the attention,
+// which subtracts the linear terms of the folded leaving pairs that are still
+// inside a query's window (the softmax attends them there).
 #include "lola_internal.cuh"
 #include "umma.cuh"
 
@@ -461,7 +467,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     for (int i = tid; i < Lmax; i += kThreads) lf[i] = i < a.pend_n ? S.pend[(size_t)st * Lmax + i] : 0;
-    long long pend_lo = a.pend_lo;
     int pend_n = a.pend_n;
     __syncthreads();
 
@@ -483,18 +488,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
             if (!(ok = okflag != 0)) break;
         }
-        // 1. fold the previous interval's leaving pairs that were not kept
-        if (pend_n > 0) {
-            const int nf = scan_excl(lf, rank, pend_n, scal);
-            for (int i = tid; i < pend_n; i += kThreads)
-                if (lf[i]) lst[rank[i]] = src.tok2vrow(pend_lo + i);
-            __syncthreads();
-            if (nf > 0) {
-                if (!(ok = fold_tc(c, lst, nf, phi_st, src, st))) break;
-                refresh_image(c);
-            }
-        }
-
         unsigned *keys = (ci & 1) ? keys1 : keys0;
         // 2. score the candidates (cache slots, then pairs leaving in [t0, t1))
         const long long Llo = t0 - eta > 0 ? t0 - eta : 0;
@@ -686,8 +679,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
 
-        // 4a. evicted cached pairs: fold now (the state this interval's queries read)
-        for (int i = tid; i < nS; i += kThreads) flag[i] = keep[i] ? 0 : 1;
+        // 4a. every pair that is not kept -- evicted cached pairs and leaving pairs --
+        //     folds now, in one pass: the state becomes the state at the interval's end
+        for (int i = tid; i < nQ; i += kThreads) flag[i] = keep[i] ? 0 : 1;
         __syncthreads();
         const int nE = scan_excl(flag, rank, nS, scal);
         for (int i = tid; i < nS; i += kThreads) {
@@ -698,8 +692,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int r = nE + tid; r < nE + (lam - nS); r += kThreads) freeSlot[r] = (short)(nS + (r - nE));
         __syncthreads();
-        if (nE > 0) {
-            if (!(ok = fold_tc(c, lst, nE, phi_st, src, st))) break;
+        const int nLf = scan_excl(flag + nS, rank, nL, scal);
+        for (int i = tid; i < nL; i += kThreads)
+            if (flag[nS + i]) lst[nE + rank[i]] = src.tok2vrow(Llo + i);
+        __syncthreads();
+        if (nE + nLf > 0) {
+            if (!(ok = fold_tc(c, lst, nE + nLf, phi_st, src, st))) break;
             refresh_image(c);
         }
         if (a.mode == 0 && P.snapImg != nullptr && tid == 0 && lead) {
@@ -788,7 +786,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
         for (int i = tid; i < nL; i += kThreads) lf[i] = keep[nS + i] ? 0 : 1;
-        pend_lo = Llo;
         pend_n = nL;
         nS = nK;
         __syncthreads();

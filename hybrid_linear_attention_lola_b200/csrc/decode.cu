@@ -34,10 +34,16 @@ constexpr int kMaxG = 8;
 constexpr uint64_t kWaitNs = 2000000000ull;   // 2 s per staging-buffer wait
 constexpr int kSMs = 148;
 constexpr int kMinPer = 8;   // items per warp of the streaming kernel, at least (many streams)
+#ifndef LOLA_DEC_MINPER_FLOOR
+#define LOLA_DEC_MINPER_FLOOR 1
+#endif
+constexpr int kMinPerFloor = LOLA_DEC_MINPER_FLOOR;   // ... and with few streams
 #ifndef LOLA_DECODE_BUFS
 #define LOLA_DECODE_BUFS 2
 #endif
 constexpr int kStreamBufs = LOLA_DECODE_BUFS;   // staging buffers per warp of the streaming kernel
+constexpr int kFewBufs = 4;   // ... when the streams are too few to fill the GPU with warps
+constexpr int kFewPer = 6;    // items per warp, at least, in that case
 
 // ---------------------------------------------------------------- shared memory plan
 
@@ -115,8 +121,11 @@ template <int VN> __device__ __forceinline__ int qidx(int x) { return qoff<VN>(x
 
 // Work items of one stream for the step at position p (identical in every CTA):
 //   [0, nkc)            32 softmax keys: cache slots [0, nS), then window tokens [wlo, p]
-//   [nkc, nkc + nlc)    16 linear-band tokens of [jlo, lhi) (left the window this
-//                       interval; folded ones are linear, kept ones are skipped)
+//   [nkc, nkc + nlc)    16 linear-band tokens of [jlo, lhi), pairs leaving the window
+//                       this interval (kept ones are skipped): with state_ahead the
+//                       folded ones still inside p's window (the state holds their
+//                       linear terms, which come off; the softmax attends them),
+//                       otherwise the folded ones that left it (their terms add)
 //   [nkc + nlc, ni)     hrows feature rows of the state (H, s)
 // With tma, softmax keys come in aligned 32-row blocks instead: cache slots
 // [32c, 32c + 32) (c < ncc), then the blocks of 32 ring slots the window
@@ -132,10 +141,18 @@ __host__ __device__ __forceinline__ Items make_items(const Dims &dm, const Decod
 {
     Items it;
     const long long p = a.pos;
-    it.jlo = a.t0 - dm.eta > 0 ? a.t0 - dm.eta : 0;
-    it.wlo = p - dm.eta + 1 > it.jlo ? p - dm.eta + 1 : it.jlo;
-    it.lhi = a.L_hi < it.wlo ? a.L_hi : it.wlo;
-    if (it.lhi < it.jlo) it.lhi = it.jlo;
+    const long long jl = a.t0 - dm.eta > 0 ? a.t0 - dm.eta : 0;   // first pair leaving in the interval
+    it.wlo = p - dm.eta + 1 > jl ? p - dm.eta + 1 : jl;
+    if (a.state_ahead) {
+        // folded pairs still inside the window: their linear terms come off the state
+        it.jlo = it.wlo;
+        it.lhi = a.L_hi > it.jlo ? a.L_hi : it.jlo;
+    } else {
+        // folded pairs that left the window: their linear terms add to the state
+        it.jlo = jl;
+        it.lhi = a.L_hi < it.wlo ? a.L_hi : it.wlo;
+        if (it.lhi < it.jlo) it.lhi = it.jlo;
+    }
     const int nwin = (int)(p - it.wlo + 1);
     it.nsoft = a.nS + nwin;
     it.ncc = (a.nS + 31) / 32;
@@ -497,7 +514,7 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
             for (int h = 0; h < kMaxG; ++h) {
                 if (h < g) {
                     gl[h] += __shfl_xor_sync(0xffffffffu, gl[h], 16);
-                    if (hf == 0) pws[h * 32 + kk] = gl[h];
+                    if (hf == 0) pws[h * 32 + kk] = a.state_ahead ? -gl[h] : gl[h];
                 }
             }
             __syncwarp();
@@ -689,6 +706,21 @@ __device__ __forceinline__ uint32_t pack2(float lo, float hi)
     return r;
 }
 // byte offset of 16-byte chunk c of row r in a [32 rows][CPR chunks] swizzled tile
+// DPL consecutive floats (16-, 8- or 4-byte aligned) through L2
+template <int DPL> __device__ __forceinline__ void ld_dpl(const float *p, float (&v)[DPL])
+{
+    if constexpr (DPL == 4) {
+        const float4 x = __ldcg((const float4 *)p);
+        v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+    } else if constexpr (DPL == 2) {
+        const float2 x = __ldcg((const float2 *)p);
+        v[0] = x.x; v[1] = x.y;
+    } else {
+#pragma unroll
+        for (int u = 0; u < DPL; ++u) v[u] = __ldcg(p + u);
+    }
+}
+
 template <int CPR> __device__ __forceinline__ uint32_t swz(int r, int c)
 {
     return (uint32_t)((c >> 3) * 32 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
@@ -744,7 +776,7 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, D
 // a warp leaves a stream it writes its partial (m, l, linear den, softmax num,
 // linear num per head); the warp that writes a stream's last partial merges them
 // (a per-stream counter).
-template <int DPL, int G>
+template <int DPL, int G, int NST>
 __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S, DecodeArgs a, int per, int wbytes,
                                                              const __grid_constant__ DecMaps maps)
 {
@@ -756,7 +788,6 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     constexpr int KS_ = d / 16;                        // k-steps of Q K^T
     constexpr int ND = d / 8;                          // n-tiles of P V (8 value dims each)
     constexpr int HR = 16;                             // state rows per item
-    constexpr int NST = kStreamBufs;                   // staging buffers per warp
     constexpr int RS = d * E + 16;                     // padded row stride of key / value tiles (bulk path)
     const bool tma = dm.dec_tma != 0;
     // bytes of a 32-row key (or value) tile: swizzled 128-byte rows (TMA path) or padded rows
@@ -976,23 +1007,37 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         if (prev != nparts - 1) return;
         // this warp wrote the stream's last partial: merge (online-softmax identity) and write out
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
-        for (int h = 0; h < g; ++h) {
+        float Mh[G], Lsh[G], LDh[G];
+#pragma unroll
+        for (int h = 0; h < G; ++h) {
+            Mh[h] = 0.f;
+            Lsh[h] = LDh[h] = 0.f;
+            if (h >= g) continue;
             // lane q holds partials q, q + 32, ...: maximum shift and the scalar sums in parallel
-            float M = 0.f;
-            for (int q2 = lane; q2 < nparts; q2 += 32) M = fmaxf(M, __ldcg(base + ((size_t)q2 * g + h) * rec));
-            M = warp_max(M);
-            float Ls = 0.f, LD = 0.f;
+            for (int q2 = lane; q2 < nparts; q2 += 32) Mh[h] = fmaxf(Mh[h], __ldcg(base + ((size_t)q2 * g + h) * rec));
+            Mh[h] = warp_max(Mh[h]);
             for (int q2 = lane; q2 < nparts; q2 += 32) {
                 const float *pr = base + ((size_t)q2 * g + h) * rec;
-                Ls = fmaf(__expf(__ldcg(pr) - M), __ldcg(pr + 1), Ls);
-                LD += __ldcg(pr + 2);
+                Lsh[h] = fmaf(__expf(__ldcg(pr) - Mh[h]), __ldcg(pr + 1), Lsh[h]);
+                LDh[h] += __ldcg(pr + 2);
             }
-            Ls = warp_sum(Ls);
-            LD = warp_sum(LD);
-            // value columns: lane owns dims [lane*DPL, lane*DPL + DPL); loads of 4 partials in flight
+            Lsh[h] = warp_sum(Lsh[h]);
+            LDh[h] = warp_sum(LDh[h]);
+        }
+        // value columns: lane owns dims [lane*DPL, lane*DPL + DPL); one head at a time, four
+        // partials in flight, DPL floats per load
+        for (int h = 0; h < g; ++h) {
             float O[DPL], LO[DPL];
 #pragma unroll
             for (int u = 0; u < DPL; ++u) O[u] = LO[u] = 0.f;
+            float M = 0.f, Ls = 0.f, LD = 0.f;
+#pragma unroll
+            for (int h2 = 0; h2 < G; ++h2)
+                if (h2 == h) {
+                    M = Mh[h2];
+                    Ls = Lsh[h2];
+                    LD = LDh[h2];
+                }
             for (int q0 = 0; q0 < nparts; q0 += 4) {
                 float mv[4], ov[4][DPL], lv[4][DPL];
 #pragma unroll
@@ -1000,11 +1045,8 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                     const int q2 = q0 + t < nparts ? q0 + t : q0;
                     const float *pr = base + ((size_t)q2 * g + h) * rec;
                     mv[t] = __ldcg(pr);
-#pragma unroll
-                    for (int u = 0; u < DPL; ++u) {
-                        ov[t][u] = __ldcg(pr + 4 + lane * DPL + u);
-                        lv[t][u] = __ldcg(pr + 4 + d + lane * DPL + u);
-                    }
+                    ld_dpl<DPL>(pr + 4 + lane * DPL, ov[t]);
+                    ld_dpl<DPL>(pr + 4 + d + lane * DPL, lv[t]);
                 }
 #pragma unroll
                 for (int t = 0; t < 4; ++t) {
@@ -1185,7 +1227,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
             for (int h = 0; h < G; ++h) {
                 if (h < g) {
                     gl[h] += __shfl_xor_sync(0xffffffffu, gl[h], 16);
-                    if (hf == 0) pws[h * 32 + kk] = lin ? gl[h] : 0.f;
+                    if (hf == 0) pws[h * 32 + kk] = lin ? (a.state_ahead ? -gl[h] : gl[h]) : 0.f;
                 }
             }
             __syncwarp();
@@ -1238,7 +1280,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
 // bytes of shared memory per warp of decode_stream_kernel
 inline int stream_warp_bytes(const Dims &dm, int G)
 {
-    const size_t b = (size_t)kStreamBufs * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
+    const size_t b = (size_t)dm.dec_nst * dm.dec_sb + (size_t)G * (dm.D + dm.D / 8) * 4 + (size_t)G * 32 * 4 + 256 + 64;
     return (int)((b + 1023) / 1024 * 1024);   // every warp's buffers start 1024-byte aligned
 }
 
@@ -1291,7 +1333,18 @@ bool decode_plan(Dims *dm)
         size_t sb = sb_keys > sb_h ? sb_keys : sb_h;
         if (sb_lin > sb) sb = sb_lin;
         dm->dec_sb = (int)((sb + 1023) / 1024 * 1024);
-        dm->dec_nst = kStreamBufs;
+        // aligned 32-row blocks: the cache and up to two more blocks for the window
+        const long long items = ((long long)dm->lam + 31) / 32 + (dm->eta + 31) / 32 + 2 +
+                                (dm->Cdec + 15) / 16 + dm->D / 16;
+        // items per warp that would spread the streams over every SM; with fewer streams
+        // than that, each warp keeps more copies in flight and takes at least kFewPer items
+        // (the partials of a stream are merged by one warp: fewer, larger partials)
+        long long mp = (long long)dm->ns * items / ((long long)kSMs * 8);
+        const bool few = mp < kMinPer;
+        dm->dec_nst = few ? kFewBufs : kStreamBufs;
+        if (few && mp < kFewPer) mp = kFewPer;
+        if (mp < kMinPerFloor) mp = kMinPerFloor;
+        if (mp > kMinPer) mp = kMinPer;
         const int G = dm->g <= 1 ? 1 : dm->g <= 2 ? 2 : dm->g <= 4 ? 4 : 8;
         // warps per CTA: the most resident warps per SM (shared memory, ~160 registers per thread)
         const size_t wb = (size_t)stream_warp_bytes(*dm, G);
@@ -1308,13 +1361,6 @@ bool decode_plan(Dims *dm)
             }
         }
         if (dm->dec_nw == 0) return false;
-        // aligned 32-row blocks: the cache and up to two more blocks for the window
-        const long long items = ((long long)dm->lam + 31) / 32 + (dm->eta + 31) / 32 + 2 +
-                                (dm->Cdec + 15) / 16 + dm->D / 16;
-        // with few streams every warp takes fewer items, so that the whole GPU streams
-        long long mp = (long long)dm->ns * items / ((long long)kSMs * 8);
-        if (mp < 1) mp = 1;
-        if (mp > kMinPer) mp = kMinPer;
         dm->dec_minper = (int)mp;
         dm->nsplit = (int)((items + mp - 1) / mp + 1);
         return true;
@@ -1407,15 +1453,20 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
         if (per < dm.dec_minper) per = dm.dec_minper;
         const long long nwarps = (total + per - 1) / per;
         const int grid = (int)((nwarps + nw - 1) / nw);
-#define LOLA_STREAM(DPL, GG)                                                                       \
+#define LOLA_STREAM_N(DPL, GG, NB)                                                                 \
     do {                                                                                           \
         static size_t attr = 0;                                                                    \
         if (smem > attr) {                                                                         \
-            cudaFuncSetAttribute(decode_stream_kernel<DPL, GG>,                                    \
+            cudaFuncSetAttribute(decode_stream_kernel<DPL, GG, NB>,                                \
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);          \
             attr = smem;                                                                           \
         }                                                                                          \
-        decode_stream_kernel<DPL, GG><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb, mp); \
+        decode_stream_kernel<DPL, GG, NB><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb, mp); \
+    } while (0)
+#define LOLA_STREAM(DPL, GG)                                                                       \
+    do {                                                                                           \
+        if (dm.dec_nst == kFewBufs) LOLA_STREAM_N(DPL, GG, kFewBufs);                              \
+        else LOLA_STREAM_N(DPL, GG, kStreamBufs);                                                  \
     } while (0)
 #define LOLA_STREAM_G(DPL)                                                                         \
     do {                                                                                           \
@@ -1429,6 +1480,7 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
         else LOLA_STREAM_G(4);
 #undef LOLA_STREAM_G
 #undef LOLA_STREAM
+#undef LOLA_STREAM_N
         return;
     }
     dim3 grid(dm.nsplit, dm.ns);

@@ -288,6 +288,8 @@ struct DecodeArgs {
     void *out;
     unsigned long long inject_ns;   // test hook: > 0 makes the streaming kernel's first warp wait
                                     // this long on an mbarrier nothing arrives at (timeout)
+    int state_ahead;        // 1: the state already holds the open interval's folded leaving pairs
+                            // (tensor-core chain); 0: they fold at the next interval's start
 };
 // Decode launch shape: splits per stream, warps per CTA, staging buffers and
 // their size (fills dm.nsplit, dec_nw, dec_nst, dec_sb); returns false if no
