@@ -30,7 +30,10 @@ _lib = None
 class OracleCfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("D", ctypes.c_int32), ("eta", ctypes.c_int32),
-                ("lam", ctypes.c_int32), ("eps", ctypes.c_double)]
+                ("lam", ctypes.c_int32), ("eps", ctypes.c_double), ("scorer", ctypes.c_int32)]
+
+
+SCORERS = {"sre": 0, "attention-weight": 1, "softmax-error": 2, "fifo": 3}
 
 
 def build(force: bool = False) -> str:
@@ -103,9 +106,11 @@ def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: i
         lambda_: int, intervals: Sequence[int], eps: float = 1e-6,
         qmask: Optional[np.ndarray] = None, want_cands: bool = False,
         want_state: bool = False, threads: Optional[int] = None,
-        compact: bool = False) -> OracleResult:
+        compact: bool = False, scorer: str = "sre") -> OracleResult:
     """Runs the recurrence from an empty state over tokens split into `intervals`.
-    compact=True (with qmask) stores only the outputs of the masked positions."""
+    compact=True (with qmask) stores only the outputs of the masked positions.
+    scorer: "sre" (the method), or the alternatives "attention-weight",
+    "softmax-error" and "fifo" (see lola_oracle.c); cand_sre then logs that score."""
     lib = _load()
     q = np.ascontiguousarray(q, np.float32)
     k = np.ascontiguousarray(k, np.float32)
@@ -117,7 +122,7 @@ def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: i
     ints = np.ascontiguousarray(np.asarray(intervals, np.int32))
     n_int = len(ints)
     ns = B * Hkv
-    cfg = OracleCfg(B, Hq, Hkv, d, D, window, lambda_, eps)
+    cfg = OracleCfg(B, Hq, Hkv, d, D, window, lambda_, eps, SCORERS[scorer])
     r = OracleResult()
     out_row = None
     n_out = T

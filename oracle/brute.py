@@ -9,7 +9,8 @@ summary, sections "Het Self-Recall Error (SRE) Mechanisme" and
     t0 it is rebuilt from scratch as the sum over the folded set
     F* = { j < t0 - eta } minus the sparse cache S, i.e. H = sum phi(k_j) v_j^T
     and s = sum phi(k_j) over F*.
-  * Selection sorts the candidates with Python's sort on (-SRE, index).
+  * Selection sorts the candidates with Python's sort on (-score, index). The
+    score is the SRE, or one of the ablation scores (see `scores`).
   * Each output row classifies every earlier key j <= p directly: softmax when
     j is inside the window of p (j > p - eta) or j is in the kept set of the
     interval; linear (weight phi(q).phi(k_j)) otherwise. The row is
@@ -28,8 +29,43 @@ def phi_rows(x: np.ndarray, W: np.ndarray) -> np.ndarray:
     return np.concatenate([softmax(z, axis=-1), softmax(-z, axis=-1)], axis=-1)
 
 
-def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6):
-    """Returns (out [B,T,Hq,d], kept list per interval per stream, sre dict per interval)."""
+def scores(scorer, cands, qrows, keys, phik, H, s, vv, eps):
+    """Score of every candidate token, NumPy: "sre" -- ||phi(k)H/(phi(k)s+eps) - v||^2;
+    "attention-weight" -- over the heads of the group, the softmax (over the
+    candidates) of q.k/sqrt(d) for the interval's first query; "softmax-error" --
+    over the heads, the squared gap between that weight and phi(q).phi(k) divided
+    by its sum over the candidates; "fifo" -- the token index."""
+    d = vv.shape[1]
+    if not cands:
+        return {}
+    if scorer == "fifo":
+        return {j: float(j) for j in cands}
+    if scorer == "sre":
+        out = {}
+        for j in cands:
+            den = float(phik[j] @ s) + eps
+            pred = (phik[j] @ H) / den if den != 0.0 else np.zeros(d)
+            out[j] = float(np.sum((pred - vv[j]) ** 2))
+        return out
+    tot = np.zeros(len(cands))
+    for qh in qrows:
+        a = softmax(np.array([float(qh @ keys[j]) for j in cands]) / np.sqrt(d))
+        if scorer == "attention-weight":
+            tot += a
+        else:
+            pq = phi_rows(qh[None, :], _W_for_scores)[0]
+            lw = np.array([float(pq @ phik[j]) for j in cands])
+            tot += (a - lw / lw.sum()) ** 2
+    return {j: float(x) for j, x in zip(cands, tot)}
+
+
+_W_for_scores = None
+
+
+def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6, scorer: str = "sre"):
+    """Returns (out [B,T,Hq,d], kept list per interval per stream, score dict per interval)."""
+    global _W_for_scores
+    _W_for_scores = np.asarray(W, np.float64)
     q = np.asarray(q, np.float64)
     k = np.asarray(k, np.float64)
     v = np.asarray(v, np.float64)
@@ -57,11 +93,8 @@ def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6):
                 s = sum((pk[j] for j in folded), np.zeros(pk.shape[1]))
                 leaving = [j for j in range(T) if t0 <= j + eta < t1]
                 cands = sorted(cache) + leaving
-                sres = {}
-                for j in cands:
-                    den = float(pk[j] @ s) + eps
-                    pred = (pk[j] @ H) / den if den != 0.0 else np.zeros(d)
-                    sres[j] = float(np.sum((pred - vv[j]) ** 2))
+                qrows = [q[b, t0, hk * g + r, :] for r in range(g)]
+                sres = scores(scorer, cands, qrows, k[b, :, hk, :], pk, H, s, vv, eps)
                 order = sorted(cands, key=lambda j: (-sres[j], j))
                 K = set(order[:min(lam, len(order))])
                 kept_log[-1].append(sorted(K))

@@ -21,7 +21,15 @@
  *     2. Every candidate is scored against the state at t0 by the Self-Recall
  *        Error SRE(k,v|H,s) = || phi(k)^T H / (phi(k)^T s + eps) - v ||^2
  *        (the SRE equation of the "Self-Recall Error" section; eps added to the
- *        denominator).
+ *        denominator). The ablations of the "Belangrijkste bijdragen" and
+ *        "Ablaties" sections swap this score for the magnitude of attention
+ *        weights or a softmax-approximation error, and the inference strategy
+ *        mentions a FIFO structure; scorer 1 / 2 / 3 select those (this build's
+ *        readings: the softmax weight of the candidate for the interval's first
+ *        query, summed over the group's heads; the squared gap between that
+ *        weight and the linear-attention weight phi(q).phi(k) normalised over the
+ *        candidates, summed over heads; the token index, i.e. the most recent
+ *        pairs stay).
  *     3. The min(lambda, |Q|) candidates of highest SRE stay in the cache
  *        (ties: lower token index stays); the rest, F, are folded.
  *     4. E = S n F is folded at the interval start: H' = H + sum phi(k) v^T,
@@ -49,6 +57,7 @@
 typedef struct {
     int32_t B, Hq, Hkv, d, D, eta, lam;
     double eps;
+    int32_t scorer; /* 0 SRE, 1 attention weight, 2 softmax-approximation error, 3 recency */
 } oracle_cfg;
 
 /* phi(x) = [softmax(x W), softmax(-x W)]  (x: d, W: d x D/2 row-major, out: D) */
@@ -188,6 +197,7 @@ static void run_stream(job_t *J, int st)
     uint8_t *lfold = (uint8_t *)calloc((size_t)T, 1); /* j in L n F for this interval */
     double *phiq = (double *)malloc(sizeof(double) * (size_t)D);
     double *sc = (double *)malloc(sizeof(double) * (size_t)(lam + eta + maxlen + 1));
+    double *sc2 = (double *)malloc(sizeof(double) * (size_t)(lam + maxlen + 1));
     int32_t *Aset = (int32_t *)malloc(sizeof(int32_t) * (size_t)(lam + eta + maxlen + 1));
     double *num = (double *)malloc(sizeof(double) * (size_t)d);
     double *lin = (double *)malloc(sizeof(double) * (size_t)d);
@@ -200,17 +210,57 @@ static void run_stream(job_t *J, int st)
         if (Llo < 0) Llo = 0;
         if (Lhi < Llo) Lhi = Llo;
         int nQ = 0;
-        /* 2. Self-Recall Error against the state at t0 */
-        for (int i = 0; i < nS; ++i) {
-            int j = S[i];
-            cand[nQ].tok = j;
-            cand[nQ].sre = oracle_sre(phik + (size_t)j * D, vd + (size_t)j * d, H, s, d, D, eps);
-            ++nQ;
-        }
-        for (int j = Llo; j < Lhi; ++j) {
-            cand[nQ].tok = j;
-            cand[nQ].sre = oracle_sre(phik + (size_t)j * D, vd + (size_t)j * d, H, s, d, D, eps);
-            ++nQ;
+        for (int i = 0; i < nS; ++i) cand[nQ++].tok = S[i];
+        for (int j = Llo; j < Lhi; ++j) cand[nQ++].tok = j;
+        /* 2. score every candidate (the highest scores stay cached) */
+        if (cfg->scorer == 0) {
+            /* Self-Recall Error against the state at t0 */
+            for (int c = 0; c < nQ; ++c) {
+                const int j = cand[c].tok;
+                cand[c].sre = oracle_sre(phik + (size_t)j * D, vd + (size_t)j * d, H, s, d, D, eps);
+            }
+        } else if (cfg->scorer == 3) {
+            /* recency: the most recent pairs stay (a first-in first-out cache) */
+            for (int c = 0; c < nQ; ++c) cand[c].sre = (double)cand[c].tok;
+        } else {
+            /* the interval's first query, every head of the group: a = softmax over the
+               candidates of q.k / sqrt(d); scorer 1 keeps the largest sum over heads of a,
+               scorer 2 the largest sum over heads of (a - b)^2, where b is the linear
+               attention weight phi(q).phi(k) normalised over the candidates */
+            for (int c = 0; c < nQ; ++c) cand[c].sre = 0.0;
+            for (int r = 0; r < g; ++r) {
+                const float *qsrc = J->q + (((size_t)b * T + t0) * Hq + hk * g + r) * d;
+                double qv[1024];
+                for (int c = 0; c < d; ++c) qv[c] = qsrc[c];
+                double mx = -INFINITY, z = 0.0, u = 0.0;
+                for (int c = 0; c < nQ; ++c) {
+                    const double *kk = kd + (size_t)cand[c].tok * d;
+                    double dot = 0.0;
+                    for (int e = 0; e < d; ++e) dot += qv[e] * kk[e];
+                    sc[c] = dot * scale;
+                    if (sc[c] > mx) mx = sc[c];
+                }
+                for (int c = 0; c < nQ; ++c) z += exp(sc[c] - mx);
+                if (cfg->scorer == 2) {
+                    oracle_phi(qv, J->W, d, D, phiq);
+                    for (int c = 0; c < nQ; ++c) {
+                        const double *pk = phik + (size_t)cand[c].tok * D;
+                        double w = 0.0;
+                        for (int e = 0; e < D; ++e) w += phiq[e] * pk[e];
+                        sc2[c] = w;
+                        u += w;
+                    }
+                }
+                for (int c = 0; c < nQ; ++c) {
+                    const double a = exp(sc[c] - mx) / z;
+                    if (cfg->scorer == 1) {
+                        cand[c].sre += a;
+                    } else {
+                        const double e2 = a - sc2[c] / u;
+                        cand[c].sre += e2 * e2;
+                    }
+                }
+            }
         }
         size_t logi = (size_t)ci * nstreams + st;
         if (J->cand_tok && J->cand_sre) {
@@ -336,7 +386,7 @@ static void run_stream(job_t *J, int st)
 
     free(kd); free(vd); free(phik); free(H); free(s); free(Hp); free(sp);
     free(status); free(S); free(cand); free(keep); free(lfold); free(phiq);
-    free(sc); free(Aset); free(num); free(lin);
+    free(sc); free(sc2); free(Aset); free(num); free(lin);
 }
 
 static void *worker(void *arg)

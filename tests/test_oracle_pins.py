@@ -341,3 +341,56 @@ def test_open_last_interval_matches_bruteforce():
     out_b, kept_b, _ = brute.run(q, k, v, W, window=eta, lambda_=lam, intervals=ints)
     np.testing.assert_allclose(r.out, out_b, rtol=1e-10, atol=1e-12)
     assert [t for t in r.kept[-1, 1] if t >= 0] == kept_b[-1][1]
+
+
+# ---------------------------------------------------------------- ablation scorers and FIFO
+
+@pytest.mark.parametrize("scorer", ["attention-weight", "softmax-error", "fifo"])
+@pytest.mark.parametrize("eta,lam,ints", [(5, 4, [4] * 10), (3, 6, [8] * 5), (4, 5, [4] * 4 + [1] * 24)])
+def test_scorers_match_set_based_bruteforce(scorer, eta, lam, ints):
+    T = sum(ints)
+    B, Hq, Hkv, d, D = 1, 4, 2, 8, 8
+    q, k, v, W = _qkvw(B, T, Hq, Hkv, d, D, 170 + eta * 7 + lam)
+    eps = 1e-6
+    r = oracle.run(q, k, v, W, window=eta, lambda_=lam, intervals=ints, eps=eps, want_cands=True,
+                   scorer=scorer)
+    out_b, kept_b, sc_b = brute.run(q, k, v, W, window=eta, lambda_=lam, intervals=ints, eps=eps,
+                                    scorer=scorer)
+    np.testing.assert_allclose(r.out, out_b, rtol=1e-10, atol=1e-12)
+    for ci in range(len(ints)):
+        for st in range(B * Hkv):
+            assert [t for t in r.kept[ci, st] if t >= 0] == kept_b[ci][st], (ci, st)
+            for t, s in zip(r.cand_tok[ci, st], r.cand_sre[ci, st]):
+                if t >= 0:
+                    assert abs(s - sc_b[ci][st][t]) <= 1e-10 * max(1.0, abs(s))
+
+
+@pytest.mark.parametrize("eta,lam", [(5, 4), (2, 7), (0, 3)])
+def test_fifo_token_by_token_is_a_wider_window(eta, lam):
+    # keeping the most recent pairs with one-token intervals leaves exactly the
+    # last eta + lam pairs in softmax and everything older in the linear state:
+    # the no-cache direct form with window eta + lam
+    B, T, Hq, Hkv, d, D = 1, 41, 4, 2, 8, 8
+    q, k, v, W = _qkvw(B, T, Hq, Hkv, d, D, 190 + eta + lam)
+    r = oracle.run(q, k, v, W, window=eta, lambda_=lam, intervals=[1] * T, eps=1e-6, scorer="fifo")
+    np.testing.assert_allclose(r.out, _window_plus_linear(q, k, v, W, eta + lam, 1e-6),
+                               rtol=1e-11, atol=1e-13)
+
+
+def test_attention_weight_one_head_keeps_the_largest_logits():
+    # with one query head per kv-head the softmax is monotone in q.k: the kept set
+    # of every interval is the lambda candidates with the largest q_t0 . k
+    B, T, Hq, Hkv, d, D = 1, 60, 2, 2, 8, 8
+    q, k, v, W = _qkvw(B, T, Hq, Hkv, d, D, 211)
+    ints, lam = [6] * 10, 5
+    r = oracle.run(q, k, v, W, window=4, lambda_=lam, intervals=ints, eps=1e-6, want_cands=True,
+                   scorer="attention-weight")
+    t0 = 0
+    for ci, C in enumerate(ints):
+        for st in range(Hkv):
+            toks = [int(t) for t in r.cand_tok[ci, st] if t >= 0]
+            if len(toks) > lam:
+                logit = {j: float(q[0, t0, st] @ k[0, j, st]) for j in toks}
+                want = sorted(sorted(toks, key=lambda j: (-logit[j], j))[:lam])
+                assert [int(t) for t in r.kept[ci, st] if t >= 0] == want
+        t0 += C
