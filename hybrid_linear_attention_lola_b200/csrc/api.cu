@@ -120,6 +120,8 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     if (c->decode_interval < 1 || c->decode_interval > 256 || c->decode_interval > c->window + 1)
         return LOLA_ERR_INVALID_ARG;
     if (!(c->eps >= 0.f)) return LOLA_ERR_INVALID_ARG;
+    if (c->scorer < LOLA_SCORE_SRE || c->scorer > LOLA_SCORE_RECENCY) return LOLA_ERR_INVALID_ARG;
+    if (c->w_per_kv_head != 0 && c->w_per_kv_head != 1) return LOLA_ERR_INVALID_ARG;
     const int nmax = c->max_prefill_tokens > 0 ? c->max_prefill_tokens : c->chunk;
     if (nmax % c->chunk != 0) return LOLA_ERR_INVALID_ARG;
     dm->B = c->batch;
@@ -142,6 +144,8 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
     dm->Nmax = nmax;
     dm->mmax = nmax / c->chunk;
     dm->eps = c->eps;
+    dm->scorer = c->scorer;
+    dm->nW = c->w_per_kv_head ? c->n_kv_heads : 1;
     if (!lola::decode_plan(dm)) return LOLA_ERR_INVALID_ARG;
     // the tensor-core chain selects into a cache (lambda = 0 runs on the SIMT chain) and
     // holds the state image as an N-contiguous operand of whole 64-column atoms
@@ -181,8 +185,8 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.KR = take(ns * dm.R * dm.d * e);
     s.VR = take(ns * dm.R * dm.d * e);
     s.pend = (uint8_t *)take(ns * dm.Lmax);
-    s.W = (float *)take((size_t)dm.d * dm.Dh * 4);
-    s.Wt = take((size_t)dm.d * dm.Dh * e);
+    s.W = (float *)take((size_t)dm.nW * dm.d * dm.Dh * 4);
+    s.Wt = take((size_t)dm.nW * dm.d * dm.Dh * e);
     s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     s.phiQd = (float *)take(dm.dtype == LOLA_BF16 ? (size_t)dm.B * dm.Hq * dm.D * 4 : 0);
@@ -297,6 +301,9 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
         ca.iglob0 = st->n_int;
         ca.phi = st->S.phiV;
         ca.nvrows = dm.lam + dm.R;
+        ca.qin = q;          // the step's query is the interval's first
+        ca.q_start = pos;
+        ca.q_n = 1;
         ca.sel_log = st->sel_log;
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;
@@ -529,6 +536,9 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         ca.iglob0 = st->n_int;
         ca.phi = st->P.phiK;
         ca.nvrows = dm.lam + dm.R + dm.Nmax;
+        ca.qin = q;
+        ca.q_start = pos0;
+        ca.q_n = n;
         ca.sel_log = st->sel_log;
         ca.sel_cap = st->sel_cap;
         ca.ovr = st->ovr;

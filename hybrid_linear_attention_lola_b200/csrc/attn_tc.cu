@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     {
-        const bf16 *Wt = (const bf16 *)S.Wt;
+        const bf16 *Wt = (const bf16 *)S.Wt + (dm.nW > 1 ? (size_t)hk * Dh * d : 0);
         for (int e = tid; e < (Dh << lgd); e += kThreads) {
             const int rr = e >> lgd, kc = e & ((1 << lgd) - 1);
             umma::cp_async16(sPr + umma::kmajor_offset(rr, kc * 8, Dh), Wt + (size_t)rr * d + kc * 8);

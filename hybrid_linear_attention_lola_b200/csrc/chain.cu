@@ -14,6 +14,7 @@
 // the fate of each leaving pair and a snapshot of (H', s') for the attention
 // kernel. Decode mode moves kept leaving pairs from the ring into cache slots.
 #include "lola_internal.cuh"
+#include "scoring.cuh"
 
 namespace lola {
 
@@ -172,9 +173,28 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncthreads();
 
-        //    Self-Recall Error against the state at the interval start
+        //    Self-Recall Error against the state at the interval start (or an ablation score)
         const int nDu = D >> 5, ndu = d >> 5;
-        for (int c = warp; c < nQ; c += nw) {
+        if (dm.scorer != kScoreSRE) {
+            float *score = (float *)keepf, *lg = (float *)tmpA, *lu = (float *)tmpB;
+            float *qs = stgPhi, *pq = stgPhi + dm.g * d, *red = (float *)scal;
+            const T *qb = (const T *)a.qin;
+            const int b = st / dm.Hkv, hk = st % dm.Hkv;
+            const size_t qrow0 = (((size_t)b * a.q_n + (size_t)(t0 - a.q_start)) * dm.Hq + (size_t)hk * dm.g) * d;
+            alt_scores<T>(
+                dm.scorer, nQ, [&](int c) { return src.krow(st, cvrow[c]); },
+                [&](int c) { return phi_st + (size_t)cvrow[c] * D; }, [&](int h) { return qb + qrow0 + (size_t)h * d; },
+                [&](int c) { return ctok[c]; }, w_of(dm, S.W, hk), dm.g, d, D, score, qs, pq, lg, lu, red);
+            for (int c = tid; c < nQ; c += nt) {
+                keys[c] = make_key(score[c], ctok[c]);
+                if (a.score_sre != nullptr && iglob < a.score_cap) {
+                    const size_t o = ((size_t)iglob * dm.ns + st) * QC + c;
+                    a.score_sre[o] = score[c];
+                    a.score_tok[o] = ctok[c];
+                }
+            }
+        }
+        for (int c = dm.scorer == kScoreSRE ? warp : nQ; c < nQ; c += nw) {
             const T *ph = phi_st + (size_t)cvrow[c] * D;
             float phr[8];
             float den = 0.f;

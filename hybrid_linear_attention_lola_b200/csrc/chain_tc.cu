@@ -30,6 +30,7 @@
 // which subtracts the linear terms of the folded leaving pairs that are still
 // inside a query's window (the softmax attends them there).
 #include "lola_internal.cuh"
+#include "scoring.cuh"
 #include "umma.cuh"
 
 namespace lola {
@@ -499,7 +500,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int cnd = tid; cnd < nQ; cnd += kThreads)
             cvrow[cnd] = cnd < nS ? slotVrow[cnd] : src.tok2vrow(Llo + (cnd - nS));
         __syncthreads();
-        const int ntile = (nQ + 127) / 128;
+        if (dm.scorer != kScoreSRE) {
+            // an ablation score instead of the SRE: every CTA scores every candidate (no
+            // key exchange); the first-query rows come from the caller's queries
+            float *score = (float *)keys;
+            float *lg = (float *)lst, *lu = (float *)((ci & 1) ? keys0 : keys1);
+            float *qs = (float *)c.X, *pq = qs + dm.g * d, *red = (float *)(base + g.off_part);
+            const bf16 *qb = (const bf16 *)a.qin;
+            const int b = st / dm.Hkv, hk = st % dm.Hkv;
+            const size_t qrow0 = (((size_t)b * a.q_n + (size_t)(t0 - a.q_start)) * dm.Hq + (size_t)hk * dm.g) * d;
+            alt_scores<bf16>(
+                dm.scorer, nQ, [&](int cc) { return src.krow(st, cvrow[cc]); },
+                [&](int cc) { return phi_st + (size_t)cvrow[cc] * D; },
+                [&](int h) { return qb + qrow0 + (size_t)h * d; },
+                [&](int cc) { return cc < nS ? slotTok[cc] : (int)(Llo + (cc - nS)); }, w_of(dm, S.W, hk), dm.g, d, D, score,
+                qs, pq, lg, lu, red);
+            for (int cc = tid; cc < nQ; cc += kThreads) {
+                const float sc = score[cc];
+                if (a.score_sre != nullptr && iglob < a.score_cap && lead) {
+                    const size_t o = ((size_t)iglob * dm.ns + st) * g.QC + cc;
+                    a.score_sre[o] = sc;
+                    a.score_tok[o] = cc < nS ? slotTok[cc] : (int)(Llo + (cc - nS));
+                }
+                keys[cc] = 0xFFFFFFFFu - __float_as_uint(fmaxf(sc, 0.f));
+            }
+            __syncthreads();
+        }
+        const int ntile = dm.scorer == kScoreSRE ? (nQ + 127) / 128 : 0;
         const int nmy = ntile > crank ? (ntile - crank + nc - 1) / nc : 0;   // this CTA's tiles
         // phi rows of this CTA's tile lt (K-major A operand) into buffer lt % nbuf by TMA
         // row gathers from warp 0 (rows r..r+3 of one 64-feature block per instruction;
@@ -616,7 +643,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncthreads();
         }
         if (!ok) break;
-        if (nc > 1) {
+        if (nc > 1 && dm.scorer == kScoreSRE) {
             // push this CTA's keys into every peer's buffer, then signal it; wait for theirs
             for (int pr = 1; pr < nc; ++pr) {
                 const uint32_t peer = (uint32_t)((crank + pr) % nc);

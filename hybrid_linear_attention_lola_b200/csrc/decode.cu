@@ -317,7 +317,7 @@ __global__ void __launch_bounds__(128) decode3_kernel(Dims dm, DevState S, Decod
         if (cg < ncg) {
 #pragma unroll 8
             for (int c = cr * per; c < (cr + 1) * per; ++c) {
-                const float4 w4 = __ldg((const float4 *)(S.W + (size_t)c * Dh) + cg);
+                const float4 w4 = __ldg((const float4 *)(w_of(dm, S.W, st % dm.Hkv) + (size_t)c * Dh) + cg);
 #pragma unroll
                 for (int r = 0; r <= kMaxG; ++r) {
                     if (r < nr) {
@@ -736,22 +736,25 @@ __global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, D
     const int d = dm.d, Dh = dm.Dh, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *Ws = smp;
     float *xs = smp + d * Dh + warp * d;
+    const int hw = blockIdx.y;   // with one W per kv-head, grid row hw takes that kv-head's rows
+    const bool by_head = gridDim.y > 1;
     {
         // 16-byte copies, all in flight at once (d * Dh is a multiple of 4)
-        const float4 *w4 = (const float4 *)S.W;
+        const float4 *w4 = (const float4 *)(S.W + (size_t)hw * d * Dh);
         float4 *s4 = (float4 *)Ws;
         const int n4 = d * Dh / 4;
 #pragma unroll 4
         for (int e = threadIdx.x; e < n4; e += blockDim.x) s4[e] = __ldg(w4 + e);
     }
     __syncthreads();
-    const int nq = dm.B * dm.Hq, nk = do_append ? dm.ns : 0;
+    const int nq = by_head ? dm.B * dm.g : dm.B * dm.Hq, nk = do_append ? (by_head ? dm.B : dm.ns) : 0;
     const int slot = (int)(a.pos & (dm.R - 1));
-    for (int r = blockIdx.x * 8 + warp; r < nq + nk; r += gridDim.x * 8) {
-        if (r < nq) {
+    for (int rr = blockIdx.x * 8 + warp; rr < nq + nk; rr += gridDim.x * 8) {
+        if (rr < nq) {
+            const int r = by_head ? (rr / dm.g) * dm.Hq + hw * dm.g + rr % dm.g : rr;
             phi_row_warp<T, float>((const T *)a.q + (size_t)r * d, Ws, xs, d, Dh, S.phiQd + (size_t)r * dm.D);
         } else {
-            const int st = r - nq;
+            const int st = by_head ? (rr - nq) * dm.Hkv + hw : rr - nq;
             const T *k = (const T *)a.k + (size_t)st * d, *v = (const T *)a.v + (size_t)st * d;
             T *kr = (T *)S.KR + ((size_t)st * dm.R + slot) * d, *vr = (T *)S.VR + ((size_t)st * dm.R + slot) * d;
             for (int c = lane; c < d; c += 32) {
@@ -1300,7 +1303,7 @@ __global__ void append_kernel(Dims dm, DevState S, const T *__restrict__ k, cons
         VR[c] = v[(size_t)st * dm.d + c];
     }
     if (with_phi && threadIdx.x < 32)
-        phi_row_warp<T, T>(k + (size_t)st * dm.d, S.W, xs, dm.d, dm.Dh,
+        phi_row_warp<T, T>(k + (size_t)st * dm.d, w_of(dm, S.W, st % dm.Hkv), xs, dm.d, dm.Dh,
                         (T *)S.phiV + ((size_t)st * (dm.lam + dm.R) + dm.lam + slot) * dm.D);
 }
 
@@ -1433,10 +1436,10 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psm);
                 attr = psm;
             }
-            const int rows = dm.B * dm.Hq + (do_append ? dm.ns : 0);
+            const int rows = (dm.B * dm.Hq + (do_append ? dm.ns : 0)) / dm.nW;
             int grid = (rows + 7) / 8;
             if (grid > kSMs * 4) grid = kSMs * 4;
-            decode_prep_kernel<__nv_bfloat16><<<grid, 256, psm, stream>>>(dm, S, a, do_append);
+            decode_prep_kernel<__nv_bfloat16><<<dim3(grid, dm.nW), 256, psm, stream>>>(dm, S, a, do_append);
         }
         const int G = dm.g <= 1 ? 1 : dm.g <= 2 ? 2 : dm.g <= 4 ? 4 : 8;
         const int wb = stream_warp_bytes(dm, G);

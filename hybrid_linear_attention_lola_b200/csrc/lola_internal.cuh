@@ -35,6 +35,8 @@ struct Dims {
     int dec_minper;   // decode (bf16): fewest work items per warp (fewer for few streams)
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
+    int scorer;       // cache scoring: 0 SRE, 1 attention weight, 2 softmax-approximation error, 3 recency
+    int nW;           // feature-map matrices: 1 (shared) or Hkv (one per kv-head)
     float eps;
 };
 
@@ -46,8 +48,8 @@ struct DevState {
     int *idxS;         // [ns][lam]    token index per cache slot, -1 = empty
     void *KR, *VR;     // [ns][R][d]   window ring (slot = token mod R)
     uint8_t *pend;     // [ns][Lmax]   1 = leaving pair of the last interval that is folded
-    float *W;          // [d][Dh]      feature-map matrix, fp32 copy
-    void *Wt;          // [Dh][d]      W transposed, in the input dtype (tensor-core operand)
+    float *W;          // [nW][d][Dh]  feature-map matrices (one per kv-head, or one shared), fp32 copy
+    void *Wt;          // [nW][Dh][d]  W transposed, in the input dtype (tensor-core operand)
     int *err;          // [4]          device error words
     // decode scratch (phi buffers hold the input dtype)
     void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
@@ -127,6 +129,12 @@ __device__ __forceinline__ float warp_min(float x)
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fminf(x, __shfl_xor_sync(0xffffffffu, x, o));
     return x;
+}
+
+// The feature-map matrix of kv-head hk (W: [nW][d][Dh]).
+__device__ __forceinline__ const float *w_of(const Dims &dm, const float *W, int hk)
+{
+    return dm.nW > 1 ? W + (size_t)hk * dm.d * dm.Dh : W;
 }
 
 // phi(x) = [softmax(x W), softmax(-x W)] of one row, computed by one warp. W (fp32, [d][Dh]) sits in shared memory; lane l owns
@@ -232,6 +240,9 @@ struct ChainArgs {
     long long sel_cap;
     const int32_t *ovr;     // test hook, may be null
     long long ovr_n;
+    const void *qin;        // queries holding every interval's first query (alternative scorers):
+    long long q_start;      //   [B][q_n][Hq][d], row 0 = token q_start
+    int q_n;
     unsigned long long inject_ns;   // test hook: > 0 makes the first interval wait this long on an
                                     // mbarrier nothing arrives at (the wait runs out: timeout)
     float *score_sre;       // test hook, may be null: SRE of every candidate

@@ -6,6 +6,8 @@
 
 namespace lola {
 
+// Blocks with blockIdx.y = w take the rows of kv-head w when every kv-head has its
+// own W (gridDim.y = n_kv_heads), all rows otherwise (gridDim.y = 1).
 template <typename T>
 __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, const float *__restrict__ W,
                                                      int nS, int n, int nvrows,
@@ -14,14 +16,18 @@ __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, cons
     extern __shared__ float sm[];
     float *Ws = sm;                                   // [d][Dh]
     float *xs = sm + dm.d * dm.Dh + (threadIdx.x >> 5) * dm.d;
-    for (int e = threadIdx.x; e < dm.d * dm.Dh; e += blockDim.x) Ws[e] = W[e];
+    const int hw = blockIdx.y;
+    const float *Wh = W + (size_t)hw * dm.d * dm.Dh;
+    for (int e = threadIdx.x; e < dm.d * dm.Dh; e += blockDim.x) Ws[e] = Wh[e];
     __syncthreads();
     const int per_stream = nS + dm.R + n;
-    const long long total = (long long)dm.ns * per_stream;
+    const int nsw = gridDim.y > 1 ? dm.B : dm.ns;     // streams this block row covers
+    const long long total = (long long)nsw * per_stream;
     const int warps = blockDim.x >> 5;
     for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < total;
          r += (long long)gridDim.x * warps) {
-        const int st = (int)(r / per_stream);
+        const int sw = (int)(r / per_stream);
+        const int st = gridDim.y > 1 ? sw * dm.Hkv + hw : sw;
         const int i = (int)(r % per_stream);
         const int vrow = i < nS ? i : dm.lam + (i - nS);
         phi_row_warp<T, T>(src.krow(st, vrow), Ws, xs, dm.d, dm.Dh,
@@ -29,20 +35,27 @@ __global__ void __launch_bounds__(256) phi_kv_kernel(Dims dm, KVSrc<T> src, cons
     }
 }
 
+// rows: query rows [..][Hq][d]; with gridDim.y = n_kv_heads, blocks of row w take the
+// query heads of kv-head w (their own W), else every row (gridDim.y = 1)
 template <typename T>
-__global__ void __launch_bounds__(256) phi_q_kernel(int d, int Dh, const float *__restrict__ W,
+__global__ void __launch_bounds__(256) phi_q_kernel(int d, int Dh, int Hq, int g, const float *__restrict__ W,
                                                     const T *__restrict__ q, long long rows,
                                                     T *__restrict__ phi_out)
 {
     extern __shared__ float sm[];
     float *Ws = sm;
     float *xs = sm + d * Dh + (threadIdx.x >> 5) * d;
-    for (int e = threadIdx.x; e < d * Dh; e += blockDim.x) Ws[e] = W[e];
+    const int hw = blockIdx.y;
+    const float *Wh = W + (size_t)hw * d * Dh;
+    for (int e = threadIdx.x; e < d * Dh; e += blockDim.x) Ws[e] = Wh[e];
     __syncthreads();
     const int warps = blockDim.x >> 5;
-    for (long long r = (long long)blockIdx.x * warps + (threadIdx.x >> 5); r < rows;
-         r += (long long)gridDim.x * warps)
+    const long long mine = gridDim.y > 1 ? rows / Hq * g : rows;
+    for (long long rr = (long long)blockIdx.x * warps + (threadIdx.x >> 5); rr < mine;
+         rr += (long long)gridDim.x * warps) {
+        const long long r = gridDim.y > 1 ? (rr / g) * Hq + (long long)hw * g + rr % g : rr;
         phi_row_warp<T, T>(q + (size_t)r * d, Ws, xs, d, Dh, phi_out + (size_t)r * 2 * Dh);
+    }
 }
 
 static int grid_for(long long rows, int warps_per_block)
@@ -58,7 +71,7 @@ void launch_phi_kv(const Dims &dm, const DevState &S, const void *kin, long long
 {
     const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
     const long long rows = (long long)dm.ns * (nS + dm.R + n);
-    const int grid = grid_for(rows, 8);
+    const dim3 grid(grid_for(rows / dm.nW, 8), dm.nW);
     if (dm.dtype == 0) {
         cudaFuncSetAttribute(phi_kv_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         KVSrc<float> src{(const float *)S.KS, (const float *)S.VS, (const float *)S.KR,
@@ -82,16 +95,16 @@ void launch_phi_q(const Dims &dm, const float *W, const void *q, long long rows,
                   cudaStream_t stream)
 {
     const size_t smem = sizeof(float) * ((size_t)dm.d * dm.Dh + 8 * dm.d);
-    const int grid = grid_for(rows, 8);
+    const dim3 grid(grid_for(rows / dm.nW, 8), dm.nW);
     if (dm.dtype == 0) {
         cudaFuncSetAttribute(phi_q_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        phi_q_kernel<float><<<grid, 256, smem, stream>>>(dm.d, dm.Dh, W, (const float *)q, rows,
+        phi_q_kernel<float><<<grid, 256, smem, stream>>>(dm.d, dm.Dh, dm.Hq, dm.g, W, (const float *)q, rows,
                                                          (float *)phi_out);
     } else {
         cudaFuncSetAttribute(phi_q_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
         phi_q_kernel<__nv_bfloat16><<<grid, 256, smem, stream>>>(
-            dm.d, dm.Dh, W, (const __nv_bfloat16 *)q, rows, (__nv_bfloat16 *)phi_out);
+            dm.d, dm.Dh, dm.Hq, dm.g, W, (const __nv_bfloat16 *)q, rows, (__nv_bfloat16 *)phi_out);
     }
 }
 
@@ -122,11 +135,14 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
         VR[e] = from_f<T>(0.f);
     }
     if (W != nullptr) {
+        // nW matrices [d][Dh] (one per kv-head, or one shared): fp32 copy and transpose
         T *Wt = (T *)S.Wt;
-        for (long long e = tid; e < (long long)dm.d * dm.Dh; e += stride) {
+        const long long per = (long long)dm.d * dm.Dh;
+        for (long long e = tid; e < per * dm.nW; e += stride) {
             S.W[e] = to_f<T>(W[e]);
-            const long long a = e / dm.Dh, i = e - a * dm.Dh;
-            Wt[i * dm.d + a] = W[e];
+            const long long h = e / per, r = e - h * per;
+            const long long a = r / dm.Dh, i = r - a * dm.Dh;
+            Wt[h * per + i * dm.d + a] = W[e];
         }
     }
     if (tid < 4) S.err[tid] = 0;

@@ -73,8 +73,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (tid == 0) umma::mbar_init(&mbar, 1);
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
-    // W^T [Dh][d] as a K-major operand of Dh rows
-    const bf16 *Wt = (const bf16 *)S.Wt;
+    // W^T [Dh][d] as a K-major operand of Dh rows; with one W per kv-head, the CTAs of
+    // grid row y take the rows of kv-head y
+    const int hw = blockIdx.y;
+    const bf16 *Wt = (const bf16 *)S.Wt + (size_t)hw * Dh * d;
     for (int e = tid; e < (Dh << lgd); e += kThreads) {
         const int r = e >> lgd, kc = e & ((1 << lgd) - 1);
         umma::cp_async16(sW + umma::kmajor_offset(r, kc * 8, Dh), Wt + (size_t)r * d + kc * 8);
@@ -87,15 +89,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t phase = 0;
     const uint32_t idesc = umma::idesc_bf16(128, Dh, false, false);
     const int per_stream = nS + dm.R + (MODE == 0 ? src.n : 0);
-    const long long ntiles = (nrows + 127) / 128;
+    const bool by_head = gridDim.y > 1;
+    // rows of this grid row: every row, or those of kv-head hw
+    const long long nmine = !by_head ? nrows : MODE == 0 ? (long long)dm.B * per_stream : nrows / dm.Hq * dm.g;
+    const long long ntiles = (nmine + 127) / 128;
     bool ok = true;
 
     for (long long tile = blockIdx.x; tile < ntiles && ok; tile += gridDim.x) {
         const long long r0 = tile * 128;
-        const int nr = (int)min(128LL, nrows - r0);
+        const int nr = (int)min(128LL, nmine - r0);
         // this thread's row: where it comes from and where its features go
         {
-            const long long gr = r0 + tid;
+            const long long rr = r0 + tid;
+            long long gr = rr;
+            if (by_head) {
+                if (MODE == 0) gr = ((rr / per_stream) * dm.Hkv + hw) * per_stream + rr % per_stream;
+                else gr = (rr / dm.g) * dm.Hq + (long long)hw * dm.g + rr % dm.g;
+            }
             const bf16 *xi = nullptr;
             bf16 *yo = nullptr;
             if (tid < nr) {
@@ -203,16 +213,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0) umma::tmem_dealloc(tz, g.ncols);
 }
 
-int phi_tc_grid(long long nrows, const Dims &dm)
+dim3 phi_tc_grid(long long nrows, const Dims &dm)
 {
+    nrows /= dm.nW;
     const PGeo g = make_pgeo(dm.d, dm.D);
     int per_sm = (int)((228 * 1024) / (g.total + 1024));
     if (per_sm < 1) per_sm = 1;
     if (per_sm > 4) per_sm = 4;
     long long tiles = (nrows + 127) / 128;
-    long long grid = 148LL * per_sm;
+    long long grid = 148LL * per_sm / dm.nW;
     if (grid > tiles) grid = tiles;
-    return (int)(grid < 1 ? 1 : grid);
+    return dim3((unsigned)(grid < 1 ? 1 : grid), (unsigned)dm.nW);
 }
 
 }  // namespace

@@ -34,7 +34,11 @@ class lola_config(ctypes.Structure):
                 ("feat_dim", ctypes.c_int32), ("window", ctypes.c_int32),
                 ("lambda_", ctypes.c_int32), ("chunk", ctypes.c_int32),
                 ("decode_interval", ctypes.c_int32), ("max_prefill_tokens", ctypes.c_int32),
-                ("eps", ctypes.c_float), ("dtype", ctypes.c_int32)]
+                ("eps", ctypes.c_float), ("dtype", ctypes.c_int32), ("scorer", ctypes.c_int32),
+                ("w_per_kv_head", ctypes.c_int32)]
+
+
+SCORERS = {"sre": 0, "attention-weight": 1, "softmax-error": 2, "fifo": 3}
 
 
 _lib = None
@@ -98,17 +102,20 @@ def _check(code: int, what: str):
 
 
 def make_config(*, batch, n_q_heads, n_kv_heads, head_dim, feat_dim, window, lambda_, chunk,
-                decode_interval, max_prefill_tokens=0, eps=1e-6, dtype="bf16") -> lola_config:
+                decode_interval, max_prefill_tokens=0, eps=1e-6, dtype="bf16",
+                scorer="sre", w_per_kv_head=False) -> lola_config:
     return lola_config(batch, n_q_heads, n_kv_heads, head_dim, feat_dim, window, lambda_, chunk,
                        decode_interval, max_prefill_tokens, eps,
-                       LOLA_F32 if dtype in ("f32", "float32") else LOLA_BF16)
+                       LOLA_F32 if dtype in ("f32", "float32") else LOLA_BF16, SCORERS[scorer],
+                       1 if w_per_kv_head else 0)
 
 
 def config_from_workload(w, max_prefill_tokens: Optional[int] = None, **over) -> lola_config:
     kw = dict(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads,
               head_dim=w.head_dim, feat_dim=w.feat_dim, window=w.window, lambda_=w.lambda_,
               chunk=w.chunk, decode_interval=w.decode_interval,
-              max_prefill_tokens=max_prefill_tokens or w.seq_len, eps=w.eps, dtype=w.dtype)
+              max_prefill_tokens=max_prefill_tokens or w.seq_len, eps=w.eps, dtype=w.dtype,
+              scorer=getattr(w, "scorer", "sre"), w_per_kv_head=getattr(w, "w_per_head", False))
     kw.update(over)
     return make_config(**kw)
 

@@ -45,6 +45,9 @@ class Workload:
     needles: int = 0         # planted near-collinear key pairs
     lowrank: int = 0         # rank of the shared key/value component (0 = none)
     lowrank_scale: float = 0.0
+    scorer: str = "sre"      # cache scoring: "sre" (the method) or an ablation
+                             # ("attention-weight", "softmax-error", "fifo")
+    w_per_head: bool = False  # one feature-map matrix per kv-head (W [H_kv, d, D/2])
 
     @property
     def group(self) -> int:
@@ -119,9 +122,13 @@ def _normal(rng: np.random.Generator, shape) -> np.ndarray:
 
 
 def make_W(w: Workload) -> np.ndarray:
-    """Feature-map matrix W [d, D/2] ~ N(0,1)/sqrt(d), rounded to the dtype."""
+    """Feature-map matrix W [d, D/2] ~ N(0,1)/sqrt(d), rounded to the dtype; with
+    w_per_head one independent matrix per kv-head, [H_kv, d, D/2]."""
     rng = np.random.Generator(np.random.PCG64([SEED_BASE + w.wid, 1]))
-    W = _normal(rng, (w.head_dim, w.feat_dim // 2)) / np.float32(np.sqrt(w.head_dim))
+    shape = (w.head_dim, w.feat_dim // 2)
+    if w.w_per_head:
+        shape = (w.n_kv_heads,) + shape
+    W = _normal(rng, shape) / np.float32(np.sqrt(w.head_dim))
     return round_to_dtype(W, w.dtype)
 
 

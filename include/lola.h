@@ -58,6 +58,27 @@ typedef enum {
 
 typedef enum { LOLA_F32 = 0, LOLA_BF16 = 1 } lola_dtype;
 
+/* How the sparse cache ranks its candidates (the cache pairs and the pairs
+ * leaving the window) at each update interval; the highest scores stay.
+ * LOLA_SCORE_SRE is the method (section "Het Self-Recall Error (SRE)
+ * Mechanisme"). The others are the alternatives the paper's ablations compare
+ * it against (sections "Belangrijkste bijdragen" and "Ablaties") and the FIFO
+ * structure the "Inferentiestrategie" section mentions; the pages do not define
+ * them, this engine's readings are, for the interval's first query q and summed
+ * over the query heads of the kv-head's group:
+ *   LOLA_SCORE_ATTN_WEIGHT    the softmax weight of the pair among the candidates,
+ *                             softmax over candidates c of q.k_c / sqrt(head_dim);
+ *   LOLA_SCORE_SOFTMAX_ERROR  (that weight - phi(q).phi(k) / sum over candidates of
+ *                             phi(q).phi(k_c))^2, how badly the linear attention
+ *                             approximates the pair's softmax weight;
+ *   LOLA_SCORE_RECENCY        the token index: the most recent pairs stay (FIFO). */
+typedef enum {
+    LOLA_SCORE_SRE = 0,
+    LOLA_SCORE_ATTN_WEIGHT = 1,
+    LOLA_SCORE_SOFTMAX_ERROR = 2,
+    LOLA_SCORE_RECENCY = 3
+} lola_scorer;
+
 typedef struct {
     int32_t batch;              /* B >= 1 */
     int32_t n_q_heads;          /* multiple of n_kv_heads, at most 8 per kv-head */
@@ -71,6 +92,9 @@ typedef struct {
     int32_t max_prefill_tokens; /* largest n_tokens of one prefill call (multiple of chunk) */
     float eps;                  /* >= 0, added to every denominator (SRE and output) */
     int32_t dtype;              /* lola_dtype of q, k, v, out and W */
+    int32_t scorer;             /* lola_scorer (0 = the Self-Recall Error) */
+    int32_t w_per_kv_head;      /* 0: one feature-map matrix W shared by every head;
+                                   1: one per kv-head (its query heads use it too) */
 } lola_config;
 
 typedef struct lola_state lola_state; /* opaque host handle */
@@ -82,9 +106,10 @@ lola_status lola_state_bytes(const lola_config *cfg, size_t *device_bytes);
 /* Creates a state in `workspace` (device, >= lola_state_bytes, 256-byte
  * aligned, owned by the caller and kept alive until lola_free_state) and
  * resets it to the empty state at position 0: H = 0, s = 0, empty cache and
- * window. W: device [head_dim][feat_dim/2] in cfg->dtype, copied in (the
- * caller may free it after the stream has passed this call). On success
- * *out receives a host handle. */
+ * window. W: device [head_dim][feat_dim/2] in cfg->dtype, or with
+ * cfg->w_per_kv_head [n_kv_heads][head_dim][feat_dim/2] (kv-head h's keys and
+ * its query heads use W[h]); copied in (the caller may free it after the stream
+ * has passed this call). On success *out receives a host handle. */
 lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspace,
                             size_t workspace_bytes, void *cuda_stream, lola_state **out);
 

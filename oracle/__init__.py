@@ -30,7 +30,8 @@ _lib = None
 class OracleCfg(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("d", ctypes.c_int32), ("D", ctypes.c_int32), ("eta", ctypes.c_int32),
-                ("lam", ctypes.c_int32), ("eps", ctypes.c_double), ("scorer", ctypes.c_int32)]
+                ("lam", ctypes.c_int32), ("eps", ctypes.c_double), ("scorer", ctypes.c_int32),
+                ("w_per_head", ctypes.c_int32)]
 
 
 SCORERS = {"sre": 0, "attention-weight": 1, "softmax-error": 2, "fifo": 3}
@@ -118,11 +119,14 @@ def run(q: np.ndarray, k: np.ndarray, v: np.ndarray, W: np.ndarray, *, window: i
     W = np.ascontiguousarray(W, np.float32)
     B, T, Hq, d = q.shape
     Hkv = k.shape[2]
-    D = 2 * W.shape[1]
+    D = 2 * W.shape[-1]
+    per_head = W.ndim == 3          # W [Hkv, d, D/2]: one feature-map matrix per kv-head
+    if per_head and W.shape[0] != Hkv:
+        raise ValueError("per-head W needs one matrix per kv-head")
     ints = np.ascontiguousarray(np.asarray(intervals, np.int32))
     n_int = len(ints)
     ns = B * Hkv
-    cfg = OracleCfg(B, Hq, Hkv, d, D, window, lambda_, eps, SCORERS[scorer])
+    cfg = OracleCfg(B, Hq, Hkv, d, D, window, lambda_, eps, SCORERS[scorer], 1 if per_head else 0)
     r = OracleResult()
     out_row = None
     n_out = T

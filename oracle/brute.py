@@ -85,7 +85,9 @@ def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6, 
         for b in range(B):
             for hk in range(Hkv):
                 st = b * Hkv + hk
-                pk = phi_rows(k[b, :, hk, :], W)            # [T, D]
+                Wh = W[hk] if np.ndim(W) == 3 else W       # one matrix per kv-head, or shared
+                _W_for_scores = np.asarray(Wh, np.float64)
+                pk = phi_rows(k[b, :, hk, :], Wh)           # [T, D]
                 vv = v[b, :, hk, :]
                 cache = set(S[st])
                 folded = [j for j in range(0, max(0, t0 - eta)) if j not in cache]
@@ -103,7 +105,7 @@ def run(q, k, v, W, *, window: int, lambda_: int, intervals, eps: float = 1e-6, 
                     for r in range(g):
                         hq = hk * g + r
                         qp = q[b, p, hq, :]
-                        pq = phi_rows(qp[None, :], W)[0]
+                        pq = phi_rows(qp[None, :], Wh)[0]
                         num = np.zeros(d)
                         den = eps
                         for j in range(0, p + 1):

@@ -58,6 +58,7 @@ typedef struct {
     int32_t B, Hq, Hkv, d, D, eta, lam;
     double eps;
     int32_t scorer; /* 0 SRE, 1 attention weight, 2 softmax-approximation error, 3 recency */
+    int32_t w_per_head; /* 1: W holds one d x D/2 matrix per kv-head (the pages leave this open) */
 } oracle_cfg;
 
 /* phi(x) = [softmax(x W), softmax(-x W)]  (x: d, W: d x D/2 row-major, out: D) */
@@ -165,6 +166,8 @@ static void run_stream(job_t *J, int st)
     const int nstreams = B * Hkv;
     const double eps = cfg->eps;
     const double scale = 1.0 / sqrt((double)d);
+    /* the feature-map matrix of this stream's kv-head (its query heads share it) */
+    const double *Wst = J->W + (cfg->w_per_head ? (size_t)hk * d * (D / 2) : 0);
     (void)B;
 
     /* per-stream copies of keys, values and phi(k) for every token */
@@ -177,7 +180,7 @@ static void run_stream(job_t *J, int st)
             kd[(size_t)t * d + c] = J->k[src + c];
             vd[(size_t)t * d + c] = J->v[src + c];
         }
-        oracle_phi(kd + (size_t)t * d, J->W, d, D, phik + (size_t)t * D);
+        oracle_phi(kd + (size_t)t * d, Wst, d, D, phik + (size_t)t * D);
     }
 
     double *H = (double *)calloc((size_t)D * d, sizeof(double));
@@ -242,7 +245,7 @@ static void run_stream(job_t *J, int st)
                 }
                 for (int c = 0; c < nQ; ++c) z += exp(sc[c] - mx);
                 if (cfg->scorer == 2) {
-                    oracle_phi(qv, J->W, d, D, phiq);
+                    oracle_phi(qv, Wst, d, D, phiq);
                     for (int c = 0; c < nQ; ++c) {
                         const double *pk = phik + (size_t)cand[c].tok * D;
                         double w = 0.0;
@@ -331,7 +334,7 @@ static void run_stream(job_t *J, int st)
                     for (int c = 0; c < d; ++c) num[c] += w * vv[c];
                 }
                 /* linear terms: phi(q)^T H', phi(q)^T s', and the folded band */
-                oracle_phi(qv, J->W, d, D, phiq);
+                oracle_phi(qv, Wst, d, D, phiq);
                 double lden = eps;
                 for (int c = 0; c < d; ++c) lin[c] = 0.0;
                 for (int rr = 0; rr < D; ++rr) {
@@ -433,8 +436,9 @@ int oracle_run(const oracle_cfg *cfg, int T, const float *q, const float *k, con
     }
     if (tot < T) return -3;
     int Dh = cfg->D / 2;
-    double *W = (double *)malloc(sizeof(double) * (size_t)cfg->d * Dh);
-    for (int i = 0; i < cfg->d * Dh; ++i) W[i] = Wf[i];
+    const int nW = cfg->w_per_head ? cfg->Hkv : 1;
+    double *W = (double *)malloc(sizeof(double) * (size_t)nW * cfg->d * Dh);
+    for (int i = 0; i < nW * cfg->d * Dh; ++i) W[i] = Wf[i];
     job_t J;
     memset(&J, 0, sizeof(J));
     J.cfg = cfg; J.T = T; J.q = q; J.k = k; J.v = v; J.W = W;

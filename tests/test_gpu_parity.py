@@ -61,7 +61,8 @@ def _case(w, plan, *, modes=("forced", "own"), subset=None, qmask_every=None,
         qmask[-1] = 1
         rows = np.flatnonzero(qmask)
     r = oracle.run(qo, ko, vo, W, window=w.window, lambda_=w.lambda_, intervals=ints,
-                   eps=w.eps, qmask=qmask, want_cands=True, compact=qmask is not None)
+                   eps=w.eps, qmask=qmask, want_cands=True, compact=qmask is not None,
+                   scorer=w.scorer)
     smap = [b * w.n_kv_heads + h for b in bsel for h in hsel]
     ns = w.batch * w.n_kv_heads
     res = {}
@@ -280,3 +281,43 @@ def test_token_by_token_intervals():
     w = wl.WORKLOADS["token-by-token"]
     res = _case(w, [("prefill", w.seq_len), ("decode", w.decode_steps)], modes=ALL)
     assert res["free"]["exact"] == res["free"]["intervals_checked"]
+
+
+# ---------------------------------------------------------------- the pages' ablation scorers, FIFO
+
+@pytest.mark.parametrize("scorer", ["attention-weight", "softmax-error", "fifo"])
+def test_ablation_scorer_bf16(scorer):
+    # tensor-core chain on a two-CTA cluster per stream (the scores are computed by
+    # every CTA, no key exchange), then decode intervals scored at their first step
+    w = _small_bf16(n_q_heads=4, n_kv_heads=2, window=16, lambda_=150, chunk=32, decode_interval=16,
+                    scorer=scorer)
+    _case(w, [("prefill", 256), ("decode", 40)], modes=ALL, scores=True, name=f"bf16 scorer {scorer}")
+
+
+@pytest.mark.parametrize("scorer", ["attention-weight", "softmax-error", "fifo"])
+def test_ablation_scorer_f32(scorer):
+    w = _small(n_q_heads=4, n_kv_heads=2, window=8, lambda_=20, chunk=16, decode_interval=8,
+               head_dim=64, feat_dim=64, scorer=scorer)
+    _case(w, [("prefill", 128), ("decode", 24)], modes=ALL, scores=True, name=f"f32 scorer {scorer}")
+
+
+# ---------------------------------------------------------------- one feature map per kv-head
+
+def test_per_head_feature_maps_bf16():
+    # tensor-core feature map (grid rows by kv-head), chain, attention, decode preparation
+    w = _small_bf16(n_q_heads=8, n_kv_heads=4, window=16, lambda_=150, chunk=32, decode_interval=16,
+                    w_per_head=True)
+    _case(w, [("prefill", 256), ("decode", 40)], modes=ALL, name="bf16 per-head W")
+
+
+def test_per_head_feature_maps_bf16_query_kernel():
+    # no cache: SIMT chain with the tensor-core query feature map (grid rows by kv-head)
+    w = _small_bf16(n_q_heads=8, n_kv_heads=4, window=12, lambda_=0, chunk=16, decode_interval=8,
+                    w_per_head=True)
+    _case(w, [("prefill", 128), ("decode", 24)], modes=("free",), name="bf16 per-head W, no cache")
+
+
+def test_per_head_feature_maps_f32_with_softmax_error():
+    w = _small(n_q_heads=6, n_kv_heads=3, window=8, lambda_=20, chunk=16, decode_interval=8,
+               head_dim=64, feat_dim=64, w_per_head=True, scorer="softmax-error")
+    _case(w, [("prefill", 128), ("decode", 24)], modes=ALL, name="f32 per-head W, softmax-error")

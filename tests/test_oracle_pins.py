@@ -394,3 +394,37 @@ def test_attention_weight_one_head_keeps_the_largest_logits():
                 want = sorted(sorted(toks, key=lambda j: (-logit[j], j))[:lam])
                 assert [int(t) for t in r.kept[ci, st] if t >= 0] == want
         t0 += C
+
+
+# ---------------------------------------------------------------- one feature map per kv-head
+
+def test_per_head_feature_maps_match_set_based_bruteforce():
+    B, Hq, Hkv, d, D = 1, 4, 2, 8, 8
+    ints = [4] * 10
+    T = sum(ints)
+    q, k, v, W0 = _qkvw(B, T, Hq, Hkv, d, D, 230)
+    W = np.stack([W0, _rand((d, D // 2), 234, 1.0 / np.sqrt(d))])
+    r = oracle.run(q, k, v, W, window=5, lambda_=4, intervals=ints, eps=1e-6, want_cands=True)
+    out_b, kept_b, _ = brute.run(q, k, v, W, window=5, lambda_=4, intervals=ints, eps=1e-6)
+    np.testing.assert_allclose(r.out, out_b, rtol=1e-10, atol=1e-12)
+    for ci in range(len(ints)):
+        for st in range(B * Hkv):
+            assert [t for t in r.kept[ci, st] if t >= 0] == kept_b[ci][st]
+
+
+def test_per_head_feature_maps_are_separable_by_head():
+    # each kv-head (with its query heads and its own W) run alone equals its slice of
+    # the joint run: the head -> matrix mapping of keys and queries
+    B, Hq, Hkv, d, D = 2, 6, 3, 8, 8
+    ints = [5] * 8
+    T = sum(ints)
+    q, k, v, _ = _qkvw(B, T, Hq, Hkv, d, D, 240)
+    W = np.stack([_rand((d, D // 2), 250 + h, 1.0 / np.sqrt(d)) for h in range(Hkv)])
+    r = oracle.run(q, k, v, W, window=4, lambda_=5, intervals=ints, eps=1e-6)
+    g = Hq // Hkv
+    for h in range(Hkv):
+        rh = oracle.run(q[:, :, h * g:(h + 1) * g], k[:, :, h:h + 1], v[:, :, h:h + 1], W[h], window=4,
+                        lambda_=5, intervals=ints, eps=1e-6)
+        np.testing.assert_allclose(r.out[:, :, h * g:(h + 1) * g], rh.out, rtol=1e-13, atol=1e-15)
+        for b in range(B):
+            np.testing.assert_array_equal(r.kept[:, b * Hkv + h], rh.kept[:, b])
