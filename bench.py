@@ -331,6 +331,18 @@ def run_engine(args, ws, rank, local):
     T = w.seq_len
     q, k, v, _ = wl.make_inputs(w, T=T)
     W = wl.make_W(w)
+    w_job = w                    # the whole job's workload (all ranks)
+    shard = None
+    if args.shard and ws > 1:
+        # this rank's block of the batch's (sequence, kv-head) streams (strong scaling)
+        from hybrid_linear_attention_lola_b200 import shard as SH
+        shard = SH.partition(w.batch, w.n_q_heads, w.n_kv_heads, ws, rank)
+        q = np.ascontiguousarray(q[shard.b0:shard.b1, :, shard.h0 * shard.g:shard.h1 * shard.g])
+        k = np.ascontiguousarray(k[shard.b0:shard.b1, :, shard.h0:shard.h1])
+        v = np.ascontiguousarray(v[shard.b0:shard.b1, :, shard.h0:shard.h1])
+        if w.w_per_head:
+            W = np.ascontiguousarray(W[shard.h0:shard.h1])
+        w = w.replace(batch=shard.batch, n_kv_heads=shard.n_kv_heads, n_q_heads=shard.n_q_heads)
     cfg = L.config_from_workload(w, max_prefill_tokens=T)
     S = L.LolaState(cfg, torch.from_numpy(W), dev)
     dt = S.dtype
@@ -379,7 +391,10 @@ def run_engine(args, ws, rank, local):
     clk = clocks.stop() if clocks else None
     L.lola_set_timing(S.handle, False)
     ms_step = max_over_ranks(sum(times) / len(times), ws, dev)
-    value = whole_job_rate(w.batch * T, ws, ms_step / 1e3)
+    # tokens of the whole job: every rank's own batch (replicas), or one batch split
+    # over the ranks (shard)
+    job_tokens = w_job.batch * T if shard is not None else w.batch * T * ws
+    value = job_tokens / (ms_step / 1e3)
 
     roofline = prefill_roofline(w, T, ms_step, phase_ms, args.steps, peaks, peak_src)
 
@@ -414,7 +429,7 @@ def run_engine(args, ws, rank, local):
         et.append(e0.elapsed_time(e1))
     barrier(ws)
     e2e_ms = max_over_ranks(sum(et) / len(et), ws, dev)
-    e2e = {"value": whole_job_rate(w.batch * T, ws, e2e_ms / 1e3), "unit": UNIT,
+    e2e = {"value": job_tokens / (e2e_ms / 1e3), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 4)}
     S.close()
     del qd, kd, vd, out
@@ -428,13 +443,15 @@ def run_engine(args, ws, rank, local):
 
     line = {"metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": ws,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": f"{w.name} prefill", "batch": w.batch,
-                       "seq_len": T, "n_q_heads": w.n_q_heads, "n_kv_heads": w.n_kv_heads,
+            "higher_is_better": True, "scaling": "strong" if shard is not None else "weak",
+            "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": f"{w_job.name} prefill", "batch": w_job.batch,
+                       "seq_len": T, "n_q_heads": w_job.n_q_heads, "n_kv_heads": w_job.n_kv_heads,
                        "head_dim": w.head_dim, "feat_dim": w.feat_dim, "window": w.window,
                        "lambda": w.lambda_, "chunk": w.chunk,
-                       "parallelism": f"replicas x{ws} (independent streams, no collective)",
+                       "parallelism": (f"streams sharded over {ws} ranks by {shard.by} (no collective on the "
+                                       f"data path)" if shard is not None
+                                       else f"replicas x{ws} (independent streams, no collective)"),
                        "l2": "flushed (256 MiB write) before every timed step"},
             "roofline": roofline, "e2e": e2e, "gpu_launches": launches, "clocks": clk,
             "decode": decode, "memory": memory_report(w, sb)}
@@ -572,6 +589,9 @@ def main(argv=None):
     ap.add_argument("--decode-workload", default="decode-batched,long-context",
                     help="comma-separated decode workloads (or none)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--shard", action="store_true",
+                    help="with N > 1 ranks, split one batch's streams over the ranks (strong "
+                         "scaling) instead of running N replicas")
     ap.add_argument("--batch", type=int, default=None,
                     help="override the prefill workload's batch (smaller cases for profiling)")
     ap.add_argument("--decode-prefix", type=int, default=None,
