@@ -198,6 +198,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     extern __shared__ uint8_t smraw[];
     __shared__ uint64_t bar_x, bar_s[2], bar_o[2];   // setup MMAs; scores of tile i (i & 1); PV of tile i
+    __shared__ uint64_t bar_h;                        // the snapshot H' has landed (bulk copy)
     __shared__ uint32_t tslot;
     __shared__ int okflag;
     const uint32_t raw = umma::smem_u32(smraw);
@@ -222,6 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma::mbar_init(&bar_s[1], 1);
         umma::mbar_init(&bar_o[0], 1);
         umma::mbar_init(&bar_o[1], 1);
+        umma::mbar_init(&bar_h, 1);
     }
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
     umma::fence_before_sync();
@@ -267,9 +269,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::cp_async16(sPr + umma::kmajor_offset(rr, kc * 8, Dh), Wt + (size_t)rr * d + kc * 8);
         }
     }
-    // the snapshot: H' as an N-contiguous [FP][d] operand, then s' as row 0 of a K-major 16 x FP operand
+    // the snapshot: H' as an N-contiguous [FP][d] operand, stored in exactly that layout: one
+    // bulk copy, in flight during Z and phi(Q) (waited for before the readout); then s' as
+    // row 0 of a K-major 16 x FP operand
     const uint8_t *img = (const uint8_t *)P.snapImg + ((size_t)st * dm.mmax + ci) * (size_t)(FP * (d + 16) * 2);
-    for (int e = tid; e < FP * d * 2 / 16; e += kThreads) umma::cp_async16(sH + e * 16, img + e * 16);
+    if (tid == 0) {
+        umma::mbar_arrive_expect_tx(&bar_h, (uint32_t)(FP * d * 2));
+        umma::bulk_g2s(sH, img, (uint32_t)(FP * d * 2), &bar_h);
+    }
     for (int f = tid; f < FP; f += kThreads)
         sS[f] = __bfloat162float(*(const bf16 *)(img + (size_t)FP * d * 2 + umma::kmajor_offset(0, f, 16)));
     umma::cp_async_commit();
@@ -379,8 +386,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t id_g = umma::idesc_bf16(128, KT, false, false);
     const uint32_t id_one = umma::idesc_bf16(128, 16, false, false);   // P x ones: weight sums
     const uint32_t id_pv = umma::idesc_bf16(128, d, false, true);
+    bool h_wt = false;   // thread 0: the snapshot copy was waited for
     if (ok) {
         if (tid == 0) {
+            h_wt = umma::mbar_wait_abortable(&bar_h, 0, kWaitNs, S.err, ERR_TIMEOUT);
+            if (!h_wt) raise_error(S.err, ERR_TIMEOUT);   // the MMA wait below gives up at once
             umma::fence_after_sync();
             const uint32_t a0 = umma::smem_u32(sPhq);
             mma_kn(tO, a0, 128, umma::smem_u32(sH), d, FP / 16, id_pv, false);
@@ -709,6 +719,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ---- drain: every MMA of this CTA is complete before its buffers and TMEM go away
     umma::cp_async_wait_all();
     if (tid == 0) {
+        if (!h_wt) umma::mbar_wait(&bar_h, 0, kWaitNs);   // no copy outlives the CTA
         umma::mma_commit(&bar_x);
         const bool dok = umma::mbar_wait(&bar_x, xph & 1u, kWaitNs);
         if (!dok) raise_error(S.err, ERR_TIMEOUT);

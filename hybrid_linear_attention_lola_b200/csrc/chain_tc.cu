@@ -336,15 +336,17 @@ __device__ bool fold_tc(Ctx &c, const int *lst, int cnt, const bf16 *__restrict_
         umma::fence_async_smem();
         umma::fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 || tid == 32) {
+            // two issuing threads, value columns (thread 0) and the normaliser column
+            // (thread 32): different TMEM columns, issued side by side; both commit
             umma::fence_after_sync();
             const uint32_t b1 = umma::smem_u32(B1), on = umma::smem_u32(c.ones);
             for (int bk = 0; bk < g.nblk; ++bk) {
                 const uint32_t a0 = umma::smem_u32(Af + (size_t)bk * 64 * 128 * 2);
                 for (int ks = 0; ks < ntp / 16; ++ks) {
                     const uint64_t ad = umma::mnmajor_desc(a0, ks, 128);
-                    umma::mma_ss(tH(c, bk), ad, umma::mnmajor_desc(b1, ks, g.d), id_h, 1u);
-                    umma::mma_ss(tH(c, bk) + (uint32_t)g.d, ad, umma::kmajor_desc(on, ks, 16), id_s, 1u);
+                    if (tid == 0) umma::mma_ss(tH(c, bk), ad, umma::mnmajor_desc(b1, ks, g.d), id_h, 1u);
+                    else umma::mma_ss(tH(c, bk) + (uint32_t)g.d, ad, umma::kmajor_desc(on, ks, 16), id_s, 1u);
                 }
             }
             umma::mma_commit(c.mbar);
@@ -415,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     if (tid == 0) {
-        umma::mbar_init(&mbar, 1);
+        umma::mbar_init(&mbar, 2);   // two issuing threads commit per MMA batch
         umma::mbar_init(&tbar[0], 1);
         umma::mbar_init(&tbar[1], 1);
         umma::mbar_init(&never, 1);
@@ -576,8 +578,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int hd = d >> 1;                            // value dims per thread
         for (int lt = 0; lt < nmy && ok; ++lt) {
             const int m0 = (crank + lt * nc) * 128, nr = min(128, nQ - m0);
-            if (tid == 0) {
-                // the tile's rows have landed (a timeout stops the MMA wait below at once)
+            if (tid == 0 || tid == 32) {
+                // the tile's rows have landed (a timeout stops the MMA wait below at once);
+                // thread 0 issues the numerator columns, thread 32 the denominator column
                 const int bsel = lt % g.nbuf;
                 const bool got = umma::mbar_wait_abortable(&tbar[bsel], twait[bsel] & 1u, kWaitNs, S.err, ERR_TIMEOUT);
                 if (got) ++twait[bsel];
@@ -587,8 +590,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t bh = umma::smem_u32(c.Bimg), bs = umma::smem_u32(c.Bs);
                 for (int ks = 0; ks < g.FP / 16; ++ks) {
                     const uint64_t ad = umma::kmajor_desc(a0, ks, 128);
-                    umma::mma_ss(tS(c), ad, umma::mnmajor_desc(bh, ks, d), id_sh, ks > 0 ? 1u : 0u);
-                    umma::mma_ss(tS(c) + (uint32_t)d, ad, umma::kmajor_desc(bs, ks, 16), id_ss, ks > 0 ? 1u : 0u);
+                    if (tid == 0) umma::mma_ss(tS(c), ad, umma::mnmajor_desc(bh, ks, d), id_sh, ks > 0 ? 1u : 0u);
+                    else umma::mma_ss(tS(c) + (uint32_t)d, ad, umma::kmajor_desc(bs, ks, 16), id_ss, ks > 0 ? 1u : 0u);
                 }
                 umma::mma_commit(c.mbar);
             }
