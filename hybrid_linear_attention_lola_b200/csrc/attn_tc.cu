@@ -221,8 +221,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         umma::mbar_init(&bar_x, 1);
         umma::mbar_init(&bar_s[0], 1);
         umma::mbar_init(&bar_s[1], 1);
-        umma::mbar_init(&bar_o[0], 1);
-        umma::mbar_init(&bar_o[1], 1);
+        umma::mbar_init(&bar_o[0], 2);   // PV (thread 0) and the row sums (thread 32) of tile i
+        umma::mbar_init(&bar_o[1], 2);
         umma::mbar_init(&bar_h, 1);
     }
     if (warp == 0) umma::tmem_alloc(&tslot, g.ncols);
@@ -589,11 +589,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 
     float m = 0.f;
+    int last_i = -1;                                  // last key tile whose MMAs were issued
     const int nch = (d + 16) / 16, split = nch / 2;   // O chunks (sums included) rescaled by half 0 / 1
     const float c1 = scale * 1.4426950408889634f;        // e^{x scale} = 2^{x c1}
     for (int i = 0; i < n && ok; ++i) {
-        // scores of tile i; everything issued before them (PV of tile i-2) is complete
+        // scores of tile i; everything thread 0 issued before them (PV of tile i-2) is complete
         if (!(ok = wait_mbar(&bar_s[i & 1], (uint32_t)((i >> 1) & 1), &okflag, S.err))) break;
+        if (i >= 2) {
+            // and the row sums of tile i-2 (thread 32): their weight buffer is rewritten below
+            if (lane == 0) {
+                const bool okw = umma::mbar_wait_abortable(&bar_o[i & 1], (uint32_t)(((i - 2) >> 1) & 1), kWaitNs,
+                                                           S.err, ERR_TIMEOUT);
+                if (!okw) raise_error(S.err, ERR_TIMEOUT);
+            }
+            __syncwarp();
+        }
         meta_store(i + NK + 1, pf_tok, pf_vr, pf_info);   // into the slot of tile i-1
         meta_load(i + NK + 2, pf_tok, pf_vr, pf_info);    // in flight during this tile
         issue_k(i + NK);        // into the buffer of tile i's keys
@@ -707,19 +717,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncthreads();
         if (tid == 0) {
             umma::fence_after_sync();
-            const uint32_t p0 = umma::smem_u32(sP);
-            mma_kn(tO, p0, 128, umma::smem_u32(vbuf(i)), d, KT / 16, id_pv, true);
-            // the row sums of the rounded weights the tensor core multiplied, into column d
-            mma_kk(tO + (uint32_t)d, p0, 128, umma::smem_u32(sOnes), 16, KT / 16, id_one, true);
+            mma_kn(tO, umma::smem_u32(sP), 128, umma::smem_u32(vbuf(i)), d, KT / 16, id_pv, true);
             umma::mma_commit(&bar_o[i & 1]);
             if (i + 2 < n) issue_qk(i + 2);
+        } else if (tid == 32) {
+            // the row sums of the rounded weights the tensor core multiplied, into column d,
+            // issued beside the PV by a second thread (other TMEM columns)
+            umma::fence_after_sync();
+            mma_kk(tO + (uint32_t)d, umma::smem_u32(sP), 128, umma::smem_u32(sOnes), 16, KT / 16, id_one, true);
+            umma::mma_commit(&bar_o[i & 1]);
         }
+        last_i = i;
     }
 
     // ---- drain: every MMA of this CTA is complete before its buffers and TMEM go away
     umma::cp_async_wait_all();
     if (tid == 0) {
         if (!h_wt) umma::mbar_wait(&bar_h, 0, kWaitNs);   // no copy outlives the CTA
+        // the row sums of the last two tiles (thread 32's MMAs) are complete too
+        for (int j = last_i - 1; j <= last_i; ++j)
+            if (j >= 0) umma::mbar_wait(&bar_o[j & 1], (uint32_t)((j >> 1) & 1), kWaitNs);
         umma::mma_commit(&bar_x);
         const bool dok = umma::mbar_wait(&bar_x, xph & 1u, kWaitNs);
         if (!dok) raise_error(S.err, ERR_TIMEOUT);
