@@ -157,6 +157,7 @@ lola_status derive_dims(const lola_config *c, Dims *dm)
                        ? 1 : 0;
     if (!dm->tc_chain && lola::chain_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     dm->tc_attn = dm->tc_chain;
+    dm->attn_ws = dm->tc_attn && lola::attn_ws_supported(*dm) ? 1 : 0;
     if (lola::attn_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     if (c->dtype == LOLA_BF16 && lola::phi_tc_smem_bytes(*dm) > 227 * 1024) return LOLA_ERR_INVALID_ARG;
     return LOLA_OK;
@@ -187,6 +188,7 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.pend = (uint8_t *)take(ns * dm.Lmax);
     s.W = (float *)take((size_t)dm.nW * dm.d * dm.Dh * 4);
     s.Wt = take((size_t)dm.nW * dm.d * dm.Dh * e);
+    s.WtImg = (dm.dtype == LOLA_BF16 && dm.d % 64 == 0) ? take((size_t)dm.nW * dm.d * dm.Dh * 2) : nullptr;
     s.phiV = take(ns * (dm.lam + dm.R) * dm.D * e);
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     s.phiQd = (float *)take(dm.dtype == LOLA_BF16 ? (size_t)dm.B * dm.Hq * dm.D * 4 : 0);
@@ -513,6 +515,18 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     const int seg = st->seg_len > 0 ? st->seg_len : m;
     const int nseg = (m + seg - 1) / seg;
     const bool fork = nseg > 1 && st->chain_stream != nullptr;
+    lola::AttnMaps amaps;
+    if (dm.attn_ws) {
+        lola::AttnArgs ma{};
+        ma.n_call = n;
+        ma.q = q;
+        ma.kin = k;
+        ma.vin = v;
+        if (!lola::make_attn_maps(dm, ma, st->P.phiK, &amaps)) {
+            fprintf(stderr, "lola: cuTensorMapEncodeTiled failed (prefill attention maps)\n");
+            return LOLA_ERR_CUDA;
+        }
+    }
     cudaStream_t cs = fork ? st->chain_stream : stream;
     if (fork) {
         cudaEventRecord(st->ev_fork, stream);
@@ -574,7 +588,8 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         aa.out = out;
         {
             PhaseScope ps(st, PH_ATTN, stream);
-            if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
+            if (dm.attn_ws) lola::launch_attn_ws(dm, st->S, st->P, aa, amaps, stream);
+            else if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
             else lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
             counted(1);
         }

@@ -35,6 +35,7 @@ struct Dims {
     int dec_minper;   // decode (bf16): fewest work items per warp (fewer for few streams)
     int tc_chain;     // 1: tensor-core chain (bf16), 0: SIMT chain
     int tc_attn;      // 1: tensor-core prefill attention (bf16, head_dim % 64 == 0)
+    int attn_ws;      // 1: its warp-specialised form (feature half a multiple of 64, 128 % g == 0)
     int scorer;       // cache scoring: 0 SRE, 1 attention weight, 2 softmax-approximation error, 3 recency
     int nW;           // feature-map matrices: 1 (shared) or Hkv (one per kv-head)
     float eps;
@@ -50,6 +51,8 @@ struct DevState {
     uint8_t *pend;     // [ns][Lmax]   1 = leaving pair of the last interval that is folded
     float *W;          // [nW][d][Dh]  feature-map matrices (one per kv-head, or one shared), fp32 copy
     void *Wt;          // [nW][Dh][d]  W transposed, in the input dtype (tensor-core operand)
+    void *WtImg;       // [nW][Dh * d] bfloat16 W^T as a K-major 128-byte-swizzled operand image
+                       //              (Dh rows, d columns; bfloat16 states with d % 64 == 0)
     int *err;          // [4]          device error words
     // decode scratch (phi buffers hold the input dtype)
     void *phiV;        // [ns][lam + R][D] phi of cache slots and ring rows (decode interval)
@@ -274,6 +277,18 @@ void launch_attn_prefill(const Dims &dm, const DevState &S, const PrefillScratch
                          const AttnArgs &a, cudaStream_t stream);
 void launch_attn_tc(const Dims &dm, const DevState &S, const PrefillScratch &P, const AttnArgs &a,
                     cudaStream_t stream);
+// Warp-specialised tensor-core prefill attention (bfloat16, two query tiles per CTA).
+// Tensor maps of one call: q [B * n][Hq][d] (boxes of 128 query rows of one
+// kv-head group), k and v [B * n][Hkv][d] (boxes of 64 tokens of one kv-head),
+// and the phi rows [ns * (lam + R + Nmax)][D] (64-row boxes).
+struct AttnMaps {
+    CUtensorMap q, k, v, phik;
+};
+bool attn_ws_supported(const Dims &dm);
+size_t attn_ws_smem_bytes(const Dims &dm);
+bool make_attn_maps(const Dims &dm, const AttnArgs &a, const void *phiK, AttnMaps *maps);
+void launch_attn_ws(const Dims &dm, const DevState &S, const PrefillScratch &P, const AttnArgs &a,
+                    const AttnMaps &maps, cudaStream_t stream);
 void launch_finalize_prefill(const Dims &dm, const DevState &S, const PrefillScratch &P,
                              const void *kin, const void *vin, long long call_start, int n,
                              int nK, cudaStream_t stream);
@@ -288,6 +303,9 @@ struct DecMaps {
 // 128-byte swizzle, zero fill past the extent (box_rows 1: tile::gather4 loads);
 // false if encoding fails.
 bool make_row_map(CUtensorMap *m, const void *base, unsigned long long rows, int cols, int box_rows);
+// 3-D map of a bfloat16 array [d2][d1][d0] with 64 x box1 x box2 boxes, 128-byte
+// swizzle, zero fill past the extent; false if encoding fails.
+bool make_map_3d(CUtensorMap *m, const void *base, int d0, int d1, unsigned long long d2, int box1, int box2);
 
 struct DecodeArgs {
     long long pos;          // token index of this step

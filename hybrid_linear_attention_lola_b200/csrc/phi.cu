@@ -3,6 +3,7 @@
 // "Probleemstelling"; the two-sided softmax form is this engine's fixed choice),
 // and state initialisation.
 #include "lola_internal.cuh"
+#include "umma.cuh"
 
 namespace lola {
 
@@ -143,6 +144,10 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
             const long long h = e / per, r = e - h * per;
             const long long a = r / dm.Dh, i = r - a * dm.Dh;
             Wt[h * per + i * dm.d + a] = W[e];
+            // the same W^T as a K-major operand image (Dh rows, d columns, 128-byte
+            // swizzle): one bulk copy puts it in shared memory ready for the tensor core
+            if (S.WtImg != nullptr)
+                ((T *)S.WtImg)[h * per + umma::kmajor_offset((int)i, (int)a, dm.Dh) / 2] = W[e];
         }
     }
     if (tid < 4) S.err[tid] = 0;

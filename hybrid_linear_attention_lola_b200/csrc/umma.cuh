@@ -205,22 +205,36 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// One potentially blocking probe of an mbarrier phase (acquire, CTA scope): the
+// thread sleeps until the phase completes or a hardware time slice runs out.
+__device__ __forceinline__ bool mbar_try(uint32_t a, uint32_t parity)
+{
+    uint32_t done;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}\n"
+        : "=r"(done)
+        : "r"(a), "r"(parity)
+        : "memory");
+    return done != 0;
+}
+
+// Probes between two looks at the clock (and the error word) while a wait is
+// unfinished: a hand-off that completes within them costs no timer read and no
+// global load.
+constexpr int kProbesPerCheck = 16;
+
 // Waits for the mbarrier phase `parity`; gives up after limit_ns nanoseconds of
 // wall time (measured with %globaltimer) and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t *mbar, uint32_t parity, uint64_t limit_ns)
 {
     const uint32_t a = smem_u32(mbar);
+    if (mbar_try(a, parity)) return true;
     const uint64_t start = globaltimer_ns();
     for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (done) return true;
+        for (int k = 0; k < kProbesPerCheck; ++k)
+            if (mbar_try(a, parity)) return true;
         if (globaltimer_ns() - start > limit_ns) return false;
     }
 }
@@ -239,15 +253,21 @@ __device__ __forceinline__ bool mbar_test(uint64_t *mbar, uint32_t parity)
     return done != 0;
 }
 
-// As mbar_wait, but gives up at once when *err already holds a bit of abort_mask
-// (another thread of the grid gave up). The error word, a global read, is only
-// consulted when the phase is not complete at the first probe.
+// As mbar_wait, but also gives up when *err holds a bit of abort_mask (another
+// thread of the grid gave up). The error word, a global read, is only consulted
+// between rounds of probes of an unfinished wait.
 __device__ __forceinline__ bool mbar_wait_abortable(uint64_t *mbar, uint32_t parity, uint64_t limit_ns,
                                                     const int *err, int abort_mask)
 {
-    if (mbar_test(mbar, parity)) return true;
-    if ((*(const volatile int *)err & abort_mask) != 0) return false;
-    return mbar_wait(mbar, parity, limit_ns);
+    const uint32_t a = smem_u32(mbar);
+    if (mbar_try(a, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        for (int k = 0; k < kProbesPerCheck; ++k)
+            if (mbar_try(a, parity)) return true;
+        if ((*(const volatile int *)err & abort_mask) != 0) return false;
+        if (globaltimer_ns() - start > limit_ns) return false;
+    }
 }
 
 // Expects `bytes` more transaction bytes on the mbarrier and arrives once.
@@ -344,40 +364,45 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint32_t remote_bar)
 {
     asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(remote_bar) : "memory");
 }
-// bounded wait with cluster-scope acquire (pairs with mbar_arrive_cluster)
-__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *mbar, uint32_t parity, uint64_t limit_ns)
-{
-    const uint32_t a = smem_u32(mbar);
-    const uint64_t start = globaltimer_ns();
-    for (;;) {
-        uint32_t done;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}\n"
-            : "=r"(done)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (done) return true;
-        if (globaltimer_ns() - start > limit_ns) return false;
-    }
-}
-// mbar_wait_cluster that gives up at once when *err holds a bit of abort_mask; the
-// error word is only read when the phase is not complete at the first probe
-__device__ __forceinline__ bool mbar_wait_cluster_abortable(uint64_t *mbar, uint32_t parity, uint64_t limit_ns,
-                                                            const int *err, int abort_mask)
+// one potentially blocking probe with cluster-scope acquire (pairs with mbar_arrive_cluster)
+__device__ __forceinline__ bool mbar_try_cluster(uint32_t a, uint32_t parity)
 {
     uint32_t done;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.test_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}\n"
         : "=r"(done)
-        : "r"(smem_u32(mbar)), "r"(parity)
+        : "r"(a), "r"(parity)
         : "memory");
-    if (done) return true;
-    if ((*(const volatile int *)err & abort_mask) != 0) return false;
-    return mbar_wait_cluster(mbar, parity, limit_ns);
+    return done != 0;
+}
+// bounded wait with cluster-scope acquire
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *mbar, uint32_t parity, uint64_t limit_ns)
+{
+    const uint32_t a = smem_u32(mbar);
+    if (mbar_try_cluster(a, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        for (int k = 0; k < kProbesPerCheck; ++k)
+            if (mbar_try_cluster(a, parity)) return true;
+        if (globaltimer_ns() - start > limit_ns) return false;
+    }
+}
+// mbar_wait_cluster that also gives up when *err holds a bit of abort_mask; the error
+// word is only read between rounds of probes of an unfinished wait
+__device__ __forceinline__ bool mbar_wait_cluster_abortable(uint64_t *mbar, uint32_t parity, uint64_t limit_ns,
+                                                            const int *err, int abort_mask)
+{
+    const uint32_t a = smem_u32(mbar);
+    if (mbar_try_cluster(a, parity)) return true;
+    const uint64_t start = globaltimer_ns();
+    for (;;) {
+        for (int k = 0; k < kProbesPerCheck; ++k)
+            if (mbar_try_cluster(a, parity)) return true;
+        if ((*(const volatile int *)err & abort_mask) != 0) return false;
+        if (globaltimer_ns() - start > limit_ns) return false;
+    }
 }
 // full cluster barrier (every thread of every CTA of the cluster)
 __device__ __forceinline__ void cluster_sync()
@@ -410,6 +435,19 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem)
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
                  : "memory");
+}
+// 16-byte asynchronous copy of `bytes` (0 or 16) source bytes; the rest of the 16
+// destination bytes are zero (src must still be a valid address)
+__device__ __forceinline__ void cp_async16_zfill(void *smem, const void *gmem, uint32_t bytes)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(smem)), "l"(gmem), "r"(bytes)
+                 : "memory");
+}
+// Arrive (without raising the expected count) on the mbarrier once every cp.async this
+// thread issued so far has landed.
+__device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *mbar)
+{
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(mbar)) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }

@@ -174,7 +174,12 @@ def test_gqa_group_of_eight_and_eps_zero():
 
 
 # ---------------------------------------------------------------- edge cases (bfloat16)
-# head_dim 64 keeps these on the tensor-core chain and attention and the streaming decode
+# head_dim 64 keeps these on the tensor-core chain and attention and the streaming decode.
+# Feature dim 64 (feature half 32) takes the single-tile attention kernel, feature dim
+# 128 the warp-specialised one (two query tiles per CTA where the interval has them).
+
+ATTN = pytest.mark.parametrize("feat", [64, 128], ids=["tile-attn", "ws-attn"])
+
 
 def _small_bf16(**kw):
     base = dict(head_dim=64, feat_dim=64, dtype="bf16")
@@ -182,21 +187,24 @@ def _small_bf16(**kw):
     return _small(**base)
 
 
-def test_bf16_no_window_no_cache_is_linear_attention():
-    w = _small_bf16(window=0, lambda_=0, decode_interval=1)
-    _case(w, [("prefill", 64), ("decode", 16)], modes=("free",), name="bf16 linear only")
+@ATTN
+def test_bf16_no_window_no_cache_is_linear_attention(feat):
+    w = _small_bf16(window=0, lambda_=0, decode_interval=1, feat_dim=feat)
+    _case(w, [("prefill", 64), ("decode", 16)], modes=("free",), name=f"bf16 linear only D{feat}")
 
 
-def test_bf16_chunk_longer_than_window_ragged_tiles():
+@ATTN
+def test_bf16_chunk_longer_than_window_ragged_tiles(feat):
     # partial cache and window tiles, query rows past the interval, and kept leaving
     # pairs that are later than some queries of their interval (chunk > window)
-    w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6)
-    _case(w, [("prefill", 240), ("decode", 13)], modes=ALL, name="bf16 chunk > window, ragged")
+    w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6, feat_dim=feat)
+    _case(w, [("prefill", 240), ("decode", 13)], modes=ALL, name=f"bf16 chunk > window, ragged D{feat}")
 
 
-def test_bf16_zero_window_with_cache():
-    w = _small_bf16(window=0, lambda_=9, chunk=8, decode_interval=1)
-    _case(w, [("prefill", 80), ("decode", 5)], modes=ALL, name="bf16 zero window")
+@ATTN
+def test_bf16_zero_window_with_cache(feat):
+    w = _small_bf16(window=0, lambda_=9, chunk=8, decode_interval=1, feat_dim=feat)
+    _case(w, [("prefill", 80), ("decode", 5)], modes=ALL, name=f"bf16 zero window D{feat}")
 
 
 def test_bf16_gqa_group_of_eight():
@@ -204,10 +212,29 @@ def test_bf16_gqa_group_of_eight():
     _case(w, [("prefill", 160)], modes=ALL, name="bf16 GQA 8")
 
 
-def test_bf16_token_by_token():
+@ATTN
+def test_bf16_token_by_token(feat):
     # C = C_dec = 1 on the tensor-core chain and attention and the streaming decode
-    w = _small_bf16(window=16, lambda_=24, chunk=1, decode_interval=1, n_q_heads=4, n_kv_heads=2)
-    _case(w, [("prefill", 96), ("decode", 32)], modes=ALL, name="bf16 token-by-token")
+    w = _small_bf16(window=16, lambda_=24, chunk=1, decode_interval=1, n_q_heads=4, n_kv_heads=2, feat_dim=feat)
+    _case(w, [("prefill", 96), ("decode", 32)], modes=ALL, name=f"bf16 token-by-token D{feat}")
+
+
+@ATTN
+def test_bf16_decode_then_prefill_then_decode(feat):
+    # the second prefill call starts with window and band rows from the ring (16-byte
+    # gathers instead of tiled loads) and cached pairs of the earlier calls
+    w = _small_bf16(window=16, lambda_=40, chunk=16, decode_interval=8, n_q_heads=8, n_kv_heads=2,
+                    batch=2, feat_dim=feat)
+    _case(w, [("prefill", 32), ("decode", 24), ("prefill", 48), ("decode", 20)], modes=ALL,
+          name=f"bf16 decode/prefill interleaved D{feat}")
+
+
+@ATTN
+def test_bf16_long_chunk_two_band_chunks(feat):
+    # chunk 128 > 64: two band chunks per interval and four query tiles per interval
+    w = _small_bf16(window=64, lambda_=96, chunk=128, decode_interval=32, n_q_heads=8, n_kv_heads=2,
+                    feat_dim=feat)
+    _case(w, [("prefill", 512), ("decode", 64)], modes=ALL, name=f"bf16 chunk 128 D{feat}")
 
 
 def test_bf16_head_dim_32():
