@@ -27,11 +27,11 @@
 //   the interval folds); the band weights -G/s- of folded leaving pairs still
 //   inside a row's window go through one P V product per 64-key chunk.
 // Main loop, per 64-key tile (window keys [t0 - eta, t1), then the interval's
-// cached keys): S = Q K^T, P = e^{s - m} with a lazily moved shift m, O += P V and
-// the row sums of P (one more MMA against a ones operand). Key and value tiles
+// cached keys): S = Q K^T, P = e^{s - m} with a lazily moved shift m, O += P V; each
+// softmax thread keeps the sum of its row's rounded weights. Key and value tiles
 // stream through shared-memory rings: window tiles of this call's tokens as tiled
 // TMA boxes, others (scattered cache rows) by 16-byte cp.async gathers.
-// Finally out = O / (l + eps e^{-m}).
+// Finally out = O / (l + sum of weights + eps e^{-m}).
 // Every wait is bounded; a timeout sets the device error word and every role
 // leaves its loop, drains its copies and MMAs, and the CTA exits.
 #include "lola_internal.cuh"
@@ -61,7 +61,7 @@ struct TileMeta {
 };
 
 // Shared memory (offsets from a 1024-byte aligned base):
-//   [Q tiles][ones][metadata ring][X]
+//   [Q tiles][metadata ring][X]
 // X during the setup: [phi(Q) half of each tile (W^T first)][H' half][s' half]
 //                     [phi(K_L) half per band chunk] ... [V_L per band chunk]
 // X in the main loop: [P of each tile][key ring][value ring]
@@ -70,7 +70,7 @@ struct TileMeta {
 struct WGeo {
     int d, D, Dh, nq, nch, NBa, NK, NV;
     size_t qtile, ptile, tileb;
-    size_t off_ones, off_meta, off_X;
+    size_t off_meta, off_X;
     size_t x_hh, x_sh, x_pk, x_vl, x_K, x_V;
     size_t total;
 };
@@ -91,8 +91,7 @@ inline WGeo make_wgeo_n(const Dims &dm, int nq, int NK, int NV)
     g.qtile = (size_t)128 * dm.d * 2;
     g.ptile = (size_t)128 * KT * 2;
     g.tileb = (size_t)KT * dm.d * 2;
-    g.off_ones = (size_t)nq * g.qtile;
-    g.off_meta = g.off_ones + 16 * KT * 2;
+    g.off_meta = (size_t)nq * g.qtile;
     g.off_X = al(g.off_meta + (size_t)kMS * sizeof(TileMeta), 1024);
     const size_t pq = (size_t)nq * 128 * g.Dh * 2, wt = (size_t)g.Dh * dm.d * 2;
     g.x_hh = al(pq > wt ? pq : wt, 1024);
@@ -155,10 +154,11 @@ __device__ __forceinline__ void mma_kn(uint32_t dt, uint32_t a0, int ra, uint32_
     for (int ks = 0; ks < nks; ++ks)
         umma::mma_ss(dt, da + kstep_k(ks, ra), db + (uint64_t)(ks * sb), idesc, (acc || ks > 0) ? 1u : 0u);
 }
-// O += P V and the row sums of P: P is a K-major 128 x 64 weight tile, V a 64-key value
-// tile in the [n/64][key][128 B] layout (N-contiguous; 64-column blocks KT * 128 bytes
-// apart, 8-key groups 1024 bytes apart)
-__device__ __forceinline__ void mma_pv(uint32_t dt, uint32_t p0, uint32_t v0, int d, uint32_t ones0)
+// O += P V: P is a K-major 128 x 64 weight tile, V a 64-key value tile in the
+// [n/64][key][128 B] layout (N-contiguous; 64-column blocks KT * 128 bytes apart,
+// 8-key groups 1024 bytes apart). The row sums of P are kept by the softmax threads
+// (a 128 x 16 MMA against a ones operand costs as much issue time as a 128 x 64 one).
+__device__ __forceinline__ void mma_pv(uint32_t dt, uint32_t p0, uint32_t v0, int d)
 {
     const uint64_t da = umma::kmajor_desc(p0, 0, 128);
     const uint64_t db = umma::make_desc(v0, (uint32_t)(KT * 128), 1024);
@@ -166,7 +166,13 @@ __device__ __forceinline__ void mma_pv(uint32_t dt, uint32_t p0, uint32_t v0, in
 #pragma unroll
     for (int ks = 0; ks < KT / 16; ++ks)
         umma::mma_ss(dt, da + kstep_k(ks, 128), db + (uint64_t)((ks * 2048) >> 4), id_pv, 1u);
-    mma_kk(dt + (uint32_t)d, p0, 128, ones0, 16, KT / 16, umma::idesc_bf16(128, 16, false, false), true);
+}
+
+// sum of the eight bf16 values of four packed pairs
+__device__ __forceinline__ float sum_bf16x8(uint32_t a, uint32_t b, uint32_t c, uint32_t d)
+{
+    return (umma::bf16lo_to_f32(a) + umma::bf16hi_to_f32(a)) + (umma::bf16lo_to_f32(b) + umma::bf16hi_to_f32(b)) +
+           (umma::bf16lo_to_f32(c) + umma::bf16hi_to_f32(c)) + (umma::bf16lo_to_f32(d) + umma::bf16hi_to_f32(d));
 }
 
 // fp32 x scalar over n columns (n a multiple of 16) of this warp's 32 TMEM lanes
@@ -231,7 +237,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t raw = umma::smem_u32(smraw);
     uint8_t *base = smraw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *sX = base + G.off_X;
-    uint8_t *sOnes = base + G.off_ones;
     TileMeta *meta = (TileMeta *)(base + G.off_meta);
     uint8_t *sHH = sX + G.x_hh, *sSH = sX + G.x_sh, *sPK = sX + G.x_pk, *sVL = sX + G.x_vl;
     auto sQ = [&](int q) { return base + (size_t)q * G.qtile; };
@@ -288,18 +293,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::mbar_init(&bread[q], 4);
         }
     }
-    // ones operand: row 0 of a K-major 16 x 64 tile (row sums of P)
-    for (int e = tid; e < 16 * KT; e += kThreads) {
-        const int rr = e / KT, k = e - rr * KT;
-        *(bf16 *)(sOnes + umma::kmajor_offset(rr, k, 16)) = __float2bfloat16_rn(rr == 0 ? 1.f : 0.f);
-    }
     if (warp == kWarpM) umma::tmem_alloc(&tslot, 512);
     umma::fence_async_smem();
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tm = tslot;
-    // TMEM: O of tile q (d columns + the sums column d) at q * NBa; score / band buffer
+    // TMEM: O of tile q (d columns + the linear denominator in column d) at q * NBa; score / band buffer
     // of tile q and chunk c after them; Z of tile q at q * Dh (setup only)
     auto tO = [&](int q) { return tm + (uint32_t)(q * G.NBa); };
     auto tG = [&](int q, int c) { return tm + (uint32_t)(G.nq * G.NBa + (c * G.nq + q) * KT); };
@@ -560,19 +560,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             bool ok = true;
             int u = 0;   // uses of the weight buffers (band chunks, then key tiles)
-            auto pv_step = [&](int j) -> bool {
-                if (!waitb(&vfull[j % NV], (uint32_t)((j / NV) & 1), err)) return false;
-                umma::fence_async_smem();   // the gathered rows (generic-proxy copies) to the tensor core
-                for (int q = 0; q < nqe; ++q) {
-                    if (!waitb(&pfull[q], (uint32_t)(u & 1), err)) return false;
-                    umma::fence_after_sync();
-                    mma_pv(tO(q), umma::smem_u32(sP(q)), umma::smem_u32(vbuf(j)), d, umma::smem_u32(sOnes));
-                    umma::mma_commit(&pfree[q]);
-                }
-                ++u;
-                umma::mma_commit(&vempty[j % NV]);
-                return true;
-            };
             // Z = Q W
             if ((ok = waitb(&bq, 0, err))) {
                 umma::fence_after_sync();
@@ -602,30 +589,67 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int q = 0; q < nqe && ok; ++q) {
                     if (!(ok = waitb(&pfull[q], (uint32_t)(u & 1), err))) break;
                     umma::fence_after_sync();
-                    mma_pv(tO(q), umma::smem_u32(sP(q)), umma::smem_u32(sVL + (size_t)c * G.tileb), d,
-                           umma::smem_u32(sOnes));
+                    mma_pv(tO(q), umma::smem_u32(sP(q)), umma::smem_u32(sVL + (size_t)c * G.tileb), d);
                     umma::mma_commit(&pfree[q]);
                 }
                 ++u;
             }
             umma::mma_commit(&bband);   // V_L is free once these products are done
-            // key tiles: S(i) of both tiles, then the P V products of tile i - 1
+            // key tiles, an event loop over the two query tiles: S_q(i) = Q_q K(i)^T goes out
+            // once the key tile has landed and tile q's softmax has read S_q(i - 1); P_q V(j)
+            // once the value tile has landed and tile q's weights are written. The two tiles
+            // never wait for each other; a key (value) buffer is released after both tiles'
+            // products that read it.
             const uint32_t id_s = umma::idesc_bf16(128, KT, false, false);
-            for (int i = 0; i < n && ok; ++i) {
-                if (!(ok = waitb(&kfull[i % NK], (uint32_t)((i / NK) & 1), err))) break;
-                umma::fence_async_smem();   // the gathered rows (generic-proxy copies) to the tensor core
-                for (int q = 0; q < nqe && ok; ++q) {
-                    if (!(ok = i == 0 ? waitb(&bread[q], 0, err) : waitb(&sfree[q], (uint32_t)((i - 1) & 1), err)))
-                        break;
+            int qk[2] = {0, 0}, pv[2] = {0, 0};
+            for (int q = nqe; q < 2; ++q) qk[q] = pv[q] = n;   // no such tile
+            uint64_t t_last = 0;
+            unsigned idle = 0;
+            while (ok && (pv[0] < n || pv[1] < n)) {
+                bool prog = false;
+                for (int q = 0; q < nqe; ++q) {
+                    const int i = qk[q];
+                    if (i >= n) continue;
+                    if (!umma::mbar_test(&kfull[i % NK], (uint32_t)((i / NK) & 1))) continue;
+                    if (!(i == 0 ? umma::mbar_test(&bread[q], 0) : umma::mbar_test(&sfree[q], (uint32_t)((i - 1) & 1))))
+                        continue;
+                    umma::fence_async_smem();   // the gathered rows (generic-proxy copies) to the tensor core
                     umma::fence_after_sync();
                     mma_kk(tG(q, 0), umma::smem_u32(sQ(q)), 128, umma::smem_u32(kbuf(i)), KT, d / 16, id_s, false);
                     umma::mma_commit(&sfull[q]);
+                    qk[q] = i + 1;
+                    if (qk[0] > i && qk[1] > i) umma::mma_commit(&kempty[i % NK]);
+                    prog = true;
                 }
-                if (!ok) break;
-                umma::mma_commit(&kempty[i % NK]);
-                if (i >= 1 && !(ok = pv_step(i - 1))) break;
+                for (int q = 0; q < nqe; ++q) {
+                    const int j = pv[q];
+                    if (j >= qk[q]) continue;
+                    if (!umma::mbar_test(&vfull[j % NV], (uint32_t)((j / NV) & 1))) continue;
+                    if (!umma::mbar_test(&pfull[q], (uint32_t)((nchi + j) & 1))) continue;
+                    umma::fence_async_smem();
+                    umma::fence_after_sync();
+                    mma_pv(tO(q), umma::smem_u32(sP(q)), umma::smem_u32(vbuf(j)), d);
+                    umma::mma_commit(&pfree[q]);
+                    pv[q] = j + 1;
+                    if (pv[0] > j && pv[1] > j) umma::mma_commit(&vempty[j % NV]);
+                    prog = true;
+                }
+                if (prog) {
+                    idle = 0;
+                    continue;
+                }
+                // nothing ready: back off; give up after kWaitNs without progress, or at once
+                // once another thread has recorded an error
+                if (idle++ == 0) t_last = umma::globaltimer_ns();
+                __nanosleep(32);
+                if ((idle & 255u) == 0) {
+                    if ((*(const volatile int *)err & ERR_TIMEOUT) != 0) ok = false;
+                    else if (umma::globaltimer_ns() - t_last > kWaitNs) {
+                        raise_error(err, ERR_TIMEOUT);
+                        ok = false;
+                    }
+                }
             }
-            if (ok && n >= 1) ok = pv_step(n - 1);
             umma::mma_commit(&bdone);
             // every MMA of this CTA is complete before TMEM and the buffers go away
             umma::mma_commit(&bdrain);
@@ -717,6 +741,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         const float rsn = 1.f / sn;
         int u = 0;
+        float lsum = 0.f;   // sum of the row's rounded weights (band and softmax), at shift m
         if (ok && (ok = waitw(&bpass[1], 0, err))) {
             umma::fence_after_sync();
             tmem_scale(tO(q) + lo, d + 16, rsn);   // O = phi(Q) H1, column d = phi(Q).s1
@@ -755,9 +780,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float w[8];
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) w[jj] = ((sub >> (j0w + jj)) & 1ull) ? -gv[j0w + jj] * rsn : 0.f;
-                    *(uint4 *)(myP + umma::kmajor_offset(r, j0w, 128)) =
-                        u4(umma::pack_bf16x2(w[0], w[1]), umma::pack_bf16x2(w[2], w[3]),
-                           umma::pack_bf16x2(w[4], w[5]), umma::pack_bf16x2(w[6], w[7]));
+                    const uint4 pw = u4(umma::pack_bf16x2(w[0], w[1]), umma::pack_bf16x2(w[2], w[3]),
+                                        umma::pack_bf16x2(w[4], w[5]), umma::pack_bf16x2(w[6], w[7]));
+                    lsum += sum_bf16x8(pw.x, pw.y, pw.z, pw.w);
+                    *(uint4 *)(myP + umma::kmajor_offset(r, j0w, 128)) = pw;
                 }
                 umma::fence_async_smem();
                 umma::fence_before_sync();
@@ -859,11 +885,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_scale(tO(q) + lo, d + 16, grow_m ? __expf(m - tmax) : 1.f);
                 umma::tmem_wait_st();
             }
+            if (grow_m) lsum *= __expf(m - tmax);
             m = mnew;
 #pragma unroll
-            for (int w = 0; w < 8; ++w)
+            for (int w = 0; w < 8; ++w) {
+                lsum += sum_bf16x8(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
                 *(uint4 *)(myP + umma::kmajor_offset(r, 8 * w, 128)) =
                     u4(pk[4 * w], pk[4 * w + 1], pk[4 * w + 2], pk[4 * w + 3]);
+            }
             umma::fence_async_smem();
             umma::fence_before_sync();
             __syncwarp();
@@ -880,7 +909,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float v[16];
             umma::tmem_ld16(tO(q) + lo + (uint32_t)d, v);
             umma::tmem_wait_ld();
-            const float rden = 1.f / (v[0] + dm.eps * __expf(-m));
+            const float rden = 1.f / (v[0] + lsum + dm.eps * __expf(-m));
             bf16 *out = (bf16 *)a.out;
             const size_t orow = ((size_t)b * a.n_call + (size_t)(t0 - a.pos0) + (size_t)(grow / gq)) * dm.Hq +
                                 (size_t)hk * gq + grow % gq;
