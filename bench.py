@@ -39,9 +39,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch of a kernel, copied from ncu captures (profiles/dram_traffic.json);
 # an entry counts only while the kernel's source file is unchanged since its capture
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "dram_traffic.json")
-KERNEL_SOURCES = {"attn": "hybrid_linear_attention_lola_b200/csrc/attn_tc.cu",
-                  "chain": "hybrid_linear_attention_lola_b200/csrc/chain_tc.cu",
-                  "decode": "hybrid_linear_attention_lola_b200/csrc/decode.cu"}
+_CSRC = "hybrid_linear_attention_lola_b200/csrc/"
+_HEADERS = (_CSRC + "umma.cuh", _CSRC + "lola_internal.cuh")
+KERNEL_SOURCES = {"attn": (_CSRC + "attn_ws.cu",) + _HEADERS,
+                  "chain": (_CSRC + "chain_tc.cu", _CSRC + "scoring.cuh") + _HEADERS,
+                  "decode": (_CSRC + "decode.cu",) + _HEADERS}
 
 
 # ---------------------------------------------------------------- helpers
@@ -59,10 +61,14 @@ def host_cores() -> int:
     return len(os.sched_getaffinity(0))
 
 
-def source_sha(rel: str) -> str:
+def source_sha(rels) -> str:
+    """Hash of a kernel's source files (its .cu and the headers it includes)."""
     import hashlib
-    with open(os.path.join(ROOT, rel), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for rel in ((rels,) if isinstance(rels, str) else rels):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def captured_traffic(kernel: str, workload: str):
