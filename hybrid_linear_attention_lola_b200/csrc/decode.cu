@@ -726,12 +726,34 @@ template <int CPR> __device__ __forceinline__ uint32_t swz(int r, int c)
     return (uint32_t)((c >> 3) * 32 * 128 + r * 128 + (((c & 7) ^ (r & 7)) << 4));
 }
 
+// Launches `kernel` as a programmatic dependent of the previous kernel on the stream:
+// it may start while that one still runs and orders itself with griddep_wait().
+template <typename... P, typename... A>
+void launch_dependent(void (*kernel)(P...), int grid, int block, size_t smem, cudaStream_t stream, A... args)
+{
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)grid);
+    cfg.blockDim = dim3((unsigned)block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, kernel, args...);
+}
+
 // Step preparation (bfloat16 path): phi(q) of every query row into an fp32
 // scratch, and, when the step appends, the new pair into the window ring with
 // phi(k) of it in the phi rows. One warp per row; W (fp32) in shared memory.
+// The streaming kernel that follows is launched as a programmatic dependent: it
+// starts at once and waits for this grid only before it reads phi(q) or the
+// appended pair.
 template <typename T>
 __global__ void __launch_bounds__(256) decode_prep_kernel(Dims dm, DevState S, DecodeArgs a, int do_append)
 {
+    umma::griddep_launch_dependents();
     extern __shared__ float smp[];
     const int d = dm.d, Dh = dm.Dh, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     float *Ws = smp;
@@ -837,6 +859,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         if (it < IT.nkc && tma) {
             if (lane == 0) {
                 const bool cache = it < IT.ncc;
+                if (!cache) umma::griddep_wait();   // window rows include the pair the preparation appends
                 const int y = cache ? it * 32 : ((IT.wblk0 + (it - IT.ncc)) & ((R >> 5) - 1)) * 32;
                 const CUtensorMap *mk = cache ? &maps.ks : &maps.kr;
                 const CUtensorMap *mv = cache ? &maps.vs : &maps.vr;
@@ -850,6 +873,7 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
         } else if (it < IT.nkc) {
             const int k0 = it * 32;
             const int nv = min(32, IT.nsoft - k0);
+            if (k0 + 32 > nS) umma::griddep_wait();   // window rows (the appended pair among them)
             if (lane == 0) umma::mbar_arrive_expect_tx(bar, (uint32_t)nv * 2 * d * E);
             __syncwarp();
             uint8_t *kd = buf + (size_t)lane * RS, *vd = buf + KTB + (size_t)lane * RS;
@@ -918,6 +942,10 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
     // false: the wait for the previous stream's phi(q) copy gave up (error word set)
     auto begin = [&](int st) -> bool {
         const int b = st / dm.Hkv, hk = st % dm.Hkv;
+        // linear-band or state items of st in this warp's range need phi(q); a warp with
+        // only key chunks of st neither copies it nor waits for the preparation
+        const long long st_end = min((long long)st * ni + ni, i0 + nmine);
+        const bool wantq = (int)(st_end - 1 - (long long)st * ni) >= IT.nkc;
         const T *qg = (const T *)a.q + ((size_t)b * dm.Hq + (size_t)hk * g) * d;
         const bool hv = gq < g;
 #pragma unroll
@@ -936,15 +964,19 @@ __global__ void __launch_bounds__(128) decode_stream_kernel(Dims dm, DevState S,
                 okq = umma::mbar_wait(&mb[NST], (nbeg - 1) & 1u, kWaitNs);
                 if (!okq) raise_error(S.err, ERR_TIMEOUT);
             }
-            if (okq) {
+            if (okq && wantq) {
+                umma::griddep_wait();   // phi(q) is written by the preparation grid
                 umma::mbar_arrive_expect_tx(&mb[NST], (uint32_t)(g * D * 4));
                 umma::bulk_g2s(phq, S.phiQd + ((size_t)b * dm.Hq + (size_t)hk * g) * D, (uint32_t)(g * D * 4),
                                &mb[NST]);
             }
         }
         if (__shfl_sync(0xffffffffu, okq ? 1 : 0, 0) == 0) return false;
-        ++nbeg;
-        need_q = true;
+        need_q = false;   // the previous stream's copy has landed (waited for above)
+        if (wantq) {
+            ++nbeg;
+            need_q = true;
+        }
         const int nL = (int)(a.L_hi - a.L_lo);
         for (int i = lane; i < nL; i += 32) fate[i] = S.pend[(size_t)st * dm.Lmax + i];
         mrow = 0.f;
@@ -1464,7 +1496,7 @@ void launch_decode_attn(const Dims &dm, const DevState &S, const DecodeArgs &a, 
                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);          \
             attr = smem;                                                                           \
         }                                                                                          \
-        decode_stream_kernel<DPL, GG, NB><<<grid, nw * 32, smem, stream>>>(dm, S, a, (int)per, wb, mp); \
+        launch_dependent(decode_stream_kernel<DPL, GG, NB>, grid, nw * 32, smem, stream, dm, S, a, (int)per, wb, mp); \
     } while (0)
 #define LOLA_STREAM(DPL, GG)                                                                       \
     do {                                                                                           \
