@@ -31,11 +31,15 @@ struct lola_state {
     int pend_n;
     long long n_int;         // update intervals run since init/reset
     bool phiV_valid;         // phi rows of the cache slots and the ring are current
-    // prefill segments: chain on a high-priority library stream, attention on the caller's
+    // prefill segments: chain on a high-priority library stream, the attention of even
+    // segments on the caller's stream and of odd segments on a second library stream, so
+    // that a segment's last partial wave of CTAs overlaps the next segment's first
     static constexpr int kMaxSeg = 64;
     int seg_len;                     // intervals per segment (0: the whole call)
     cudaStream_t chain_stream;
+    cudaStream_t attn_stream;
     cudaEvent_t ev_fork;
+    cudaEvent_t ev_attn;             // the second attention stream's work of a call is done
     cudaEvent_t ev_seg[kMaxSeg];
     lola::DecMaps maps;              // TMA descriptors of the cache / ring arrays (bf16 decode)
     CUtensorMap phik_map, phik_box;  // row maps (1-row and 128-row boxes) of the prefill and the
@@ -410,6 +414,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->timing = false;
     st->seg_len = 0;
     st->chain_stream = nullptr;
+    st->attn_stream = nullptr;
     if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
         // segments of at least 8 intervals, at most kMaxSeg of them per call
         int len = dm.mmax / 32;
@@ -418,11 +423,15 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
         int lo = 0, hi = 0;
         bool okc = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
                    cudaStreamCreateWithPriority(&st->chain_stream, cudaStreamNonBlocking, hi) == cudaSuccess &&
-                   cudaEventCreateWithFlags(&st->ev_fork, cudaEventDisableTiming) == cudaSuccess;
+                   cudaStreamCreateWithPriority(&st->attn_stream, cudaStreamNonBlocking, lo) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&st->ev_fork, cudaEventDisableTiming) == cudaSuccess &&
+                   cudaEventCreateWithFlags(&st->ev_attn, cudaEventDisableTiming) == cudaSuccess;
         for (int i = 0; okc && i < lola_state::kMaxSeg; ++i)
             okc = cudaEventCreateWithFlags(&st->ev_seg[i], cudaEventDisableTiming) == cudaSuccess;
         if (!okc) {
             cudaGetLastError();
+            if (st->chain_stream != nullptr) cudaStreamDestroy(st->chain_stream);
+            if (st->attn_stream != nullptr) cudaStreamDestroy(st->attn_stream);
             delete st;
             return LOLA_ERR_CUDA;
         }
@@ -437,6 +446,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
         fprintf(stderr, "lola: cuTensorMapEncodeTiled failed (phi row maps)\n");
         cudaGetLastError();
         if (st->chain_stream != nullptr) cudaStreamDestroy(st->chain_stream);
+        if (st->attn_stream != nullptr) cudaStreamDestroy(st->attn_stream);
         delete st;
         return LOLA_ERR_CUDA;
     }
@@ -444,6 +454,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
         fprintf(stderr, "lola: cuTensorMapEncodeTiled failed\n");
         cudaGetLastError();
         if (st->chain_stream != nullptr) cudaStreamDestroy(st->chain_stream);
+        if (st->attn_stream != nullptr) cudaStreamDestroy(st->attn_stream);
         delete st;
         return LOLA_ERR_CUDA;
     }
@@ -528,9 +539,11 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         }
     }
     cudaStream_t cs = fork ? st->chain_stream : stream;
+    const bool two = fork && st->attn_stream != nullptr;
     if (fork) {
         cudaEventRecord(st->ev_fork, stream);
         cudaStreamWaitEvent(cs, st->ev_fork, 0);
+        if (two) cudaStreamWaitEvent(st->attn_stream, st->ev_fork, 0);
     }
     for (int sg = 0; sg < nseg; ++sg) {
         const int ci0 = sg * seg;
@@ -571,9 +584,12 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
             counted(1);
         }
         if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+        // the attention of this segment: on the caller's stream, or (odd segments) on the
+        // second attention stream, after the segment's chain
+        cudaStream_t as = (two && (sg & 1)) ? st->attn_stream : stream;
         if (fork) {
             cudaEventRecord(st->ev_seg[sg], cs);
-            cudaStreamWaitEvent(stream, st->ev_seg[sg], 0);
+            cudaStreamWaitEvent(as, st->ev_seg[sg], 0);
         }
         for (int ci = 0; ci < ms; ++ci) advance_interval(st, pos0 + (long long)(ci0 + ci) * dm.C, dm.C);
 
@@ -587,13 +603,18 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         aa.vin = v;
         aa.out = out;
         {
-            PhaseScope ps(st, PH_ATTN, stream);
-            if (dm.attn_ws) lola::launch_attn_ws(dm, st->S, st->P, aa, amaps, stream);
-            else if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, stream);
-            else lola::launch_attn_prefill(dm, st->S, st->P, aa, stream);
+            PhaseScope ps(st, PH_ATTN, as);
+            if (dm.attn_ws) lola::launch_attn_ws(dm, st->S, st->P, aa, amaps, as);
+            else if (dm.tc_attn) lola::launch_attn_tc(dm, st->S, st->P, aa, as);
+            else lola::launch_attn_prefill(dm, st->S, st->P, aa, as);
             counted(1);
         }
         if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+    }
+    if (two) {
+        // the caller's stream joins the second attention stream before the finalisation
+        cudaEventRecord(st->ev_attn, st->attn_stream);
+        cudaStreamWaitEvent(stream, st->ev_attn, 0);
     }
 
     {
@@ -719,6 +740,11 @@ lola_status lola_free_state(lola_state *st)
         cudaStreamDestroy(st->chain_stream);
         cudaEventDestroy(st->ev_fork);
         for (int i = 0; i < lola_state::kMaxSeg; ++i) cudaEventDestroy(st->ev_seg[i]);
+    }
+    if (st->attn_stream != nullptr) {
+        cudaStreamSynchronize(st->attn_stream);
+        cudaStreamDestroy(st->attn_stream);
+        cudaEventDestroy(st->ev_attn);
     }
     delete st;
     return LOLA_OK;

@@ -107,8 +107,10 @@ inline WGeo make_wgeo_n(const Dims &dm, int nq, int NK, int NV)
     return g;
 }
 
-// Two query tiles per CTA where TMEM and shared memory allow, then the deepest
-// rings that fit (keys one deeper than values).
+// Two query tiles per CTA (the kernel exists to share every key and value tile between
+// them; with one tile per CTA the single-tile kernel, whose eight warps all gather and
+// all run the softmax, is faster), then the deepest rings that fit (keys one deeper
+// than values). Other shapes take the single-tile kernel.
 inline bool make_wgeo(const Dims &dm, WGeo *out)
 {
     if (dm.dtype != 1 || !dm.tc_chain || dm.d % 64 != 0 || (dm.D / 2) % 64 != 0 || 128 % dm.g != 0 || dm.lam <= 0)
@@ -116,7 +118,7 @@ inline bool make_wgeo(const Dims &dm, WGeo *out)
     const int tpi = (dm.C * dm.g + 127) / 128;
     const int nch = (dm.C + KT - 1) / KT;
     const int NBa = (dm.d + 16 + 31) / 32 * 32;
-    for (int nq = tpi >= 2 ? 2 : 1; nq >= 1; --nq) {
+    for (int nq = tpi >= 2 ? 2 : 0; nq >= 2; --nq) {
         if (nq * NBa + nq * nch * KT > 512 || nq * (dm.D / 2) > 512) continue;
         for (int s = 2 * kMaxRing; s >= 4; --s) {
             const WGeo g = make_wgeo_n(dm, nq, (s + 1) / 2, s / 2);

@@ -175,8 +175,9 @@ def test_gqa_group_of_eight_and_eps_zero():
 
 # ---------------------------------------------------------------- edge cases (bfloat16)
 # head_dim 64 keeps these on the tensor-core chain and attention and the streaming decode.
-# Feature dim 64 (feature half 32) takes the single-tile attention kernel, feature dim
-# 128 the warp-specialised one (two query tiles per CTA where the interval has them).
+# Feature dim 64 (feature half 32) takes the single-tile attention kernel. The
+# warp-specialised one takes feature dim 128 with intervals of more than 128 query rows
+# (two query tiles per CTA): WS marks the cases whose shape gives it those.
 
 ATTN = pytest.mark.parametrize("feat", [64, 128], ids=["tile-attn", "ws-attn"])
 
@@ -195,9 +196,10 @@ def test_bf16_no_window_no_cache_is_linear_attention(feat):
 
 @ATTN
 def test_bf16_chunk_longer_than_window_ragged_tiles(feat):
-    # partial cache and window tiles, query rows past the interval, and kept leaving
-    # pairs that are later than some queries of their interval (chunk > window)
-    w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6, feat_dim=feat)
+    # partial cache and window tiles, query rows past the interval (192 rows: the second
+    # query tile half full), and kept leaving pairs that are later than some queries of
+    # their interval (chunk > window)
+    w = _small_bf16(window=5, lambda_=37, chunk=48, decode_interval=6, n_q_heads=8, n_kv_heads=2, feat_dim=feat)
     _case(w, [("prefill", 240), ("decode", 13)], modes=ALL, name=f"bf16 chunk > window, ragged D{feat}")
 
 
@@ -222,10 +224,11 @@ def test_bf16_token_by_token(feat):
 @ATTN
 def test_bf16_decode_then_prefill_then_decode(feat):
     # the second prefill call starts with window and band rows from the ring (16-byte
-    # gathers instead of tiled loads) and cached pairs of the earlier calls
-    w = _small_bf16(window=16, lambda_=40, chunk=16, decode_interval=8, n_q_heads=8, n_kv_heads=2,
+    # gathers instead of tiled loads) and cached pairs of the earlier calls; 256 query
+    # rows per interval
+    w = _small_bf16(window=16, lambda_=40, chunk=32, decode_interval=8, n_q_heads=16, n_kv_heads=2,
                     batch=2, feat_dim=feat)
-    _case(w, [("prefill", 32), ("decode", 24), ("prefill", 48), ("decode", 20)], modes=ALL,
+    _case(w, [("prefill", 64), ("decode", 24), ("prefill", 64), ("decode", 20)], modes=ALL,
           name=f"bf16 decode/prefill interleaved D{feat}")
 
 
