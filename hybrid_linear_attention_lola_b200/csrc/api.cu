@@ -41,6 +41,10 @@ struct lola_state {
     cudaEvent_t ev_fork;
     cudaEvent_t ev_attn;             // the second attention stream's work of a call is done
     cudaEvent_t ev_seg[kMaxSeg];
+    // prefill from host memory: copy streams (host to device, device to host) and the
+    // events of the two staging slots (created at the first such call)
+    cudaStream_t h2d_stream, d2h_stream;
+    cudaEvent_t ev_h2d[2], ev_comp[2], ev_d2h[2], ev_host;
     lola::DecMaps maps;              // TMA descriptors of the cache / ring arrays (bf16 decode)
     CUtensorMap phik_map, phik_box;  // row maps (1-row and 128-row boxes) of the prefill and the
     CUtensorMap phiv_map, phiv_box;  // decode phi rows (tensor-core chain)
@@ -353,6 +357,42 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
 
 }  // namespace
 
+namespace {
+
+// Staging of lola_prefill_host: two slots, each holding a piece's q, k, v and out.
+struct HostSlot {
+    size_t q, kv, total;   // bytes of the q (and out) piece, of a k (or v) piece, of a slot
+};
+HostSlot host_slot(const Dims &dm, int64_t piece)
+{
+    HostSlot h;
+    const size_t e = elem_bytes(dm);
+    h.q = (size_t)dm.B * piece * dm.Hq * dm.d * e;
+    h.kv = (size_t)dm.B * piece * dm.Hkv * dm.d * e;
+    h.total = 2 * align_up(h.q) + 2 * align_up(h.kv);
+    return h;
+}
+
+bool make_host_streams(lola_state *st)
+{
+    if (st->h2d_stream != nullptr) return true;
+    bool ok = cudaStreamCreateWithFlags(&st->h2d_stream, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&st->d2h_stream, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&st->ev_host, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < 2; ++i)
+        ok = cudaEventCreateWithFlags(&st->ev_h2d[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&st->ev_comp[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaEventCreateWithFlags(&st->ev_d2h[i], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) {
+        // the handles created so far stay valid until lola_free_state destroys them
+        cudaGetLastError();
+        return false;
+    }
+    return true;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char *lola_status_string(lola_status s)
@@ -415,6 +455,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->seg_len = 0;
     st->chain_stream = nullptr;
     st->attn_stream = nullptr;
+    st->h2d_stream = st->d2h_stream = nullptr;
     if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
         // segments of at least 8 intervals, at most kMaxSeg of them per call
         int len = dm.mmax / 32;
@@ -628,6 +669,73 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     return check_launch();
 }
 
+lola_status lola_prefill_host_staging_bytes(const lola_config *cfg, int64_t piece_tokens, size_t *bytes)
+{
+    if (!bytes) return LOLA_ERR_INVALID_ARG;
+    Dims dm;
+    const lola_status r = derive_dims(cfg, &dm);
+    if (r != LOLA_OK) return r;
+    if (piece_tokens <= 0 || piece_tokens % dm.C != 0) return LOLA_ERR_SHAPE;
+    if (piece_tokens > dm.Nmax) return LOLA_ERR_WORKSPACE;
+    *bytes = 2 * host_slot(dm, piece_tokens).total;
+    return LOLA_OK;
+}
+
+lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, const void *v, int64_t n_tokens,
+                              void *out, void *staging, size_t staging_bytes, int64_t piece_tokens,
+                              void *cuda_stream)
+{
+    if (!st || !q || !k || !v || !out || !staging) return LOLA_ERR_INVALID_ARG;
+    const Dims &dm = st->dm;
+    if (n_tokens <= 0 || n_tokens % dm.C != 0 || piece_tokens <= 0 || piece_tokens % dm.C != 0)
+        return LOLA_ERR_SHAPE;
+    if (piece_tokens > dm.Nmax) return LOLA_ERR_WORKSPACE;
+    if (((uintptr_t)staging & (kAlign - 1)) != 0) return LOLA_ERR_INVALID_ARG;
+    const HostSlot hs = host_slot(dm, piece_tokens);
+    if (staging_bytes < 2 * hs.total) return LOLA_ERR_WORKSPACE;
+    if (st->pos != st->interval_end) return LOLA_ERR_STATE;
+    if (!make_host_streams(st)) return LOLA_ERR_CUDA;
+    cudaStream_t stream = (cudaStream_t)cuda_stream;
+    const size_t e = elem_bytes(dm);
+    const size_t qrow = (size_t)dm.Hq * dm.d * e, kvrow = (size_t)dm.Hkv * dm.d * e;   // bytes per token
+    // the copy streams start after the caller's earlier work (which may still use the staging)
+    cudaEventRecord(st->ev_host, stream);
+    cudaStreamWaitEvent(st->h2d_stream, st->ev_host, 0);
+    cudaStreamWaitEvent(st->d2h_stream, st->ev_host, 0);
+    int i = 0;
+    for (int64_t t0 = 0; t0 < n_tokens; t0 += piece_tokens, ++i) {
+        const int64_t len = n_tokens - t0 < piece_tokens ? n_tokens - t0 : piece_tokens;
+        const int slot = i & 1;
+        char *qd = (char *)staging + (size_t)slot * hs.total;
+        char *kd = qd + align_up(hs.q), *vd = kd + align_up(hs.kv), *od = vd + align_up(hs.kv);
+        // inputs of this piece (rows t0 .. t0 + len of every sequence) into the slot, once the
+        // compute of the piece two back has read it
+        if (i >= 2) cudaStreamWaitEvent(st->h2d_stream, st->ev_comp[slot], 0);
+        cudaMemcpy2DAsync(qd, (size_t)len * qrow, (const char *)q + (size_t)t0 * qrow, (size_t)n_tokens * qrow,
+                          (size_t)len * qrow, (size_t)dm.B, cudaMemcpyHostToDevice, st->h2d_stream);
+        cudaMemcpy2DAsync(kd, (size_t)len * kvrow, (const char *)k + (size_t)t0 * kvrow, (size_t)n_tokens * kvrow,
+                          (size_t)len * kvrow, (size_t)dm.B, cudaMemcpyHostToDevice, st->h2d_stream);
+        cudaMemcpy2DAsync(vd, (size_t)len * kvrow, (const char *)v + (size_t)t0 * kvrow, (size_t)n_tokens * kvrow,
+                          (size_t)len * kvrow, (size_t)dm.B, cudaMemcpyHostToDevice, st->h2d_stream);
+        cudaEventRecord(st->ev_h2d[slot], st->h2d_stream);
+        // the piece: its inputs have landed and the slot's outputs of two pieces back are out
+        cudaStreamWaitEvent(stream, st->ev_h2d[slot], 0);
+        if (i >= 2) cudaStreamWaitEvent(stream, st->ev_d2h[slot], 0);
+        const lola_status r = lola_prefill_chunk(st, qd, kd, vd, len, od, stream);
+        if (r != LOLA_OK) return r;
+        cudaEventRecord(st->ev_comp[slot], stream);
+        // its outputs back to the host rows
+        cudaStreamWaitEvent(st->d2h_stream, st->ev_comp[slot], 0);
+        cudaMemcpy2DAsync((char *)out + (size_t)t0 * qrow, (size_t)n_tokens * qrow, od, (size_t)len * qrow,
+                          (size_t)len * qrow, (size_t)dm.B, cudaMemcpyDeviceToHost, st->d2h_stream);
+        cudaEventRecord(st->ev_d2h[slot], st->d2h_stream);
+    }
+    // the caller's stream passes this call once the last output copy is done
+    cudaEventRecord(st->ev_host, st->d2h_stream);
+    cudaStreamWaitEvent(stream, st->ev_host, 0);
+    return check_launch();
+}
+
 lola_status lola_decode_step(lola_state *st, const void *q, const void *k, const void *v,
                              void *out, void *cuda_stream)
 {
@@ -745,6 +853,18 @@ lola_status lola_free_state(lola_state *st)
         cudaStreamSynchronize(st->attn_stream);
         cudaStreamDestroy(st->attn_stream);
         cudaEventDestroy(st->ev_attn);
+    }
+    if (st->h2d_stream != nullptr) {
+        cudaStreamSynchronize(st->h2d_stream);
+        cudaStreamSynchronize(st->d2h_stream);
+        cudaStreamDestroy(st->h2d_stream);
+        cudaStreamDestroy(st->d2h_stream);
+        for (int i = 0; i < 2; ++i) {
+            cudaEventDestroy(st->ev_h2d[i]);
+            cudaEventDestroy(st->ev_comp[i]);
+            cudaEventDestroy(st->ev_d2h[i]);
+        }
+        cudaEventDestroy(st->ev_host);
     }
     delete st;
     return LOLA_OK;

@@ -11,16 +11,20 @@
 //       otherwise                                      -> softmax (inside the window)
 //   * the readout phi(q)^T H', phi(q)^T s' of the state.
 //
-// One kernel per step streams everything a step reads exactly once from HBM.
-// A stream's work is cut into items of 32 rows: key chunks (32 keys: their key
-// and value rows) and state chunks (32 feature rows of H and s). The items are
-// dealt round-robin to the warps of the stream's CTAs; every warp copies its
-// next items into a ring of shared-memory buffers with bulk asynchronous copies
-// (TMA, one mbarrier per buffer) while it works on the current one. Scores:
-// one lane per key against the g queries of the group (shared memory). P V:
-// one lane per pair of value dimensions, the key weights broadcast from shared
-// memory. The online-softmax state of every warp is merged at the end, across
-// the CTAs of a stream by the last CTA to finish (a per-stream counter).
+// A step streams everything it reads once from HBM. bfloat16: a preparation
+// kernel computes phi(q) and appends the new pair; the streaming kernel, launched
+// as its programmatic dependent, cuts every stream's work into items -- key chunks
+// (32 keys: their key and value rows, 128-byte-swizzled TMA tiles), linear-band
+// chunks (16 leaving pairs: phi and value rows) and state chunks (16 feature rows
+// of H and s) -- and gives every warp a contiguous run of the items of all
+// streams, staged through the warp's own ring of shared-memory buffers (one
+// mbarrier per buffer) while it works on the current one. A key chunk is one
+// mma.sync m16n8k16 pass for Q K^T (the group's heads as the M rows) and one for
+// P V, the score fragments reused as the P operand; band and state chunks run on
+// the CUDA cores. A warp leaving a stream writes its partial (shift, softmax and
+// linear sums per head); the warp that writes a stream's last partial merges them
+// (a per-stream counter). float32: one kernel (decode3_kernel) does the same with
+// SIMT scores and a per-CTA split of each stream.
 #include "lola_internal.cuh"
 #include "umma.cuh"
 

@@ -60,6 +60,8 @@ def load_library() -> ctypes.CDLL:
         "lola_init_state": (I32, [C, P, P, SZ, P, ctypes.POINTER(P)]),
         "lola_reset_state": (I32, [P, P]),
         "lola_prefill_chunk": (I32, [P, P, P, P, I64, P, P]),
+        "lola_prefill_host": (I32, [P, P, P, P, I64, P, P, SZ, I64, P]),
+        "lola_prefill_host_staging_bytes": (I32, [C, I64, ctypes.POINTER(SZ)]),
         "lola_decode_step": (I32, [P, P, P, P, P, P]),
         "lola_decode_step_static": (I32, [P, P, P, P, P, P]),
         "lola_position": (I64, [P]),
@@ -149,6 +151,20 @@ def lola_reset_state(h: int, stream: int):
 def lola_prefill_chunk(h: int, q: int, k: int, v: int, n_tokens: int, out: int, stream: int):
     _check(load_library().lola_prefill_chunk(h, q, k, v, n_tokens, out, stream),
            "lola_prefill_chunk")
+
+
+def lola_prefill_host(h: int, q: int, k: int, v: int, n_tokens: int, out: int, staging: int,
+                      staging_bytes: int, piece_tokens: int, stream: int):
+    """Prefill from host buffers, the copies pipelined with the compute in pieces."""
+    _check(load_library().lola_prefill_host(h, q, k, v, n_tokens, out, staging, staging_bytes,
+                                            piece_tokens, stream), "lola_prefill_host")
+
+
+def lola_prefill_host_staging_bytes(cfg: lola_config, piece_tokens: int) -> int:
+    n = ctypes.c_size_t(0)
+    _check(load_library().lola_prefill_host_staging_bytes(ctypes.byref(cfg), piece_tokens, ctypes.byref(n)),
+           "lola_prefill_host_staging_bytes")
+    return n.value
 
 
 def lola_decode_step(h: int, q: int, k: int, v: int, out: int, stream: int):
@@ -255,6 +271,20 @@ class LolaState:
             out = self.torch.empty_like(q)
         lola_prefill_chunk(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), n,
                            out.data_ptr(), self._stream())
+        return out
+
+    def prefill_host(self, q, k, v, out, piece_tokens, staging=None):
+        """Prefill from host tensors q, k, v (pinned, contiguous, the state's dtype) into
+        the host tensor out; copies and compute overlap piece by piece. staging: a device
+        uint8 tensor of lola_prefill_host_staging_bytes bytes (allocated here if None)."""
+        nbytes = lola_prefill_host_staging_bytes(self.cfg, piece_tokens)
+        if staging is None:
+            staging = self.torch.empty(nbytes, dtype=self.torch.uint8, device=self.device)
+        for t in (q, k, v, out):
+            if t.device.type != "cpu" or not t.is_contiguous() or t.dtype != self.dtype:
+                raise ValueError("prefill_host takes contiguous host tensors of the state's dtype")
+        lola_prefill_host(self.handle, q.data_ptr(), k.data_ptr(), v.data_ptr(), q.shape[1], out.data_ptr(),
+                          staging.data_ptr(), staging.numel(), piece_tokens, self._stream())
         return out
 
     def decode(self, q, k, v, out=None):

@@ -125,6 +125,25 @@ lola_status lola_reset_state(lola_state *st, void *cuda_stream);
 lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, const void *v,
                                int64_t n_tokens, void *out, void *cuda_stream);
 
+/* Chunkwise prefill from host memory: the same computation as lola_prefill_chunk
+ * over n_tokens tokens, with q, k, v and out in HOST memory ([B][n_tokens][heads]
+ * [head_dim], as for lola_prefill_chunk; pinned memory lets the copies run
+ * asynchronously). The call cuts the tokens into pieces of piece_tokens (a positive
+ * multiple of cfg.chunk, at most max_prefill_tokens; the last piece may be shorter
+ * but is a multiple of cfg.chunk) and runs lola_prefill_chunk on each piece in
+ * turn, while the next piece's inputs go to the device and the previous piece's
+ * outputs come back on two copy streams of the library. staging: device memory
+ * owned by the caller, at least lola_prefill_host_staging_bytes(cfg, piece_tokens)
+ * bytes, 256-byte aligned (two slots of q, k, v and out pieces); the call
+ * allocates nothing. The call returns once the work is queued; when cuda_stream
+ * has passed it, every output row is in `out` on the host. Errors as for
+ * lola_prefill_chunk, and LOLA_ERR_WORKSPACE for a staging buffer that is too
+ * small. */
+lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, const void *v, int64_t n_tokens,
+                              void *out, void *staging, size_t staging_bytes, int64_t piece_tokens,
+                              void *cuda_stream);
+lola_status lola_prefill_host_staging_bytes(const lola_config *cfg, int64_t piece_tokens, size_t *bytes);
+
 /* One token per sequence: q [B][n_q_heads][head_dim], k, v [B][n_kv_heads][head_dim],
  * out [B][n_q_heads][head_dim]. When the position is at an interval boundary,
  * an update interval of length decode_interval opens here (score, select, fold);

@@ -106,3 +106,19 @@ def test_no_cache_config_is_sized(lib, dtype):
     n = ctypes.c_size_t(0)
     assert lib.lola_state_bytes(ctypes.byref(cfg), ctypes.byref(n)) == 0
     assert n.value > 0
+
+
+def test_host_prefill_staging_bytes(lib):
+    # two slots of q, k, v and out pieces, each rounded up to 256 bytes
+    w = wl.WORKLOADS["prefill-8b"]
+    cfg = L.config_from_workload(w, max_prefill_tokens=w.seq_len)
+    piece = 4096
+    e = 2
+    q = w.batch * piece * w.n_q_heads * w.head_dim * e
+    kv = w.batch * piece * w.n_kv_heads * w.head_dim * e
+    up = lambda x: (x + 255) // 256 * 256
+    assert L.lola_prefill_host_staging_bytes(cfg, piece) == 2 * (2 * up(q) + 2 * up(kv))
+    n = ctypes.c_size_t(0)
+    assert lib.lola_prefill_host_staging_bytes(ctypes.byref(cfg), 100, ctypes.byref(n)) == 2   # not a multiple of the chunk
+    assert lib.lola_prefill_host_staging_bytes(ctypes.byref(cfg), 2 * w.seq_len, ctypes.byref(n)) == 5  # past max_prefill_tokens
+    assert lib.lola_prefill_host(None, None, None, None, 64, None, None, 0, 64, None) == 1
