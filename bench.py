@@ -413,7 +413,7 @@ def run_engine(args, ws, rank, local):
     oh = torch.empty(qh.shape, dtype=dt).pin_memory()
     h2d = qh.numel() * qh.element_size() + kh.numel() * kh.element_size() * 2
     d2h = oh.numel() * oh.element_size()
-    piece = max(w.chunk, (T // 4) // w.chunk * w.chunk)
+    piece = max(w.chunk, (T // max(1, args.e2e_pieces)) // w.chunk * w.chunk)
     staging = torch.empty(L.lola_prefill_host_staging_bytes(S.cfg, piece), dtype=torch.uint8, device=dev)
 
     def e2e_step():
@@ -604,6 +604,9 @@ def main(argv=None):
                     help="override the prefill workload's batch (smaller cases for profiling)")
     ap.add_argument("--decode-prefix", type=int, default=None,
                     help="override the decode workloads' prefilled prefix length")
+    ap.add_argument("--e2e-pieces", type=int, default=4,
+                    help="pieces the end-to-end prefill from host buffers is cut into (copies of one "
+                         "piece overlap the compute of the next)")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="override the number of timed decode steps")
     args = ap.parse_args(argv)
