@@ -604,7 +604,7 @@ def main(argv=None):
                     help="override the prefill workload's batch (smaller cases for profiling)")
     ap.add_argument("--decode-prefix", type=int, default=None,
                     help="override the decode workloads' prefilled prefix length")
-    ap.add_argument("--e2e-pieces", type=int, default=4,
+    ap.add_argument("--e2e-pieces", type=int, default=8,
                     help="pieces the end-to-end prefill from host buffers is cut into (copies of one "
                          "piece overlap the compute of the next)")
     ap.add_argument("--decode-steps", type=int, default=None,
