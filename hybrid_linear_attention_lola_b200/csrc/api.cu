@@ -34,13 +34,17 @@ struct lola_state {
     // prefill segments: chain on a high-priority library stream, the attention of even
     // segments on the caller's stream and of odd segments on a second library stream, so
     // that a segment's last partial wave of CTAs overlaps the next segment's first
-    static constexpr int kMaxSeg = 64;
+    static constexpr int kMaxSeg = lola::kMaxSegments;
     int seg_len;                     // intervals per segment (0: the whole call)
     cudaStream_t chain_stream;
     cudaStream_t attn_stream;
     cudaEvent_t ev_fork;
     cudaEvent_t ev_attn;             // the second attention stream's work of a call is done
     cudaEvent_t ev_seg[kMaxSeg];
+    // one chain launch per call: the attention of segment s waits (stream memory
+    // operation) until seg_done[s] reaches seg_expect[s], the streams' running count
+    bool seg_wait;
+    uint32_t seg_expect[lola::kMaxSegments];
     // prefill from host memory: copy streams (host to device, device to host) and the
     // events of the two staging slots (created at the first such call)
     cudaStream_t h2d_stream, d2h_stream;
@@ -201,6 +205,7 @@ size_t layout(const Dims &dm, char *base, lola::DevState *S, lola::PrefillScratc
     s.part = (float *)take(ns * dm.nsplit * dm.g * (2 * dm.d + 4) * 4);
     s.phiQd = (float *)take(dm.dtype == LOLA_BF16 ? (size_t)dm.B * dm.Hq * dm.D * 4 : 0);
     s.dec_cnt = (int *)take(ns * 4);
+    s.seg_done = (int *)take(lola::kMaxSegments * 4);
     lola::PrefillScratch p{};
     const size_t nv = (size_t)dm.lam + dm.R + dm.Nmax;
     p.phiK = take(ns * nv * dm.D * e);
@@ -359,6 +364,22 @@ lola_status decode_step_impl(lola_state *st, const void *q, const void *k, const
 
 namespace {
 
+// cuStreamWaitValue32: a stream waits until a 32-bit word in device memory reaches a
+// value (no kernel spins; the stream's front end holds the next work)
+using WaitValueFn = CUresult (*)(CUstream, CUdeviceptr, cuuint32_t, unsigned int);
+WaitValueFn wait_value_fn()
+{
+    static WaitValueFn fn = []() -> WaitValueFn {
+        void *f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuStreamWaitValue32", &f, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            return nullptr;
+        return (WaitValueFn)f;
+    }();
+    return fn;
+}
+
 // Staging of lola_prefill_host: two slots, each holding a piece's q, k, v and out.
 struct HostSlot {
     size_t q, kv, total;   // bytes of the q (and out) piece, of a k (or v) piece, of a slot
@@ -455,6 +476,8 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->seg_len = 0;
     st->chain_stream = nullptr;
     st->attn_stream = nullptr;
+    st->seg_wait = wait_value_fn() != nullptr;
+    for (int i = 0; i < lola::kMaxSegments; ++i) st->seg_expect[i] = 0;
     st->h2d_stream = st->d2h_stream = nullptr;
     if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
         // segments of at least 8 intervals, at most kMaxSeg of them per call
@@ -586,50 +609,69 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         cudaStreamWaitEvent(cs, st->ev_fork, 0);
         if (two) cudaStreamWaitEvent(st->attn_stream, st->ev_fork, 0);
     }
+    // With stream memory operations the chain is one launch for the whole call and counts
+    // finished segments in device memory; the attention of segment s waits for its count
+    // (the launch boundaries between chain segments cost the chain about 85 us each, its
+    // SMs briefly free for waiting attention CTAs). Otherwise one chain launch per segment,
+    // the attention gated by an event.
+    const bool one = fork && dm.tc_chain && st->seg_wait && nseg <= lola::kMaxSegments;
     for (int sg = 0; sg < nseg; ++sg) {
         const int ci0 = sg * seg;
         const int ms = m - ci0 < seg ? m - ci0 : seg;
-        lola::ChainArgs ca{};
-        ca.mode = 0;
-        ca.pos0 = pos0 + (long long)ci0 * dm.C;
-        ca.n_int = ms;
-        ca.ilen = dm.C;
-        ca.call_start = pos0;
-        ca.n_call = n;
-        ca.kin = k;
-        ca.vin = v;
-        ca.nS0 = st->nS;
-        ca.pend_lo = st->pend_lo;
-        ca.pend_n = st->pend_n;
-        ca.iglob0 = st->n_int;
-        ca.phi = st->P.phiK;
-        ca.nvrows = dm.lam + dm.R + dm.Nmax;
-        ca.qin = q;
-        ca.q_start = pos0;
-        ca.q_n = n;
-        ca.sel_log = st->sel_log;
-        ca.sel_cap = st->sel_cap;
-        ca.ovr = st->ovr;
-        ca.ovr_n = st->ovr_n;
-        ca.score_sre = st->score_sre;
-        ca.score_tok = st->score_tok;
-        ca.score_cap = st->score_cap;
-        ca.inject_ns = take_injection(st, 1);
-        ca.ci0 = ci0;
-        ca.cont = sg > 0 ? 1 : 0;
-        {
-            PhaseScope ps(st, PH_CHAIN, cs);
-            ca.snap_f32 = dm.tc_attn ? 0 : 1;
-            if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, st->phik_map, st->phik_box, cs);
-            else lola::launch_chain(dm, st->S, &st->P, ca, cs);
-            counted(1);
+        if (!one || sg == 0) {
+            lola::ChainArgs ca{};
+            ca.mode = 0;
+            ca.pos0 = pos0 + (long long)ci0 * dm.C;
+            ca.n_int = one ? m : ms;
+            ca.ilen = dm.C;
+            ca.call_start = pos0;
+            ca.n_call = n;
+            ca.kin = k;
+            ca.vin = v;
+            ca.nS0 = st->nS;
+            ca.pend_lo = st->pend_lo;
+            ca.pend_n = st->pend_n;
+            ca.iglob0 = st->n_int;
+            ca.phi = st->P.phiK;
+            ca.nvrows = dm.lam + dm.R + dm.Nmax;
+            ca.qin = q;
+            ca.q_start = pos0;
+            ca.q_n = n;
+            ca.sel_log = st->sel_log;
+            ca.sel_cap = st->sel_cap;
+            ca.ovr = st->ovr;
+            ca.ovr_n = st->ovr_n;
+            ca.score_sre = st->score_sre;
+            ca.score_tok = st->score_tok;
+            ca.score_cap = st->score_cap;
+            ca.inject_ns = take_injection(st, 1);
+            ca.ci0 = ci0;
+            ca.cont = sg > 0 ? 1 : 0;
+            if (one) {
+                ca.seg_done = st->S.seg_done;
+                ca.seg_len = seg;
+            }
+            {
+                PhaseScope ps(st, PH_CHAIN, cs);
+                ca.snap_f32 = dm.tc_attn ? 0 : 1;
+                if (dm.tc_chain) lola::launch_chain_tc(dm, st->S, &st->P, ca, st->phik_map, st->phik_box, cs);
+                else lola::launch_chain(dm, st->S, &st->P, ca, cs);
+                counted(1);
+            }
+            if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+            if (fork) cudaEventRecord(st->ev_seg[sg], cs);
         }
-        if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
         // the attention of this segment: on the caller's stream, or (odd segments) on the
         // second attention stream, after the segment's chain
         cudaStream_t as = (two && (sg & 1)) ? st->attn_stream : stream;
-        if (fork) {
-            cudaEventRecord(st->ev_seg[sg], cs);
+        if (one) {
+            // every stream's chain has counted this segment (the count runs across calls)
+            const uint32_t target = st->seg_expect[sg] + (uint32_t)dm.ns;
+            st->seg_expect[sg] = target;
+            if (wait_value_fn()((CUstream)as, (CUdeviceptr)(st->S.seg_done + sg), target, CU_STREAM_WAIT_VALUE_GEQ) !=
+                CUDA_SUCCESS)
+                cudaStreamWaitEvent(as, st->ev_seg[0], 0);   // the whole chain, then
+        } else if (fork) {
             cudaStreamWaitEvent(as, st->ev_seg[sg], 0);
         }
         for (int ci = 0; ci < ms; ++ci) advance_interval(st, pos0 + (long long)(ci0 + ci) * dm.C, dm.C);
@@ -657,6 +699,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         cudaEventRecord(st->ev_attn, st->attn_stream);
         cudaStreamWaitEvent(stream, st->ev_attn, 0);
     }
+    if (one) cudaStreamWaitEvent(stream, st->ev_seg[0], 0);   // and the chain
 
     {
         PhaseScope ps(st, PH_FINAL, stream);

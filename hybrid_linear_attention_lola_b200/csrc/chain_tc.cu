@@ -474,6 +474,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
 
     bool ok = true;
+    int seg_sig = 0;   // segments of the call counted in a.seg_done (lead CTA, thread 0)
     const uint32_t id_sh = umma::idesc_bf16(128, d, false, true);
     const uint32_t id_ss = umma::idesc_bf16(128, 16, false, false);
     for (int ci = 0; ci < a.n_int && ok; ++ci) {
@@ -819,6 +820,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         pend_n = nL;
         nS = nK;
         __syncthreads();
+        if (a.seg_done != nullptr && lead && tid == 0 && ((ci + 1) % a.seg_len == 0 || ci == a.n_int - 1)) {
+            // this stream's intervals of the segment are done: its logs (plain stores) and
+            // snapshot images (bulk stores, waited for here) are visible before the count
+            umma::bulk_wait_all();
+            umma::fence_async_global();
+            __threadfence();
+            atomicAdd(&a.seg_done[ci / a.seg_len], 1);
+            seg_sig = ci / a.seg_len + 1;
+        }
     }
 
     if (ok && lead) {
@@ -856,6 +866,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     }
     if (tid == 0) umma::bulk_wait_all();
+    if (a.seg_done != nullptr && lead && tid == 0) {
+        // gave up (or had no interval): count every segment not counted yet
+        __threadfence();
+        const int nseg = (a.n_int + a.seg_len - 1) / a.seg_len;
+        for (int sg = seg_sig; sg < nseg; ++sg) atomicAdd(&a.seg_done[sg], 1);
+    }
     umma::fence_before_sync();
     __syncthreads();
     if (warp == 0) umma::tmem_dealloc(c.tm, g.ncols);

@@ -23,6 +23,7 @@
 namespace lola {
 
 enum : int { ERR_BOUNDS = 1, ERR_TIMEOUT = 2 };
+constexpr int kMaxSegments = 64;   // prefill segments per call, at most
 
 struct Dims {
     int B, Hq, Hkv, g, d, D, Dh, eta, lam, C, Cdec, R, Lmax, ns, dtype;
@@ -59,6 +60,9 @@ struct DevState {
     float *part;       // [ns][nsplit][g][2d + 4] partials of the warps / CTAs sharing a stream
     float *phiQd;      // [B][Hq][D]   fp32 phi(q) of the decode step (bfloat16 path)
     int *dec_cnt;      // [ns] finished decode CTAs per stream (reset by the last one)
+    int *seg_done;     // [kMaxSegments] prefill: streams whose chain has finished a segment of
+                       //   the call, counted up across calls (the attention of a segment waits
+                       //   for its count with a stream memory operation)
 };
 
 // Per-prefill-call scratch.
@@ -253,6 +257,11 @@ struct ChainArgs {
     long long score_cap;
     int snap_f32;           // prefill: also write fp32 (H', s') snapshots
     int ci0;                // prefill: index of the first interval within the call
+    int *seg_done;          // prefill, may be null: the lead CTA of every stream adds 1 to
+    int seg_len;            //   seg_done[s] once it has finished the intervals of segment s
+                            //   (seg_len intervals each; the call's logs and snapshots of them
+                            //   are written and visible), and to every segment left when it
+                            //   gives up, so that no wait for a count is left without it
     int cont;               // prefill: the call's earlier intervals ran in an earlier launch
                             // (slot contents come from the scratch, not the state)
 };

@@ -152,6 +152,10 @@ __global__ void init_state_kernel(Dims dm, DevState S, const T *__restrict__ W)
     }
     if (tid < 4) S.err[tid] = 0;
     for (long long e = tid; e < dm.ns; e += stride) S.dec_cnt[e] = 0;
+    // the segment counts only grow (the host keeps the value each wait expects): zeroed
+    // when the state is created, never by a reset
+    if (W != nullptr && S.seg_done != nullptr)
+        for (long long e = tid; e < kMaxSegments; e += stride) S.seg_done[e] = 0;
 }
 
 void launch_init_state(const Dims &dm, const DevState &S, const void *W, cudaStream_t stream)
