@@ -32,6 +32,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from hybrid_linear_attention_lola_b200 import workloads as wl  # noqa: E402
+from hybrid_linear_attention_lola_b200.lola import SCHEDULES  # noqa: E402
 
 METRIC = "LoLA prefill & decode tokens/sec on 1xB200; % of tensor/HBM roofline"
 UNIT = "tokens/s"
@@ -351,6 +352,7 @@ def run_engine(args, ws, rank, local):
         w = w.replace(batch=shard.batch, n_kv_heads=shard.n_kv_heads, n_q_heads=shard.n_q_heads)
     cfg = L.config_from_workload(w, max_prefill_tokens=T)
     S = L.LolaState(cfg, torch.from_numpy(W), dev)
+    S.set_prefill_schedule(args.prefill_schedule, args.segment_intervals)
     dt = S.dtype
     qd = torch.from_numpy(q).to(dev, dt)
     kd = torch.from_numpy(k).to(dev, dt)
@@ -457,6 +459,8 @@ def run_engine(args, ws, rank, local):
                        "seq_len": T, "n_q_heads": w_job.n_q_heads, "n_kv_heads": w_job.n_kv_heads,
                        "head_dim": w.head_dim, "feat_dim": w.feat_dim, "window": w.window,
                        "lambda": w.lambda_, "chunk": w.chunk,
+                       "prefill_schedule": args.prefill_schedule
+                       + (f", {args.segment_intervals} intervals per segment" if args.segment_intervals else ""),
                        "parallelism": (f"streams sharded over {ws} ranks by {shard.by} (no collective on the "
                                        f"data path)" if shard is not None
                                        else f"replicas x{ws} (independent streams, no collective)"),
@@ -607,6 +611,10 @@ def main(argv=None):
     ap.add_argument("--e2e-pieces", type=int, default=8,
                     help="pieces the end-to-end prefill from host buffers is cut into (copies of one "
                          "piece overlap the compute of the next)")
+    ap.add_argument("--prefill-schedule", default="auto", choices=sorted(SCHEDULES),
+                    help="how a prefill call overlaps its chain and its attention (lola_set_prefill_schedule)")
+    ap.add_argument("--segment-intervals", type=int, default=0,
+                    help="update intervals per prefill segment (0: the library's choice)")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="override the number of timed decode steps")
     args = ap.parse_args(argv)

@@ -1,6 +1,7 @@
 // Host side of the C ABI declared in include/lola.h: argument checks, the
 // workspace layout, and the order in which one prefill call or decode step
 // enqueues its kernels on the caller's stream.
+#include <algorithm>
 #include <atomic>
 #include <cstdio>
 #include <cstring>
@@ -14,6 +15,7 @@
 namespace lola {
 size_t chain_smem_bytes(const Dims &dm);
 size_t attn_smem_bytes(const Dims &dm);
+int chain_tc_prefill_ctas(const Dims &dm);   // CTAs (SMs) a tensor-core prefill chain occupies
 }
 
 struct lola_state {
@@ -35,7 +37,10 @@ struct lola_state {
     // segments on the caller's stream and of odd segments on a second library stream, so
     // that a segment's last partial wave of CTAs overlaps the next segment's first
     static constexpr int kMaxSeg = lola::kMaxSegments;
-    int seg_len;                     // intervals per segment (0: the whole call)
+    bool overlap;                    // the streams and events of segmented prefill exist
+    int sms;                         // SMs of the state's device
+    int sched_mode;                  // lola_schedule of the following prefill calls
+    int seg_user;                    // intervals per segment asked for (0: the mode's default)
     cudaStream_t chain_stream;
     cudaStream_t attn_stream;
     cudaEvent_t ev_fork;
@@ -412,6 +417,33 @@ bool make_host_streams(lola_state *st)
     return true;
 }
 
+// The schedule of a segmented prefill call: one chain launch for the call or one per
+// segment, and the intervals per segment (at most kMaxSegments segments per call).
+// Automatic choice: one chain launch saves the chain the gap at every launch boundary
+// (about 85 us on a B200), but holds its SMs for the whole call. Where the chain takes
+// more than a third of the SMs, the attention beside it falls behind, and one launch per
+// segment does better: between two chain launches the chain's SMs take waiting attention
+// work, and the attention stays close behind the chain. Measured on a B200 (per call):
+// 32 streams on 64 SMs, 256 intervals: 11.96 ms per segment vs 12.40 ms one launch;
+// 8 streams on 40 SMs: 512 intervals 22.63 vs 23.19 ms, 64 intervals 1.17 vs 1.26 ms
+// in favour of one launch. Segments of 16 intervals measured best in both forms; a
+// shorter call (m intervals) keeps at least four segments of at least 8 intervals
+// (32-interval calls: 18.75 ms per 16384 tokens in segments of 8, 19.06 in segments of 16).
+void prefill_schedule(const lola_state *st, int m, bool *one_chain, int *len)
+{
+    const Dims &dm = st->dm;
+    int mode = st->sched_mode;
+    if (mode == LOLA_SCHEDULE_AUTO)
+        mode = 3 * lola::chain_tc_prefill_ctas(dm) > st->sms ? LOLA_SCHEDULE_SEGMENTS : LOLA_SCHEDULE_ONE_CHAIN;
+    int l = st->seg_user;
+    if (l <= 0) {
+        l = mode == LOLA_SCHEDULE_ONE_CHAIN ? std::max(16, dm.mmax / 32) : std::max(16, dm.mmax / 16);
+        l = std::min(l, std::max(8, (m + 3) / 4));
+    }
+    *len = std::max(l, (dm.mmax + lola::kMaxSegments - 1) / lola::kMaxSegments);
+    *one_chain = mode == LOLA_SCHEDULE_ONE_CHAIN;
+}
+
 }  // namespace
 
 extern "C" {
@@ -473,17 +505,22 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     layout(dm, (char *)workspace, &st->S, &st->P);
     reset_host(st);
     st->timing = false;
-    st->seg_len = 0;
+    st->overlap = false;
+    st->sms = 0;
+    {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess ||
+            cudaDeviceGetAttribute(&st->sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            cudaGetLastError();
+    }
+    st->sched_mode = LOLA_SCHEDULE_AUTO;
+    st->seg_user = 0;
     st->chain_stream = nullptr;
     st->attn_stream = nullptr;
     st->seg_wait = wait_value_fn() != nullptr;
     for (int i = 0; i < lola::kMaxSegments; ++i) st->seg_expect[i] = 0;
     st->h2d_stream = st->d2h_stream = nullptr;
     if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
-        // segments of at least 8 intervals, at most kMaxSeg of them per call
-        int len = dm.mmax / 32;
-        if (len < 8) len = 8;
-        while ((dm.mmax + len - 1) / len > lola_state::kMaxSeg) ++len;
         int lo = 0, hi = 0;
         bool okc = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
                    cudaStreamCreateWithPriority(&st->chain_stream, cudaStreamNonBlocking, hi) == cudaSuccess &&
@@ -499,7 +536,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
             delete st;
             return LOLA_ERR_CUDA;
         }
-        st->seg_len = len;
+        st->overlap = true;
     }
     const unsigned long long rk = (unsigned long long)dm.ns * (dm.lam + dm.R + dm.Nmax);
     const unsigned long long rv = (unsigned long long)dm.ns * (dm.lam + dm.R);
@@ -587,7 +624,9 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     // stream, a few SMs) runs on the library's high-priority stream; the attention
     // of the segment follows on the caller's stream once that chain is done, so it
     // overlaps the chain of the next segments on the other SMs.
-    const int seg = st->seg_len > 0 ? st->seg_len : m;
+    bool one_chain = false;
+    int seg = m;
+    if (st->overlap) prefill_schedule(st, m, &one_chain, &seg);
     const int nseg = (m + seg - 1) / seg;
     const bool fork = nseg > 1 && st->chain_stream != nullptr;
     lola::AttnMaps amaps;
@@ -614,7 +653,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     // (the launch boundaries between chain segments cost the chain about 85 us each, its
     // SMs briefly free for waiting attention CTAs). Otherwise one chain launch per segment,
     // the attention gated by an event.
-    const bool one = fork && dm.tc_chain && st->seg_wait && nseg <= lola::kMaxSegments;
+    const bool one = fork && one_chain && dm.tc_chain && st->seg_wait && nseg <= lola::kMaxSegments;
     for (int sg = 0; sg < nseg; ++sg) {
         const int ci0 = sg * seg;
         const int ms = m - ci0 < seg ? m - ci0 : seg;
@@ -848,6 +887,16 @@ lola_status lola_sync(lola_state *st, void *cuda_stream)
         cudaMemset(st->S.dec_cnt, 0, (size_t)st->dm.ns * sizeof(int));
         return (err[0] & lola::ERR_TIMEOUT) ? LOLA_ERR_TIMEOUT : LOLA_ERR_DEVICE;
     }
+    return LOLA_OK;
+}
+
+lola_status lola_set_prefill_schedule(lola_state *st, int32_t mode, int32_t intervals_per_segment)
+{
+    if (!st || intervals_per_segment < 0) return LOLA_ERR_INVALID_ARG;
+    if (mode != LOLA_SCHEDULE_AUTO && mode != LOLA_SCHEDULE_ONE_CHAIN && mode != LOLA_SCHEDULE_SEGMENTS)
+        return LOLA_ERR_INVALID_ARG;
+    st->sched_mode = mode;
+    st->seg_user = intervals_per_segment;
     return LOLA_OK;
 }
 

@@ -890,6 +890,22 @@ size_t snap_image_bytes(const Dims &dm)
     return (size_t)g.NB * g.FP * 2;
 }
 
+// CTAs per stream of a prefill chain. With few streams a cluster of up to 5 CTAs per
+// stream shares the scoring, one SRE tile each or more (at most LOLA_CHAIN_CTAS CTAs in all,
+// so that the attention keeps the other SMs; wider clusters measured slower: the key
+// exchange grows with the width).
+static int prefill_cluster(const Dims &dm)
+{
+    const int tiles = (dm.lam + dm.C + 127) / 128;   // SRE tiles of a full interval
+    int nc = LOLA_CHAIN_CTAS / dm.ns;
+    if (nc > tiles) nc = tiles;
+    if (nc > 5) nc = 5;
+    if (nc < 1) nc = 1;
+    return nc;
+}
+
+int chain_tc_prefill_ctas(const Dims &dm) { return dm.ns * prefill_cluster(dm); }
+
 void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P, const ChainArgs &a,
                      const CUtensorMap &phimap, const CUtensorMap &boxmap, cudaStream_t stream)
 {
@@ -900,17 +916,7 @@ void launch_chain_tc(const Dims &dm, const DevState &S, const PrefillScratch *P,
     cudaFuncSetAttribute(chain_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     PrefillScratch Pv{};
     if (P) Pv = *P;
-    // prefill with few streams: a cluster of up to 5 CTAs per stream shares the scoring,
-    // one SRE tile each or more (at most LOLA_CHAIN_CTAS CTAs, so that the attention keeps the
-    // other SMs; wider clusters measured slower: the key exchange grows with the width)
-    int nc = 1;
-    if (a.mode == 0) {
-        const int tiles = (dm.lam + dm.C + 127) / 128;   // SRE tiles of a full interval
-        nc = LOLA_CHAIN_CTAS / dm.ns;
-        if (nc > tiles) nc = tiles;
-        if (nc > 5) nc = 5;
-        if (nc < 1) nc = 1;
-    }
+    const int nc = a.mode == 0 ? prefill_cluster(dm) : 1;
     if (nc == 1) {
         chain_tc_kernel<<<dm.ns, kThreads, smem, stream>>>(dm, S, Pv, a, src, 1, phimap, boxmap);
         return;

@@ -74,6 +74,7 @@ def load_library() -> ctypes.CDLL:
         "lola_free_state": (I32, [P]),
         "lola_status_string": (ctypes.c_char_p, [I32]),
         "lola_set_timing": (I32, [P, ctypes.c_int]),
+        "lola_set_prefill_schedule": (I32, [P, I32, I32]),
         "lola_timing_read": (I32, [P, P, P]),
         "lola_launch_count": (I64, []),
         "lola_selftest_umma": (I32, [ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P, P]),
@@ -211,6 +212,15 @@ def lola_set_timing(h: int, enable: bool):
     _check(load_library().lola_set_timing(h, 1 if enable else 0), "lola_set_timing")
 
 
+# lola_schedule: how a prefill call overlaps its chain and its attention
+SCHEDULES = {"auto": 0, "one-chain": 1, "segments": 2}
+
+
+def lola_set_prefill_schedule(h: int, mode: int, intervals_per_segment: int = 0):
+    _check(load_library().lola_set_prefill_schedule(h, mode, intervals_per_segment),
+           "lola_set_prefill_schedule")
+
+
 PHASES = ("phi", "chain", "attn", "finalize", "append", "update", "decode", "reset")
 
 
@@ -263,6 +273,11 @@ class LolaState:
 
     def reset(self):
         lola_reset_state(self.handle, self._stream())
+
+    def set_prefill_schedule(self, mode: str = "auto", intervals_per_segment: int = 0):
+        """How the following prefill calls overlap the chain and the attention:
+        "auto", "one-chain" or "segments" (see SCHEDULES)."""
+        lola_set_prefill_schedule(self.handle, SCHEDULES[mode], intervals_per_segment)
 
     def prefill(self, q, k, v, out=None):
         q, k, v = self._dev(q), self._dev(k), self._dev(v)

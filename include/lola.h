@@ -144,6 +144,41 @@ lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, cons
                               void *cuda_stream);
 lola_status lola_prefill_host_staging_bytes(const lola_config *cfg, int64_t piece_tokens, size_t *bytes);
 
+/* How a prefill call overlaps its two parts (no counterpart in the paper, which
+ * describes no kernel; it changes when work runs, not what is computed). The
+ * call's update intervals run as a sequential per-stream chain (score, select,
+ * fold: the Self-Recall Error and sparse-caching steps of the "SRE" and
+ * "Inferentiestrategie" sections) on a few SMs per stream, and a parallel
+ * attention over all intervals on the other SMs, in segments of consecutive
+ * intervals: the attention of a segment starts once every stream's chain has
+ * finished that segment.
+ *   mode LOLA_SCHEDULE_AUTO      the default: LOLA_SCHEDULE_SEGMENTS where the chain
+ *        occupies more than a third of the device's SMs (many streams), else
+ *        LOLA_SCHEDULE_ONE_CHAIN
+ *   mode LOLA_SCHEDULE_ONE_CHAIN one chain launch per call; it counts finished
+ *        segments in device memory and each attention segment waits for its count
+ *        (a stream memory operation, no kernel waits on another). Falls back to
+ *        LOLA_SCHEDULE_SEGMENTS where the driver has no stream memory operations.
+ *   mode LOLA_SCHEDULE_SEGMENTS  one chain launch per segment, each attention
+ *        segment gated by an event; between two chain launches the chain's SMs
+ *        also take waiting attention work.
+ * intervals_per_segment: 0 for the library's length, with m = max_prefill_tokens /
+ * chunk intervals per call at most: max(16, m / 32) for one chain launch and
+ * max(16, m / 16) for launches per segment, lowered for a call of n intervals to
+ * max(8, ceil(n / 4)) where that is shorter; else >= 1. A length that would give
+ * more than 64 segments per call is raised to ceil(m / 64). The setting applies
+ * to the following calls of the state. Both modes and every length give the same outputs bit for bit.
+ * It takes effect only for bfloat16 configs on the tensor-core chain and
+ * attention with more than one interval per call; elsewhere it is stored and
+ * ignored. LOLA_ERR_INVALID_ARG for a null state, an unknown mode or a negative
+ * length. Host call; nothing is enqueued. */
+typedef enum {
+    LOLA_SCHEDULE_AUTO = 0,
+    LOLA_SCHEDULE_ONE_CHAIN = 1,
+    LOLA_SCHEDULE_SEGMENTS = 2
+} lola_schedule;
+lola_status lola_set_prefill_schedule(lola_state *st, int32_t mode, int32_t intervals_per_segment);
+
 /* One token per sequence: q [B][n_q_heads][head_dim], k, v [B][n_kv_heads][head_dim],
  * out [B][n_q_heads][head_dim]. When the position is at an interval boundary,
  * an update interval of length decode_interval opens here (score, select, fold);

@@ -71,6 +71,7 @@ def test_null_arguments_rejected_without_device(lib):
     assert lib.lola_prefill_chunk(None, None, None, None, 64, None, None) == 1
     assert lib.lola_decode_step(None, None, None, None, None, None) == 1
     assert lib.lola_sync(None, None) == 1
+    assert lib.lola_set_prefill_schedule(None, 0, 0) == 1
     assert lib.lola_state_bytes(None, None) == 1
     assert lib.lola_position(None) == -1
     assert lib.lola_free_state(None) == 0
