@@ -353,6 +353,10 @@ def run_engine(args, ws, rank, local):
     cfg = L.config_from_workload(w, max_prefill_tokens=T)
     S = L.LolaState(cfg, torch.from_numpy(W), dev)
     S.set_prefill_schedule(args.prefill_schedule, args.segment_intervals)
+    mode, seg_len, nseg = L.lola_prefill_plan(cfg, T, args.prefill_schedule, args.segment_intervals,
+                                              torch.cuda.get_device_properties(dev).multi_processor_count)
+    sched = (f"{args.prefill_schedule}: {mode}, {nseg} segments of {seg_len} intervals per call"
+             if nseg > 1 else f"{args.prefill_schedule}: one segment")
     dt = S.dtype
     qd = torch.from_numpy(q).to(dev, dt)
     kd = torch.from_numpy(k).to(dev, dt)
@@ -459,8 +463,7 @@ def run_engine(args, ws, rank, local):
                        "seq_len": T, "n_q_heads": w_job.n_q_heads, "n_kv_heads": w_job.n_kv_heads,
                        "head_dim": w.head_dim, "feat_dim": w.feat_dim, "window": w.window,
                        "lambda": w.lambda_, "chunk": w.chunk,
-                       "prefill_schedule": args.prefill_schedule
-                       + (f", {args.segment_intervals} intervals per segment" if args.segment_intervals else ""),
+                       "prefill_schedule": sched,
                        "parallelism": (f"streams sharded over {ws} ranks by {shard.by} (no collective on the "
                                        f"data path)" if shard is not None
                                        else f"replicas x{ws} (independent streams, no collective)"),

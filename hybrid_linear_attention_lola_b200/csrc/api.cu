@@ -417,8 +417,13 @@ bool make_host_streams(lola_state *st)
     return true;
 }
 
-// The schedule of a segmented prefill call: one chain launch for the call or one per
-// segment, and the intervals per segment (at most kMaxSegments segments per call).
+// Configs whose prefill runs in overlapped segments: the tensor-core chain and attention,
+// more than one interval per call.
+bool segmented_prefill(const Dims &dm) { return dm.tc_chain && dm.tc_attn && dm.mmax > 1; }
+
+// The schedule of a segmented prefill call of m intervals (mode and seg_user as given to
+// lola_set_prefill_schedule, sms the device's SMs): one chain launch for the call or one
+// per segment, and the intervals per segment (at most kMaxSegments segments per call).
 // Automatic choice: one chain launch saves the chain the gap at every launch boundary
 // (about 85 us on a B200), but holds its SMs for the whole call. Where the chain takes
 // more than a third of the SMs, the attention beside it falls behind, and one launch per
@@ -429,13 +434,11 @@ bool make_host_streams(lola_state *st)
 // in favour of one launch. Segments of 16 intervals measured best in both forms; a
 // shorter call (m intervals) keeps at least four segments of at least 8 intervals
 // (32-interval calls: 18.75 ms per 16384 tokens in segments of 8, 19.06 in segments of 16).
-void prefill_schedule(const lola_state *st, int m, bool *one_chain, int *len)
+void plan_schedule(const Dims &dm, int mode, int seg_user, int sms, int m, bool *one_chain, int *len)
 {
-    const Dims &dm = st->dm;
-    int mode = st->sched_mode;
     if (mode == LOLA_SCHEDULE_AUTO)
-        mode = 3 * lola::chain_tc_prefill_ctas(dm) > st->sms ? LOLA_SCHEDULE_SEGMENTS : LOLA_SCHEDULE_ONE_CHAIN;
-    int l = st->seg_user;
+        mode = 3 * lola::chain_tc_prefill_ctas(dm) > sms ? LOLA_SCHEDULE_SEGMENTS : LOLA_SCHEDULE_ONE_CHAIN;
+    int l = seg_user;
     if (l <= 0) {
         l = mode == LOLA_SCHEDULE_ONE_CHAIN ? std::max(16, dm.mmax / 32) : std::max(16, dm.mmax / 16);
         l = std::min(l, std::max(8, (m + 3) / 4));
@@ -520,7 +523,7 @@ lola_status lola_init_state(const lola_config *cfg, const void *W, void *workspa
     st->seg_wait = wait_value_fn() != nullptr;
     for (int i = 0; i < lola::kMaxSegments; ++i) st->seg_expect[i] = 0;
     st->h2d_stream = st->d2h_stream = nullptr;
-    if (dm.tc_chain && dm.tc_attn && dm.mmax > 1) {
+    if (segmented_prefill(dm)) {
         int lo = 0, hi = 0;
         bool okc = cudaDeviceGetStreamPriorityRange(&lo, &hi) == cudaSuccess &&
                    cudaStreamCreateWithPriority(&st->chain_stream, cudaStreamNonBlocking, hi) == cudaSuccess &&
@@ -620,13 +623,13 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
     }
     if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
 
-    // The call's intervals run in segments. The chain of a segment (sequential per
-    // stream, a few SMs) runs on the library's high-priority stream; the attention
-    // of the segment follows on the caller's stream once that chain is done, so it
-    // overlaps the chain of the next segments on the other SMs.
+    // The call's intervals run in segments. The chain (sequential per stream, a few SMs)
+    // runs on the library's high-priority stream; the attention of a segment follows once
+    // the chain has finished that segment, on the caller's stream or the second attention
+    // stream, so it overlaps the chain of the next segments on the other SMs.
     bool one_chain = false;
     int seg = m;
-    if (st->overlap) prefill_schedule(st, m, &one_chain, &seg);
+    if (st->overlap) plan_schedule(dm, st->sched_mode, st->seg_user, st->sms, m, &one_chain, &seg);
     const int nseg = (m + seg - 1) / seg;
     const bool fork = nseg > 1 && st->chain_stream != nullptr;
     lola::AttnMaps amaps;
@@ -648,11 +651,10 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         cudaStreamWaitEvent(cs, st->ev_fork, 0);
         if (two) cudaStreamWaitEvent(st->attn_stream, st->ev_fork, 0);
     }
-    // With stream memory operations the chain is one launch for the whole call and counts
-    // finished segments in device memory; the attention of segment s waits for its count
-    // (the launch boundaries between chain segments cost the chain about 85 us each, its
-    // SMs briefly free for waiting attention CTAs). Otherwise one chain launch per segment,
-    // the attention gated by an event.
+    // One chain launch for the whole call (where the schedule asks for it and the driver has
+    // stream memory operations): the chain counts finished segments in device memory and the
+    // attention of segment s waits for its count. Otherwise one chain launch per segment,
+    // the attention gated by an event (plan_schedule weighs the two).
     const bool one = fork && one_chain && dm.tc_chain && st->seg_wait && nseg <= lola::kMaxSegments;
     for (int sg = 0; sg < nseg; ++sg) {
         const int ci0 = sg * seg;
@@ -897,6 +899,28 @@ lola_status lola_set_prefill_schedule(lola_state *st, int32_t mode, int32_t inte
         return LOLA_ERR_INVALID_ARG;
     st->sched_mode = mode;
     st->seg_user = intervals_per_segment;
+    return LOLA_OK;
+}
+
+lola_status lola_prefill_plan(const lola_config *cfg, int32_t mode, int32_t intervals_per_segment, int32_t sms,
+                              int64_t n_tokens, int32_t *mode_out, int32_t *len_out, int32_t *segments_out)
+{
+    if (!mode_out || !len_out || !segments_out || sms < 1 || intervals_per_segment < 0) return LOLA_ERR_INVALID_ARG;
+    if (mode != LOLA_SCHEDULE_AUTO && mode != LOLA_SCHEDULE_ONE_CHAIN && mode != LOLA_SCHEDULE_SEGMENTS)
+        return LOLA_ERR_INVALID_ARG;
+    Dims dm;
+    const lola_status r = derive_dims(cfg, &dm);
+    if (r != LOLA_OK) return r;
+    if (n_tokens <= 0 || n_tokens % dm.C != 0) return LOLA_ERR_SHAPE;
+    if (n_tokens > dm.Nmax) return LOLA_ERR_WORKSPACE;
+    const int m = (int)(n_tokens / dm.C);
+    bool one = false;
+    int len = m;
+    if (segmented_prefill(dm)) plan_schedule(dm, mode, intervals_per_segment, sms, m, &one, &len);
+    const int nseg = (m + len - 1) / len;
+    *mode_out = one && nseg > 1 ? LOLA_SCHEDULE_ONE_CHAIN : LOLA_SCHEDULE_SEGMENTS;
+    *len_out = nseg > 1 ? len : m;
+    *segments_out = nseg;
     return LOLA_OK;
 }
 

@@ -75,6 +75,8 @@ def load_library() -> ctypes.CDLL:
         "lola_status_string": (ctypes.c_char_p, [I32]),
         "lola_set_timing": (I32, [P, ctypes.c_int]),
         "lola_set_prefill_schedule": (I32, [P, I32, I32]),
+        "lola_prefill_plan": (I32, [C, I32, I32, I32, I64, ctypes.POINTER(I32), ctypes.POINTER(I32),
+                                    ctypes.POINTER(I32)]),
         "lola_timing_read": (I32, [P, P, P]),
         "lola_launch_count": (I64, []),
         "lola_selftest_umma": (I32, [ctypes.c_int, P, P, P, ctypes.c_int, ctypes.c_int, P, P]),
@@ -219,6 +221,17 @@ SCHEDULES = {"auto": 0, "one-chain": 1, "segments": 2}
 def lola_set_prefill_schedule(h: int, mode: int, intervals_per_segment: int = 0):
     _check(load_library().lola_set_prefill_schedule(h, mode, intervals_per_segment),
            "lola_set_prefill_schedule")
+
+
+def lola_prefill_plan(cfg: lola_config, n_tokens: int, mode: str = "auto", intervals_per_segment: int = 0,
+                      sms: int = 148) -> tuple:
+    """(schedule name, intervals per segment, segments) of a prefill call of n_tokens."""
+    mo, ln, ns = ctypes.c_int32(0), ctypes.c_int32(0), ctypes.c_int32(0)
+    _check(load_library().lola_prefill_plan(ctypes.byref(cfg), SCHEDULES[mode], intervals_per_segment, sms,
+                                            n_tokens, ctypes.byref(mo), ctypes.byref(ln), ctypes.byref(ns)),
+           "lola_prefill_plan")
+    name = {v: k for k, v in SCHEDULES.items()}[mo.value]
+    return name, ln.value, ns.value
 
 
 PHASES = ("phi", "chain", "attn", "finalize", "append", "update", "decode", "reset")

@@ -179,6 +179,20 @@ typedef enum {
 } lola_schedule;
 lola_status lola_set_prefill_schedule(lola_state *st, int32_t mode, int32_t intervals_per_segment);
 
+/* The schedule a prefill call of n_tokens tokens gets on a state with this config
+ * whose schedule was set to (mode, intervals_per_segment), on a device of `sms`
+ * SMs (148 on a B200): *mode_out LOLA_SCHEDULE_ONE_CHAIN or LOLA_SCHEDULE_SEGMENTS,
+ * *len_out the intervals per segment and *segments_out the segments of the call. A
+ * call of one segment (every call of a config that does not run the tensor-core
+ * chain and attention, or of one interval) runs its chain and then its attention
+ * on the caller's stream and reports LOLA_SCHEDULE_SEGMENTS with len = its
+ * intervals. At run time LOLA_SCHEDULE_ONE_CHAIN becomes LOLA_SCHEDULE_SEGMENTS
+ * where the driver has no stream memory operations. Pure host computation. Errors:
+ * LOLA_ERR_INVALID_ARG (null output, sms < 1, bad mode or length, bad config),
+ * LOLA_ERR_SHAPE / LOLA_ERR_WORKSPACE for n_tokens as in lola_prefill_chunk. */
+lola_status lola_prefill_plan(const lola_config *cfg, int32_t mode, int32_t intervals_per_segment, int32_t sms,
+                              int64_t n_tokens, int32_t *mode_out, int32_t *len_out, int32_t *segments_out);
+
 /* One token per sequence: q [B][n_q_heads][head_dim], k, v [B][n_kv_heads][head_dim],
  * out [B][n_q_heads][head_dim]. When the position is at an interval boundary,
  * an update interval of length decode_interval opens here (score, select, fold);

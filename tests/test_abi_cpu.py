@@ -123,3 +123,36 @@ def test_host_prefill_staging_bytes(lib):
     assert lib.lola_prefill_host_staging_bytes(ctypes.byref(cfg), 100, ctypes.byref(n)) == 2   # not a multiple of the chunk
     assert lib.lola_prefill_host_staging_bytes(ctypes.byref(cfg), 2 * w.seq_len, ctypes.byref(n)) == 5  # past max_prefill_tokens
     assert lib.lola_prefill_host(None, None, None, None, 64, None, None, 0, 64, None) == 1
+
+
+def test_prefill_plan(lib):
+    """The schedule each call gets (pure host): per-segment launches where the chain holds
+    more than a third of a 148-SM device, one chain launch elsewhere; 16-interval segments,
+    at least four of at least 8 intervals in a short call, at most 64 per call."""
+    w8 = wl.WORKLOADS["prefill-8b"]         # 32 streams, chain on 64 SMs
+    c8 = L.config_from_workload(w8, max_prefill_tokens=w8.seq_len)
+    assert L.lola_prefill_plan(c8, w8.seq_len) == ("segments", 16, 16)
+    assert L.lola_prefill_plan(c8, 2048) == ("segments", 8, 4)            # a 32-interval piece
+    assert L.lola_prefill_plan(c8, 64) == ("segments", 1, 1)              # one interval
+    assert L.lola_prefill_plan(c8, w8.seq_len, sms=256) == ("one-chain", 16, 16)
+    assert L.lola_prefill_plan(c8, w8.seq_len, "one-chain", 1) == ("one-chain", 4, 64)   # at most 64
+    assert L.lola_prefill_plan(c8, w8.seq_len, "segments", 3) == ("segments", 4, 64)
+    assert L.lola_prefill_plan(c8, w8.seq_len, "segments", 100) == ("segments", 100, 3)
+    wl_ = wl.WORKLOADS["long-context"]      # 8 streams, chain on 40 SMs, 512 intervals
+    cl = L.config_from_workload(wl_, max_prefill_tokens=wl_.seq_len)
+    assert L.lola_prefill_plan(cl, wl_.seq_len) == ("one-chain", 16, 32)
+    assert L.lola_prefill_plan(cl, wl_.seq_len, "segments") == ("segments", 32, 16)
+    w1 = wl.WORKLOADS["prefill-1b"]         # 8 streams, 64 intervals
+    c1 = L.config_from_workload(w1, max_prefill_tokens=w1.seq_len)
+    assert L.lola_prefill_plan(c1, w1.seq_len) == ("one-chain", 16, 4)
+    # fp32 runs the SIMT chain and attention: one segment whatever the setting
+    cf = L.config_from_workload(w1, max_prefill_tokens=w1.seq_len, dtype="f32")
+    assert L.lola_prefill_plan(cf, w1.seq_len, "one-chain", 8) == ("segments", 64, 1)
+    o = [ctypes.c_int32(0) for _ in range(3)]
+    ref = [ctypes.byref(x) for x in o]
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 3, 0, 148, 64, *ref) == 1       # unknown mode
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 0, -1, 148, 64, *ref) == 1      # negative length
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 0, 0, 0, 64, *ref) == 1         # no SMs
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 0, 0, 148, 100, *ref) == 2      # not a multiple of chunk
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 0, 0, 148, 2 * w8.seq_len, *ref) == 5
+    assert lib.lola_prefill_plan(ctypes.byref(c8), 0, 0, 148, 64, None, None, None) == 1
