@@ -72,10 +72,11 @@ def source_sha(rels) -> str:
     return h.hexdigest()[:16]
 
 
-def captured_traffic(kernel: str, workload: str):
+def captured_traffic(kernel: str, workload: str, units=None):
     """DRAM bytes (read + write) per launch of `kernel` on `workload` from the
     committed ncu summary, or (None, reason) when there is none for the current
-    source of the kernel."""
+    source of the kernel. An entry that stores bytes per unit of work (one interval
+    of one stream) is scaled to a launch of `units` such units."""
     try:
         with open(TRAFFIC_FILE) as f:
             entries = json.load(f)
@@ -86,7 +87,13 @@ def captured_traffic(kernel: str, workload: str):
             src = KERNEL_SOURCES.get(kernel)
             if src is None or e.get("source_sha") != source_sha(src):
                 return None, "kernel changed since its ncu capture"
-            return e.get("dram_bytes_per_launch"), "ncu capture (profiles/dram_traffic.json)"
+            if units is not None and e.get("dram_bytes_per_unit") is not None:
+                return (round(e["dram_bytes_per_unit"] * units),
+                        f"ncu capture (profiles/dram_traffic.json) of {e['captured_launch']}, "
+                        f"scaled to this launch by its {units} units ({e['unit']})")
+            if e.get("dram_bytes_per_launch") is None:
+                return None, "no ncu capture of the kernel's current launch form"
+            return e["dram_bytes_per_launch"], "ncu capture (profiles/dram_traffic.json)"
     return None, "no ncu capture for this kernel and workload"
 
 
@@ -274,7 +281,7 @@ def cpu_baseline(w, budget_s=15.0, threads=None, single_thread=True):
 
 # ---------------------------------------------------------------- roofline
 
-def prefill_roofline(w, T, ms_step, phase_ms, steps, peaks, peak_src):
+def prefill_roofline(w, T, ms_step, phase_ms, steps, peaks, peak_src, launch_intervals=None):
     """Headline: the whole prefill step's algorithmic FLOPs over its time, against the
     measured bf16 tensor peak (burst; the sustained figure beside it). Per phase: the
     attention (tensor-bound contractions) and the chain (sequential per stream: its
@@ -296,13 +303,16 @@ def prefill_roofline(w, T, ms_step, phase_ms, steps, peaks, peak_src):
                       "frac_of_sustained": round(a / sust, 5), "bound": bound}
     # traffic of the dominant kernel (the phase with the most device time)
     dom = max((p for p in ("attn", "chain") if p in per_call), key=per_call.get, default="attn")
-    traffic, tsrc = captured_traffic(dom, w.name)
+    streams = w.batch * w.n_kv_heads
+    units = launch_intervals * streams if launch_intervals else None
+    traffic, tsrc = captured_traffic(dom, w.name, units)
     if w != wl.WORKLOADS.get(w.name):
         traffic, tsrc = None, "workload overridden on the command line (no capture for it)"
     return {"bound": "tensor", "kernel": f"whole prefill step (dominant kernel: {dom})",
             "achieved": round(ach, 3), "peak": burst, "unit": "TFLOP/s", "frac": round(ach / burst, 5),
             "frac_of_sustained": round(ach / sust, 5), "peak_sustained": sust,
             "traffic": traffic, "traffic_kernel": dom, "traffic_source": tsrc,
+            "traffic_launch": (f"{launch_intervals} intervals x {streams} streams" if launch_intervals else None),
             "peak_source": f"{peak_src} bf16 dense (burst; sustained beside it)",
             "algorithmic_tflop_per_step": round(total / 1e12, 5), "phases": phases,
             "phase_ms": {ph: round(v, 4) for ph, v in per_call.items()}}
@@ -408,7 +418,8 @@ def run_engine(args, ws, rank, local):
     job_tokens = w_job.batch * T if shard is not None else w.batch * T * ws
     value = job_tokens / (ms_step / 1e3)
 
-    roofline = prefill_roofline(w, T, ms_step, phase_ms, args.steps, peaks, peak_src)
+    roofline = prefill_roofline(w, T, ms_step, phase_ms, args.steps, peaks, peak_src,
+                                launch_intervals=seg_len if nseg > 1 else T // w.chunk)
 
     # end to end through the C ABI from pinned host memory: lola_prefill_host copies every
     # input to the device and every output back inside the timed region, overlapping the

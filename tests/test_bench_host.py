@@ -34,6 +34,34 @@ def test_decode_bytes_per_step():
     assert abs(per_stream / 193.9e3 - 1) < 0.02
 
 
+def test_attention_traffic_scales_with_the_launch():
+    # the committed capture is per unit (one interval of one stream); a launch of n units
+    # reads n times that, and the 8-interval launch at batch 4 is the stored per-launch figure
+    e = next(x for x in __import__("json").load(open(bench.TRAFFIC_FILE)) if x["kernel"] == "attn")
+    t8, src = bench.captured_traffic("attn", "prefill-8b", 8 * 32)
+    assert abs(t8 / e["dram_bytes_per_launch"] - 1) < 1e-6 and "scaled" in src
+    t16, _ = bench.captured_traffic("attn", "prefill-8b", 16 * 32)
+    assert abs(t16 / t8 - 2) < 1e-6
+    assert bench.captured_traffic("attn", "prefill-8b")[0] == e["dram_bytes_per_launch"]
+    assert bench.captured_traffic("chain", "prefill-8b", 512)[0] is None
+
+
+def test_traffic_is_null_once_the_kernel_changes(monkeypatch):
+    monkeypatch.setattr(bench, "source_sha", lambda rels: "0" * 16)
+    t, why = bench.captured_traffic("attn", "prefill-8b", 512)
+    assert t is None and "changed" in why
+
+
+def test_prefill_roofline_reports_the_launch_it_scales_to():
+    w = wl.WORKLOADS["prefill-8b"]
+    phases = {"attn": [180.0, 160], "chain": [106.0, 160], "phi": [2.7, 10]}   # 10 steps
+    peaks = {"bf16_tflops": 1717.8, "bf16_tflops_sustained": 1424.0}
+    r = bench.prefill_roofline(w, w.seq_len, 11.97, phases, 10, peaks, "measured", launch_intervals=16)
+    assert r["traffic_kernel"] == "attn" and r["traffic_launch"] == "16 intervals x 32 streams"
+    assert r["traffic"] == bench.captured_traffic("attn", "prefill-8b", 16 * 32)[0]
+    assert abs(r["frac"] - r["achieved"] / 1717.8) < 1e-4
+
+
 def _free_port():
     s = socket.socket()
     s.bind(("127.0.0.1", 0))
