@@ -700,6 +700,11 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
                 counted(1);
             }
             if (check_launch() != LOLA_OK) return LOLA_ERR_CUDA;
+            if (one) {
+                // the launched chain counts every segment of the call (also when it gives up),
+                // so every target moves now, whatever happens to the attention launches below
+                for (int s2 = 0; s2 < nseg; ++s2) st->seg_expect[s2] += (uint32_t)dm.ns;
+            }
             if (fork) cudaEventRecord(st->ev_seg[sg], cs);
         }
         // the attention of this segment: on the caller's stream, or (odd segments) on the
@@ -707,8 +712,7 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
         cudaStream_t as = (two && (sg & 1)) ? st->attn_stream : stream;
         if (one) {
             // every stream's chain has counted this segment (the count runs across calls)
-            const uint32_t target = st->seg_expect[sg] + (uint32_t)dm.ns;
-            st->seg_expect[sg] = target;
+            const uint32_t target = st->seg_expect[sg];
             if (wait_value_fn()((CUstream)as, (CUdeviceptr)(st->S.seg_done + sg), target, CU_STREAM_WAIT_VALUE_GEQ) !=
                 CUDA_SUCCESS)
                 cudaStreamWaitEvent(as, st->ev_seg[0], 0);   // the whole chain, then
