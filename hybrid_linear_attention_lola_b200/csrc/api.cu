@@ -790,6 +790,14 @@ lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, cons
     cudaEventRecord(st->ev_host, stream);
     cudaStreamWaitEvent(st->h2d_stream, st->ev_host, 0);
     cudaStreamWaitEvent(st->d2h_stream, st->ev_host, 0);
+    // the caller's stream passes this call once both copy streams are done (also after an
+    // error, so that no copy into the caller's buffers outlives what the stream says)
+    auto join = [&]() {
+        cudaEventRecord(st->ev_host, st->h2d_stream);
+        cudaStreamWaitEvent(stream, st->ev_host, 0);
+        cudaEventRecord(st->ev_host, st->d2h_stream);
+        cudaStreamWaitEvent(stream, st->ev_host, 0);
+    };
     int i = 0;
     for (int64_t t0 = 0; t0 < n_tokens; t0 += piece_tokens, ++i) {
         const int64_t len = n_tokens - t0 < piece_tokens ? n_tokens - t0 : piece_tokens;
@@ -810,7 +818,10 @@ lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, cons
         cudaStreamWaitEvent(stream, st->ev_h2d[slot], 0);
         if (i >= 2) cudaStreamWaitEvent(stream, st->ev_d2h[slot], 0);
         const lola_status r = lola_prefill_chunk(st, qd, kd, vd, len, od, stream);
-        if (r != LOLA_OK) return r;
+        if (r != LOLA_OK) {
+            join();
+            return r;
+        }
         cudaEventRecord(st->ev_comp[slot], stream);
         // its outputs back to the host rows
         cudaStreamWaitEvent(st->d2h_stream, st->ev_comp[slot], 0);
@@ -818,9 +829,7 @@ lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, cons
                           (size_t)len * qrow, (size_t)dm.B, cudaMemcpyDeviceToHost, st->d2h_stream);
         cudaEventRecord(st->ev_d2h[slot], st->d2h_stream);
     }
-    // the caller's stream passes this call once the last output copy is done
-    cudaEventRecord(st->ev_host, st->d2h_stream);
-    cudaStreamWaitEvent(stream, st->ev_host, 0);
+    join();
     return check_launch();
 }
 
