@@ -138,9 +138,10 @@ lola_status lola_prefill_chunk(lola_state *st, const void *q, const void *k, con
  * allocates nothing. The call returns once the work is queued; when cuda_stream
  * has passed it, every output row is in `out` on the host. Errors as for
  * lola_prefill_chunk, and LOLA_ERR_WORKSPACE for a staging buffer that is too
- * small. An error from a piece after the first ends the call with the pieces
- * before it done (outputs copied back, state advanced past them); the copies
- * already queued finish before cuda_stream passes the call. */
+ * small. An error from a piece after the first ends the call: the pieces before
+ * it are done and their outputs copied back, the state after the failing piece is
+ * undefined (reset it), and the copies already queued finish before cuda_stream
+ * passes the call. */
 lola_status lola_prefill_host(lola_state *st, const void *q, const void *k, const void *v, int64_t n_tokens,
                               void *out, void *staging, size_t staging_bytes, int64_t piece_tokens,
                               void *cuda_stream);
